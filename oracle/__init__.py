@@ -1,0 +1,21 @@
+"""fp64 CPU oracle for the Ideogram 4 DiT block hot path.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py``, never by the ``joint_attention_block_b200``
+package.  It shares no code with the CUDA path.
+"""
+from .ideogram4 import (  # noqa: F401
+    attention,
+    bf16_to_f64,
+    cond_proj_forward,
+    dequant,
+    dit_block_forward,
+    e4m3_to_f64,
+    euler_cfg_step,
+    gelu,
+    inv_freq,
+    mrope,
+    mrope_angles,
+    mrope_positions,
+    rmsnorm,
+)

@@ -1,0 +1,408 @@
+"""Pins for the fp64 oracle: page facts, closed forms, invariants, library routines, brute force.
+
+Each test ties the oracle to something other than itself, so that a dropped
+term, a flipped sign, a wrong index or a transposed operand fails one of them.
+"""
+import json
+import math
+import os
+from types import SimpleNamespace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from joint_attention_block_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_facts.json")
+
+
+def facts():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- e4m3 and dequant
+
+
+def test_e4m3_all_codes_match_torch_float8():
+    """All 256 codes against torch's own float8_e4m3fn decoder (a library routine)."""
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    fin = ~np.isnan(lib)
+    assert np.array_equal(ours[fin], lib[fin])
+    assert np.array_equal(np.signbit(ours[fin]), np.signbit(lib[fin]))
+
+
+def test_e4m3_range_and_structure():
+    v = oracle.e4m3_to_f64(np.arange(256, dtype=np.uint8))
+    fin = v[~np.isnan(v)]
+    assert np.isnan(v).sum() == 2 and np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert fin.max() == facts()["e4m3_max"]["value"] == -fin.min()
+    assert v[1] == 2.0 ** -9 and v[8] == 2.0 ** -6 and v[0x38] == 1.0
+    pos = v[:0x7F]
+    assert np.all(np.diff(pos) > 0), "positive codes must be strictly increasing"
+    assert np.array_equal(v[0x80:0xFF], -v[0:0x7F])
+
+
+def test_dequant_scale_is_per_output_row():
+    """weight_scale[:, None]: row i of the real weight is code row i times scale[i]."""
+    r = np.random.default_rng(0)
+    codes = r.integers(0, 256, size=(3, 5), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38
+    scale = np.array([0.5, 2.0, 0.125], dtype=np.float32)
+    w = oracle.dequant(codes, scale)
+    for i in range(3):
+        for j in range(5):
+            assert w[i, j] == float(torch.tensor([int(codes[i, j])], dtype=torch.uint8).view(torch.float8_e4m3fn).float()) * float(scale[i])
+    with pytest.raises(ValueError):
+        oracle.dequant(codes, np.ones(5, dtype=np.float32))
+
+
+def test_scale_in_epilogue_equals_scaled_weight():
+    """scale[n] * sum_k x_k w8[n,k] == sum_k x_k (w8[n,k] scale[n]) exactly on small dyadic inputs."""
+    r = np.random.default_rng(1)
+    codes = r.integers(0, 0x70, size=(6, 8), dtype=np.uint8)
+    scale = (2.0 ** r.integers(-6, 6, size=6)).astype(np.float32)
+    x = r.integers(-8, 8, size=(4, 8)).astype(np.float64)
+    lhs = (x @ oracle.e4m3_to_f64(codes).T) * scale.astype(np.float64)[None, :]
+    rhs = x @ oracle.dequant(codes, scale).T
+    assert np.array_equal(lhs, rhs)
+
+
+def test_synthetic_quantiser_hits_448_per_row():
+    codes, scale = synth.quantize_rows_e4m3(synth.normal(9, 0, (8, 64), std=0.02))
+    w = oracle.e4m3_to_f64(codes)
+    assert np.all(np.abs(w).max(axis=1) == 448.0)
+    assert scale.dtype == np.float32 and np.all(scale > 0)
+
+
+# ---------------------------------------------------------------- page arithmetic
+
+
+def test_conditioning_width_and_cache_sizes():
+    f = facts()
+    k = f["cond_layers"]["value"] * f["cond_hidden"]["value"]
+    assert k == f["cond_features_per_token"]["value"] == synth.COND.k
+    per_tok = k * 4 / 2 ** 20
+    assert round(per_tok, 3) == f["cond_raw_mib_per_token"]["value"]
+    assert round(per_tok * 512) == f["cond_raw_mib_512_tokens"]["value"]
+    # The projected size on the page is 512 tokens * 4608 bf16 values; the graded
+    # projection width is 4096 (4.0 MiB).  Both readings are recorded.
+    assert 512 * 4608 * 2 / 2 ** 20 == f["cond_projected_mib_512_tokens"]["value"]
+    assert 512 * synth.COND.d_out * 2 / 2 ** 20 == 4.0
+
+
+def test_shapes_follow_pages():
+    f = facts()
+    assert list(synth.C1024.rope_sections) == f["mrope_section"]["value"]
+    assert sum(synth.C1024.rope_sections) == synth.C1024.head_dim // 2
+    gh, gw, ch = f["latent_grid_1024"]["value"]
+    assert (synth.C1024.grid_h, synth.C1024.grid_w, synth.LATENT_CHANNELS) == (gh, gw, ch)
+    w = synth.block_inputs(synth.TINY)
+    assert w["w_qkv"].shape == (f["qkv_rows_per_hidden"]["value"] * synth.TINY.d_model, synth.TINY.d_model)
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+
+def test_rmsnorm_unit_rms_closed_form():
+    r = np.random.default_rng(2)
+    x = r.standard_normal((7, 33)) * 3.0
+    eps = 1e-6
+    y = oracle.rmsnorm(x, np.ones(33), eps)
+    ms = np.mean(x * x, axis=1)
+    assert np.allclose(np.mean(y * y, axis=1), ms / (ms + eps), rtol=1e-13, atol=0)
+
+
+def test_rmsnorm_scale_invariance_and_gain():
+    r = np.random.default_rng(3)
+    x = r.standard_normal((5, 16))
+    g = r.standard_normal(16)
+    y1 = oracle.rmsnorm(x, g, 0.0)
+    y2 = oracle.rmsnorm(7.5 * x, g, 0.0)
+    assert np.allclose(y1, y2, rtol=1e-13, atol=1e-15)
+    assert np.allclose(y1 / g, oracle.rmsnorm(x, np.ones(16), 0.0), rtol=1e-13)
+
+
+# ---------------------------------------------------------------- M-RoPE
+
+
+def test_positions_brute_force():
+    pos = oracle.mrope_positions(3, 2, 3)
+    want = [(0, 0, 0), (1, 1, 1), (2, 2, 2)]
+    for r in range(2):
+        for c in range(3):
+            want.append((3, r, c))
+    assert pos.tolist() == [list(p) for p in want]
+    assert oracle.mrope_positions(3, 2, 3, t_img=9)[3:, 0].tolist() == [9] * 6
+    assert oracle.mrope_positions(0, 1, 1).tolist() == [[0, 0, 0]]
+
+
+def test_inv_freq_fp32_values():
+    f = oracle.inv_freq(128, 10000.0)
+    assert f[0] == 1.0
+    assert f.dtype == np.float64 and np.all(f.astype(np.float32).astype(np.float64) == f)
+    assert abs(f[32] - 0.01) < 1e-9  # theta^(-64/128) = 1e-2
+
+
+def test_text_tokens_reduce_to_1d_rope_complex():
+    """Text token j at (j, j, j): every pair turns by j * inv_freq_i, whatever the sections.
+
+    Checked against the complex form z_i * exp(i j w_i), z_i = x_i + i x_{i+hd/2}.
+    """
+    hd, theta = 16, 10000.0
+    r = np.random.default_rng(4)
+    x = r.standard_normal((6, 2, hd))
+    pos = oracle.mrope_positions(6, 0, 0)
+    y = oracle.mrope(x, pos, (2, 3, 3), theta)
+    w = np.array([theta ** (-2 * i / hd) for i in range(hd // 2)], dtype=np.float32).astype(np.float64)
+    for j in range(6):
+        for h in range(2):
+            z = x[j, h, : hd // 2] + 1j * x[j, h, hd // 2 :]
+            zr = z * np.exp(1j * j * w)
+            assert np.allclose(y[j, h, : hd // 2], zr.real, atol=1e-12)
+            assert np.allclose(y[j, h, hd // 2 :], zr.imag, atol=1e-12)
+
+
+def test_mrope_sections_pick_their_axis():
+    """A token at (0, 1, 0) turns only the h-section pairs, each by inv_freq_i; (0,0,0) is the identity."""
+    hd, secs, theta = 16, (2, 3, 3), 100.0
+    x = np.random.default_rng(5).standard_normal((3, 1, hd))
+    pos = np.array([[0, 0, 0], [0, 1, 0], [0, 0, 2]])
+    y = oracle.mrope(x, pos, secs, theta)
+    assert np.array_equal(y[0], x[0])
+    f = oracle.inv_freq(hd, theta)
+    for tok, axis_pairs, p in ((1, range(2, 5), 1), (2, range(5, 8), 2)):
+        for i in range(hd // 2):
+            a, b = x[tok, 0, i], x[tok, 0, i + hd // 2]
+            ang = p * f[i] if i in axis_pairs else 0.0
+            assert math.isclose(y[tok, 0, i], a * math.cos(ang) - b * math.sin(ang), abs_tol=1e-13)
+            assert math.isclose(y[tok, 0, i + hd // 2], b * math.cos(ang) + a * math.sin(ang), abs_tol=1e-13)
+
+
+def test_mrope_norm_and_relative_invariance():
+    hd, secs = 32, (4, 6, 6)
+    r = np.random.default_rng(6)
+    q = r.standard_normal((1, 1, hd))
+    k = r.standard_normal((1, 1, hd))
+    p1, p2 = np.array([[3, 5, 7]]), np.array([[1, 2, 9]])
+    delta = np.array([[11, -4, 6]])
+    yq = oracle.mrope(q, p1, secs, 10000.0)
+    pairs = yq[0, 0, : hd // 2] ** 2 + yq[0, 0, hd // 2 :] ** 2
+    assert np.allclose(pairs, q[0, 0, : hd // 2] ** 2 + q[0, 0, hd // 2 :] ** 2, rtol=1e-13)
+    a = np.dot(oracle.mrope(q, p1, secs, 1e4).ravel(), oracle.mrope(k, p2, secs, 1e4).ravel())
+    b = np.dot(oracle.mrope(q, p1 + delta, secs, 1e4).ravel(), oracle.mrope(k, p2 + delta, secs, 1e4).ravel())
+    assert math.isclose(a, b, rel_tol=1e-10, abs_tol=1e-12)
+
+
+# ---------------------------------------------------------------- attention
+
+
+def _attention_loops(q, k, v):
+    Sq, H, hd = q.shape
+    out = np.zeros((Sq, H, v.shape[2]))
+    for h in range(H):
+        for i in range(Sq):
+            logits = [sum(q[i, h, c] * k[j, h, c] for c in range(hd)) / math.sqrt(hd) for j in range(k.shape[0])]
+            m = max(logits)
+            ws = [math.exp(l - m) for l in logits]
+            tot = sum(ws)
+            for c in range(v.shape[2]):
+                out[i, h, c] = sum(ws[j] * v[j, h, c] for j in range(k.shape[0])) / tot
+    return out
+
+
+def test_attention_brute_force():
+    r = np.random.default_rng(7)
+    q, k, v = (r.standard_normal((5, 2, 4)) for _ in range(3))
+    assert np.allclose(oracle.attention(q, k, v), _attention_loops(q, k, v), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_special_cases():
+    r = np.random.default_rng(8)
+    v = r.standard_normal((6, 1, 4))
+    q = r.standard_normal((3, 1, 4))
+    k_same = np.repeat(r.standard_normal((1, 1, 4)), 6, axis=0)
+    assert np.allclose(oracle.attention(q, k_same, v), v.mean(axis=0, keepdims=True).repeat(3, 0), atol=1e-13)
+    assert np.allclose(oracle.attention(q[:1], k_same[:1], v[:1]), v[:1], atol=1e-15)
+    k = np.zeros((6, 1, 4))
+    k[4, 0, 0] = 1e3
+    qd = np.zeros((1, 1, 4))
+    qd[0, 0, 0] = 1.0
+    assert np.allclose(oracle.attention(qd, k, v), v[4:5], atol=1e-12)
+
+
+def test_attention_permutation_equivariance():
+    """Bidirectional and unmasked: permuting the keys with their values changes nothing."""
+    r = np.random.default_rng(9)
+    q, k, v = (r.standard_normal((7, 2, 8)) for _ in range(3))
+    perm = r.permutation(7)
+    assert np.allclose(oracle.attention(q, k, v), oracle.attention(q, k[perm], v[perm]), atol=1e-13)
+    assert np.allclose(oracle.attention(q[perm], k, v), oracle.attention(q, k, v)[perm], atol=1e-13)
+
+
+# ---------------------------------------------------------------- GELU
+
+
+def test_gelu_against_math_erf_and_identities():
+    xs = np.linspace(-6, 6, 97)
+    lib = np.array([0.5 * x * (1 + math.erf(x / math.sqrt(2))) for x in xs])
+    assert np.allclose(oracle.gelu(xs), lib, rtol=1e-14, atol=1e-15)
+    assert oracle.gelu(np.array([0.0]))[0] == 0.0
+    assert np.allclose(oracle.gelu(xs) - oracle.gelu(-xs), xs, atol=1e-14)
+    assert np.max(np.abs(oracle.gelu(xs) - oracle.gelu(xs, tanh=True))) < 1e-3
+    t = torch.nn.functional.gelu(torch.from_numpy(xs), approximate="tanh").numpy()
+    assert np.allclose(oracle.gelu(xs, tanh=True), t, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- Euler / CFG
+
+
+def test_euler_cfg_closed_forms():
+    e = synth.euler_inputs(64)
+    x, vc, vu = e["x"], e["v_cond"], e["v_uncond"]
+    fc, fu = oracle.bf16_to_f64(vc), oracle.bf16_to_f64(vu)
+    dt = -1.0 / 50
+    assert np.allclose(oracle.euler_cfg_step(x, vc, vu, 1.0, dt), x + dt * fc, rtol=0, atol=1e-15)
+    assert np.allclose(oracle.euler_cfg_step(x, vc, vu, 0.0, dt), x + dt * fu, rtol=0, atol=1e-15)
+    assert np.allclose(oracle.euler_cfg_step(x, vc, vc, 4.0, dt), oracle.euler_cfg_step(x, vc, vc, -3.0, dt), atol=1e-15)
+    # The deep dive writes gw*v_c + (1-gw)*v_u; the same update as v_u + g*(v_c - v_u).
+    assert np.allclose(oracle.euler_cfg_step(x, vc, vu, 4.0, dt), x + dt * (fu + 4.0 * (fc - fu)), atol=1e-13)
+    assert np.allclose(oracle.euler_cfg_step(x, vc, vu, 4.0, 0.0), x, atol=0)
+
+
+# ---------------------------------------------------------------- block and cond
+
+
+def _tiny_cfg(**kw):
+    base = dict(d_model=8, n_heads=2, head_dim=4, d_mlp=16, rope_sections=(1, 0, 1), rope_theta=10000.0, eps=1e-6, gelu_tanh=0)
+    base.update(kw)
+    return SimpleNamespace(**base)
+
+
+def _tiny_weights(cfg, seed=10):
+    r = np.random.default_rng(seed)
+    d, f, hd = cfg.d_model, cfg.d_mlp, cfg.head_dim
+    w = {}
+    for name, shape in (("w_qkv", (3 * d, d)), ("w_o", (d, d)), ("w_up", (f, d)), ("w_down", (d, f))):
+        codes, scale = synth.quantize_rows_e4m3(r.standard_normal(shape).astype(np.float32) * 0.3)
+        w[name], w["s_" + name[2:]] = codes, scale
+    for name, n in (("g_norm1", d), ("g_norm2", d), ("g_q", hd), ("g_k", hd)):
+        w[name] = synth.to_bf16_bits(1.0 + 0.1 * r.standard_normal(n))
+    return w
+
+
+def _block_loops(cfg, w, x, n_text, gh, gw):
+    """Whole block as explicit Python loops over tokens, heads and channels."""
+    d, H, hd, F, eps = cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.d_mlp, cfg.eps
+    S = n_text + gh * gw
+    dq = lambda name: oracle.dequant(w["w_" + name], w["s_" + name])  # noqa: E731
+    Wqkv, Wo, Wup, Wdn = dq("qkv"), dq("o"), dq("up"), dq("down")
+    g1, g2 = oracle.bf16_to_f64(w["g_norm1"]), oracle.bf16_to_f64(w["g_norm2"])
+    gq, gk = oracle.bf16_to_f64(w["g_q"]), oracle.bf16_to_f64(w["g_k"])
+
+    def norm(vec, g):
+        ms = sum(t * t for t in vec) / len(vec)
+        return [vec[i] / math.sqrt(ms + eps) * g[i] for i in range(len(vec))]
+
+    def pos_of(s):
+        if s < n_text:
+            return (s, s, s)
+        r, c = divmod(s - n_text, gw)
+        return (n_text, r, c)
+
+    secs = cfg.rope_sections
+
+    def rot(vec, p):
+        out = list(vec)
+        for i in range(hd // 2):
+            axis = 0 if i < secs[0] else (1 if i < secs[0] + secs[1] else 2)
+            ang = p[axis] * float(np.float32(cfg.rope_theta ** (-2.0 * i / hd)))
+            a, b = vec[i], vec[i + hd // 2]
+            out[i] = a * math.cos(ang) - b * math.sin(ang)
+            out[i + hd // 2] = b * math.cos(ang) + a * math.sin(ang)
+        return out
+
+    hs = [norm(list(x[s]), g1) for s in range(S)]
+    qkv = [[sum(hs[s][c] * Wqkv[o, c] for c in range(d)) for o in range(3 * d)] for s in range(S)]
+    Q = [[rot(norm(qkv[s][h * hd:(h + 1) * hd], gq), pos_of(s)) for h in range(H)] for s in range(S)]
+    K = [[rot(norm(qkv[s][d + h * hd:d + (h + 1) * hd], gk), pos_of(s)) for h in range(H)] for s in range(S)]
+    V = [[qkv[s][2 * d + h * hd:2 * d + (h + 1) * hd] for h in range(H)] for s in range(S)]
+    y = np.zeros((S, d))
+    for s in range(S):
+        o = []
+        for h in range(H):
+            logits = [sum(Q[s][h][c] * K[t][h][c] for c in range(hd)) / math.sqrt(hd) for t in range(S)]
+            m = max(logits)
+            ws = [math.exp(l - m) for l in logits]
+            o += [sum(ws[t] * V[t][h][c] for t in range(S)) / sum(ws) for c in range(hd)]
+        x1 = [x[s][c] + sum(o[i] * Wo[c, i] for i in range(d)) for c in range(d)]
+        h2 = norm(x1, g2)
+        u = [0.5 * a * (1 + math.erf(a / math.sqrt(2))) for a in (sum(h2[c] * Wup[j, c] for c in range(d)) for j in range(F))]
+        y[s] = [x1[c] + sum(u[j] * Wdn[c, j] for j in range(F)) for c in range(d)]
+    return y
+
+
+def test_block_brute_force_tiny():
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg)
+    r = np.random.default_rng(11)
+    n_text, gh, gw = 2, 2, 2
+    x_bits = synth.to_bf16_bits(r.standard_normal((1, n_text + gh * gw, cfg.d_model)))
+    got = oracle.dit_block_forward(cfg, w, x_bits, n_text, gh, gw)[0]
+    want = _block_loops(cfg, w, oracle.bf16_to_f64(x_bits)[0], n_text, gh, gw)
+    assert np.allclose(got, want, rtol=1e-11, atol=1e-11)
+
+
+def test_block_residual_special_cases():
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg)
+    r = np.random.default_rng(12)
+    x_bits = synth.to_bf16_bits(r.standard_normal((1, 6, cfg.d_model)))
+    x = oracle.bf16_to_f64(x_bits)
+    z = dict(w)
+    z["w_o"] = np.zeros_like(w["w_o"])
+    z["w_down"] = np.zeros_like(w["w_down"])
+    assert np.array_equal(oracle.dit_block_forward(cfg, z, x_bits, 2, 2, 2), x)
+    z = dict(w)
+    z["w_up"] = np.zeros_like(w["w_up"])
+    full = oracle.dit_block_forward(cfg, w, x_bits, 2, 2, 2)
+    attn_only = oracle.dit_block_forward(cfg, z, x_bits, 2, 2, 2)
+    assert not np.allclose(full, attn_only)
+    z2 = dict(z)
+    z2["w_o"] = np.zeros_like(w["w_o"])
+    assert np.array_equal(oracle.dit_block_forward(cfg, z2, x_bits, 2, 2, 2), x)
+
+
+def test_block_sampled_rows_match_full():
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg)
+    x_bits = synth.to_bf16_bits(np.random.default_rng(13).standard_normal((2, 7, cfg.d_model)))
+    full = oracle.dit_block_forward(cfg, w, x_bits, 3, 2, 2)
+    rows = np.array([6, 0, 3])
+    part = oracle.dit_block_forward(cfg, w, x_bits, 3, 2, 2, rows=rows)
+    assert np.allclose(part, full[:, rows], rtol=1e-13, atol=1e-13)
+
+
+def test_cond_proj_identity_weight():
+    """Unit gain and an identity weight (code 0x38 = 1.0 on the diagonal): output = normalised features."""
+    r = np.random.default_rng(14)
+    feats = synth.to_bf16_bits(r.standard_normal((4, 12)))
+    g = synth.to_bf16_bits(np.ones(12))
+    codes = np.zeros((5, 12), dtype=np.uint8)
+    codes[np.arange(5), np.arange(5)] = 0x38
+    out = oracle.cond_proj_forward(feats, g, 1e-6, codes, np.full(5, 2.0, dtype=np.float32))
+    f = oracle.bf16_to_f64(feats)
+    norm = f / np.sqrt(np.mean(f * f, axis=1, keepdims=True) + 1e-6)
+    assert np.allclose(out, 2.0 * norm[:, :5], rtol=1e-14)
+
+
+def test_block_flop_count():
+    s = synth.C1024
+    assert s.seq == 4608
+    assert abs(s.flops() - 2.203e12) / 2.203e12 < 1e-3
+    assert abs(synth.UNCOND1024.flops() - 1.941e12) / 1.941e12 < 1e-3
