@@ -1,0 +1,168 @@
+/*
+ * jab_dit.h -- C ABI of the B200 (sm_100a) Ideogram 4 single-stream DiT block hot path.
+ *
+ * The three calls of the hot path:
+ *   dit_block_forward   one single-stream DiT block over the joint [text; image] sequence
+ *   cond_proj_forward   the frozen llm_cond_norm / llm_cond_proj projection of the
+ *                       13 concatenated 4096-wide text-encoder hidden states
+ *   euler_cfg_step      dual-branch classifier-free guidance + one flow-matching Euler step
+ * and the per-step kernels they are built from, exposed for parity testing.
+ *
+ * Conventions (all calls):
+ *   - Every pointer is caller-owned DEVICE memory unless stated otherwise; the library
+ *     allocates nothing per call.  Scratch comes from the caller's workspace.
+ *   - bf16 data is passed as raw 16-bit patterns (uint16_t / void*), e4m3 as bytes.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on it; the return code covers synchronous argument validation and
+ *     launch errors only.  Device-side failures (a bounded wait that timed out) are
+ *     reported by dit_poll_error().
+ *   - Pointers must be 16-byte aligned; tensors are dense row-major.
+ *   - Each call runs on the CUDA device current on the calling thread.
+ */
+#ifndef JAB_DIT_H
+#define JAB_DIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DIT_API __attribute__((visibility("default")))
+#else
+#define DIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DIT_OK = 0,
+  DIT_ERR_INVALID_ARG = 1, /* null / misaligned pointer, inconsistent sizes */
+  DIT_ERR_UNSUPPORTED = 2, /* a size this build does not handle (see each call) */
+  DIT_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_bytes() */
+  DIT_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  DIT_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up (from dit_poll_error) */
+  DIT_ERR_DEVICE = 6       /* another device-side error was recorded (from dit_poll_error) */
+} dit_status;
+
+/* Shape and numerics of one block.
+ * rope_sections: rotary PAIRS per axis (t, h, w), laid out contiguously over the
+ *   first head_dim/2 frequencies; must sum to head_dim/2.  The Ideogram 4 deep dive,
+ *   section 6-3 ("3D MRoPE"), gives mrope_section = (24, 20, 20) for head_dim 128.
+ * rope_theta: RoPE base (10000 by default); inv_freq_i = fp32(theta^(-2i/head_dim)).
+ * eps: RMSNorm epsilon of every norm in the block.
+ * gelu_tanh: 0 = exact erf GELU, 1 = tanh approximation.
+ * Supported: d_model = n_heads * head_dim, head_dim in {64, 128}, d_model and d_mlp
+ * multiples of 256. */
+typedef struct {
+  int32_t d_model, n_heads, head_dim, d_mlp;
+  int32_t rope_sections[3];
+  float rope_theta, eps;
+  int32_t gelu_tanh;
+} dit_block_config;
+
+/* FP8 weights of one block, as the Ideogram 4 FP8 checkpoint stores them
+ * (unsloth diffusion_ideogram4.py commit log, fp8 loader commit): e4m3 bytes
+ * [out, in] row-major with a per-output-row fp32 weight_scale [out]; the real weight
+ * is fp8 * weight_scale[:, None].  w_qkv is the fused attention.qkv.weight [3d, d]
+ * with Q, K, V rows stacked in that order; w_o is attention.o.weight [d, d];
+ * w_up [d_mlp, d], w_down [d, d_mlp] are the FeedForward projections.
+ * Gains are bf16: g_norm1, g_norm2 [d] (the two pre-norms), g_q, g_k [head_dim]
+ * (QK-RMSNorm, shared by all heads). */
+typedef struct {
+  const uint8_t *w_qkv, *w_o, *w_up, *w_down;
+  const float *s_qkv, *s_o, *s_up, *s_down;
+  const void *g_norm1, *g_norm2, *g_q, *g_k;
+} dit_block_weights;
+
+/* Bytes of device workspace dit_block_forward needs for this shape (256-byte aligned). */
+DIT_API size_t dit_block_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w);
+
+/* One single-stream DiT block forward (Ideogram 4.0 announcement thread: self-attention,
+ * QK-RMSNorm and 3D multimodal RoPE over one sequence of text and image tokens; deep dive
+ * section 4-2: text and image tokens concatenated through the same self-attention):
+ *   h  = RMSNorm(x; g_norm1)
+ *   q,k,v = split(h W_qkv^T);  q,k = MRoPE(RMSNorm_head(q; g_q)), MRoPE(RMSNorm_head(k; g_k))
+ *   x1 = x + Attn(q, k, v) W_o^T          (bidirectional, softmax scale 1/sqrt(head_dim))
+ *   y  = x1 + GELU(RMSNorm(x1; g_norm2) W_up^T) W_down^T
+ * x_in: bf16 [batch, n_text + grid_h*grid_w, d_model], text rows first, image rows in
+ *   raster order (r*grid_w + c).
+ * x_out: bf16, same shape; must not alias x_in.
+ * t_img: temporal position of the image tokens (< 0 => n_text).  Text token j sits at
+ *   (j, j, j); image cell (r, c) at (t_img, r, c).
+ * pos: optional int32 [S, 3] (t, h, w) per token overriding the rule above; NULL to derive.
+ * workspace: >= dit_block_workspace_bytes() bytes, 256-byte aligned.
+ * Errors: INVALID_ARG (null/misaligned/aliasing), UNSUPPORTED (shape rules above),
+ *   WORKSPACE, CUDA. */
+DIT_API int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in, void* x_out,
+                      int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace cond_proj_forward needs. */
+DIT_API size_t cond_proj_workspace_bytes(int n_tok, int n_layers, int hidden, int d_out);
+
+/* llm_cond_norm + llm_cond_proj (SimpleTuner Ideogram 4 quickstart, "Text Embed Cache"):
+ *   out = RMSNorm(feats; g_norm, eps) (scale (.) W8)^T
+ * feats: bf16 [n_tok, n_layers*hidden] (13 x 4096 = 53,248 for Ideogram 4);
+ * g_norm: bf16 [n_layers*hidden]; w: e4m3 [d_out, n_layers*hidden]; scale: fp32 [d_out];
+ * out: bf16 [n_tok, d_out].  n_layers*hidden and d_out must be multiples of 256. */
+DIT_API int cond_proj_forward(const void* feats, int n_tok, int n_layers, int hidden, const void* g_norm, float eps,
+                      const uint8_t* w, const float* scale, int d_out, void* out, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/* Dual-branch CFG + Euler (Ideogram 4 deep dive, section 4-6 pseudocode):
+ *   v = v_uncond + guidance * (v_cond - v_uncond)   (= gw*v_cond + (1-gw)*v_uncond)
+ *   x = x + dt * v                                  (dt = s - t < 0 from t=1 to 0)
+ * x: fp32 [n], updated in place; v_cond, v_uncond: bf16 [n].  Arithmetic is fp32:
+ * d = v_c - v_u; v = fma(guidance, d, v_u); x = fma(dt, v, x). */
+DIT_API int euler_cfg_step(float* x, const void* v_cond, const void* v_uncond, int64_t n, float guidance, float dt,
+                   void* stream);
+
+/* ---- per-step kernels (the block is composed of these; exposed for parity tests) ---- */
+
+/* e4m3 bytes -> bf16 [n], exact for every finite code (the FP8 dequant the GEMMs use
+ * on chip, before the per-row scale). */
+DIT_API int dit_e4m3_to_bf16(const uint8_t* codes, void* out, int64_t n, void* stream);
+
+/* Row RMSNorm with gain: y = x / sqrt(mean(x^2) + eps) * g, bf16 in/out, fp32 math.
+ * x, y: [rows, cols] (may alias); g: [cols].  cols % 8 == 0. */
+DIT_API int dit_rmsnorm_rows(const void* x, const void* g, void* y, int64_t rows, int64_t cols, float eps, void* stream);
+
+/* The (t, h, w) int32 [S, 3] positions the block uses for this sequence (see dit_block_forward). */
+DIT_API int dit_mrope_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos_out, void* stream);
+
+/* Y[M, N] = epilogue( A[M, K] (W8[N, K])^T * scale[N] ).  A bf16 row-major, W8 e4m3
+ * row-major, scale fp32.  epilogue: 0 = none, 1 = GELU (gelu_tanh selects the form),
+ * 2 = + residual R[M, N] (bf16).  Y bf16 [M, N].  N % 32 == 0, K % 16 == 0. */
+DIT_API int dit_gemm_w8a16(const void* a, const uint8_t* w8, const float* scale, void* y, const void* residual, int M,
+                   int N, int K, int epilogue, int gelu_tanh, void* stream);
+
+/* Per-head QK-RMSNorm + 3D M-RoPE, in place on a fused qkv buffer bf16 [batch, S, 3d]
+ * (Q columns [0, d), K columns [d, 2d); V untouched).  pos: int32 [S, 3] or NULL
+ * (derived from n_text/grid/t_img as in dit_block_forward). */
+DIT_API int dit_qknorm_mrope(void* qkv, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
+                     const dit_block_config* cfg, const void* g_q, const void* g_k, void* workspace,
+                     size_t ws_bytes, void* stream);
+
+/* Joint bidirectional attention: out[b, s, h*hd:(h+1)*hd] = softmax(q k^T / sqrt(hd)) v
+ * over all S tokens, per head, reading q, k, v from a fused qkv buffer bf16 [batch, S, 3d].
+ * out: bf16 [batch, S, d]. */
+DIT_API int dit_joint_attention(const void* qkv, void* out, int batch, int seq, int n_heads, int head_dim, void* stream);
+
+/* Synchronise `stream`, then report (and clear) device-side errors recorded by any
+ * kernel of this library on the current device since the last poll. */
+DIT_API int dit_poll_error(void* stream);
+
+/* Set the wall-time limit of every device-side bounded wait (default 2000 ms). */
+DIT_API int dit_set_wait_timeout_ms(uint32_t ms);
+
+DIT_API const char* dit_status_str(int status);
+
+/* ABI version of this header (bumped on any signature change). */
+DIT_API int dit_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JAB_DIT_H */

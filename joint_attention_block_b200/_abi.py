@@ -1,0 +1,213 @@
+"""ctypes binding of the C ABI in ``include/jab_dit.h``.
+
+Argument marshalling only: every step runs in the CUDA library.  Device tensors
+are passed as raw pointers (``tensor.data_ptr()``) together with the current
+torch CUDA stream.  There is no fallback: if the library is missing the import
+fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libjab_b200.so")
+
+DIT_OK = 0
+STATUS_NAMES = {
+    0: "DIT_OK",
+    1: "DIT_ERR_INVALID_ARG",
+    2: "DIT_ERR_UNSUPPORTED",
+    3: "DIT_ERR_WORKSPACE",
+    4: "DIT_ERR_CUDA",
+    5: "DIT_ERR_TIMEOUT",
+    6: "DIT_ERR_DEVICE",
+}
+
+
+class DitError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} ({lib().dit_status_str(status).decode()})")
+
+
+class BlockConfig(ctypes.Structure):
+    _fields_ = [
+        ("d_model", ctypes.c_int32),
+        ("n_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("d_mlp", ctypes.c_int32),
+        ("rope_sections", ctypes.c_int32 * 3),
+        ("rope_theta", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("gelu_tanh", ctypes.c_int32),
+    ]
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_qkv", "w_o", "w_up", "w_down", "s_qkv", "s_o", "s_up", "s_down",
+                                                "g_norm1", "g_norm2", "g_q", "g_k")]
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+SIGNATURES = {
+    "dit_block_workspace_bytes": (_SZ, [ctypes.POINTER(BlockConfig), _I, _I, _I, _I]),
+    "dit_block_forward": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I, _I, _I, _I,
+                               _P, _P, _SZ, _P]),
+    "cond_proj_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "cond_proj_forward": (_I, [_P, _I, _I, _I, _P, _F, _P, _P, _I, _P, _P, _SZ, _P]),
+    "euler_cfg_step": (_I, [_P, _P, _P, _I64, _F, _F, _P]),
+    "dit_e4m3_to_bf16": (_I, [_P, _P, _I64, _P]),
+    "dit_rmsnorm_rows": (_I, [_P, _P, _P, _I64, _I64, _F, _P]),
+    "dit_mrope_positions": (_I, [_I, _I, _I, _I, _P, _P]),
+    "dit_gemm_w8a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dit_qknorm_mrope": (_I, [_P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(BlockConfig), _P, _P, _P, _SZ, _P]),
+    "dit_joint_attention": (_I, [_P, _P, _I, _I, _I, _I, _P]),
+    "dit_poll_error": (_I, [_P]),
+    "dit_set_wait_timeout_ms": (_I, [ctypes.c_uint32]),
+    "dit_status_str": (ctypes.c_char_p, [_I]),
+    "dit_abi_version": (_I, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m joint_attention_block_b200.build` "
+                "(there is no CPU fallback)"
+            )
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the C ABI must be contiguous")
+    return t.data_ptr()
+
+
+def _check(name: str, status: int) -> None:
+    if status != DIT_OK:
+        raise DitError(name, status)
+
+
+def make_config(shape) -> BlockConfig:
+    c = BlockConfig()
+    c.d_model, c.n_heads, c.head_dim, c.d_mlp = shape.d_model, shape.n_heads, shape.head_dim, shape.d_mlp
+    for i in range(3):
+        c.rope_sections[i] = int(shape.rope_sections[i])
+    c.rope_theta, c.eps, c.gelu_tanh = float(shape.rope_theta), float(shape.eps), int(shape.gelu_tanh)
+    return c
+
+
+def make_weights(w) -> BlockWeights:
+    """``w``: dict of device tensors named like the struct fields."""
+    bw = BlockWeights()
+    for name, _ in BlockWeights._fields_:
+        setattr(bw, name, _ptr(w[name]))
+    return bw
+
+
+# ---------------------------------------------------------------- the three calls
+
+
+def block_workspace_bytes(cfg: BlockConfig, batch: int, n_text: int, grid_h: int, grid_w: int) -> int:
+    return int(lib().dit_block_workspace_bytes(ctypes.byref(cfg), batch, n_text, grid_h, grid_w))
+
+
+def dit_block_forward(cfg: BlockConfig, weights: BlockWeights, x: torch.Tensor, out: torch.Tensor, n_text: int,
+                      grid_h: int, grid_w: int, workspace: torch.Tensor, t_img: int = -1,
+                      pos: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check("dit_block_forward", lib().dit_block_forward(
+        ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
+        _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def cond_proj_workspace_bytes(n_tok: int, n_layers: int, hidden: int, d_out: int) -> int:
+    return int(lib().cond_proj_workspace_bytes(n_tok, n_layers, hidden, d_out))
+
+
+def cond_proj_forward(feats: torch.Tensor, n_layers: int, hidden: int, g: torch.Tensor, eps: float, w: torch.Tensor,
+                      scale: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    _check("cond_proj_forward", lib().cond_proj_forward(
+        _ptr(feats), feats.shape[0], n_layers, hidden, _ptr(g), eps, _ptr(w), _ptr(scale), out.shape[1], _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def euler_cfg_step(x: torch.Tensor, v_cond: torch.Tensor, v_uncond: torch.Tensor, guidance: float, dt: float,
+                   stream=None) -> None:
+    _check("euler_cfg_step", lib().euler_cfg_step(_ptr(x), _ptr(v_cond), _ptr(v_uncond), x.numel(), guidance, dt,
+                                                  _stream(stream)))
+
+
+# ---------------------------------------------------------------- per-step kernels
+
+
+def e4m3_to_bf16(codes: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    _check("dit_e4m3_to_bf16", lib().dit_e4m3_to_bf16(_ptr(codes), _ptr(out), codes.numel(), _stream(stream)))
+
+
+def rmsnorm_rows(x: torch.Tensor, g: torch.Tensor, y: torch.Tensor, eps: float, stream=None) -> None:
+    cols = x.shape[-1]
+    _check("dit_rmsnorm_rows", lib().dit_rmsnorm_rows(_ptr(x), _ptr(g), _ptr(y), x.numel() // cols, cols, eps,
+                                                      _stream(stream)))
+
+
+def mrope_positions(n_text: int, grid_h: int, grid_w: int, t_img: int, out: torch.Tensor, stream=None) -> None:
+    _check("dit_mrope_positions", lib().dit_mrope_positions(n_text, grid_h, grid_w, t_img, _ptr(out),
+                                                            _stream(stream)))
+
+
+def gemm_w8a16(a: torch.Tensor, w8: torch.Tensor, scale: torch.Tensor, y: torch.Tensor,
+               residual: Optional[torch.Tensor] = None, epilogue: int = 0, gelu_tanh: int = 0, stream=None) -> None:
+    M, K = a.shape
+    N = w8.shape[0]
+    _check("dit_gemm_w8a16", lib().dit_gemm_w8a16(_ptr(a), _ptr(w8), _ptr(scale), _ptr(y), _ptr(residual), M, N, K,
+                                                  epilogue, gelu_tanh, _stream(stream)))
+
+
+def qknorm_mrope(qkv: torch.Tensor, cfg: BlockConfig, n_text: int, grid_h: int, grid_w: int, g_q: torch.Tensor,
+                 g_k: torch.Tensor, workspace: torch.Tensor, t_img: int = -1, pos: Optional[torch.Tensor] = None,
+                 stream=None) -> None:
+    _check("dit_qknorm_mrope", lib().dit_qknorm_mrope(
+        _ptr(qkv), qkv.shape[0], n_text, grid_h, grid_w, t_img, _ptr(pos), ctypes.byref(cfg), _ptr(g_q), _ptr(g_k),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def joint_attention(qkv: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int, stream=None) -> None:
+    _check("dit_joint_attention", lib().dit_joint_attention(_ptr(qkv), _ptr(out), qkv.shape[0], qkv.shape[1], n_heads,
+                                                            head_dim, _stream(stream)))
+
+
+def poll_error(stream=None) -> int:
+    return int(lib().dit_poll_error(_stream(stream)))
+
+
+def set_wait_timeout_ms(ms: int) -> None:
+    _check("dit_set_wait_timeout_ms", lib().dit_set_wait_timeout_ms(ms))

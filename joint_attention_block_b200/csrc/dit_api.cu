@@ -1,0 +1,335 @@
+// The C ABI: argument validation, workspace carving and the composition of the
+// block forward, the conditioning projection and the CFG/Euler step from the
+// kernels in the other translation units.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/jab_dit.h"
+#include "internal.h"
+
+namespace jab {
+
+// ------------------------------------------------------------------ device error word
+
+// One word per device: the first device-side error recorded since the last poll.
+__device__ uint32_t g_device_error;
+
+static std::atomic<uint64_t> g_timeout_ns{2000ull * 1000ull * 1000ull};
+static std::mutex g_mu;
+static uint32_t* g_err_ptr[64] = {nullptr};
+
+cudaError_t current_guard(KernelGuard* g) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return e;
+    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  g->err = g_err_ptr[dev];
+  g->timeout_ns = g_timeout_ns.load();
+  return cudaSuccess;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint64_t gdim[3], gstr[2];
+  cuuint32_t bdim[3];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
+  CUresult r = fn(map, dtype, static_cast<cuuint32_t>(rank), base, gdim, gstr, bdim, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace jab
+
+using namespace jab;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA; }
+
+int check_config(const dit_block_config* c) {
+  if (c == nullptr) return DIT_ERR_INVALID_ARG;
+  if (c->n_heads <= 0 || c->head_dim <= 0 || c->d_model != c->n_heads * c->head_dim) return DIT_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return DIT_ERR_UNSUPPORTED;
+  if (c->d_model % 256 != 0 || c->d_mlp <= 0 || c->d_mlp % 256 != 0) return DIT_ERR_UNSUPPORTED;
+  if (c->rope_sections[0] < 0 || c->rope_sections[1] < 0 || c->rope_sections[2] < 0) return DIT_ERR_INVALID_ARG;
+  if (c->rope_sections[0] + c->rope_sections[1] + c->rope_sections[2] != c->head_dim / 2) return DIT_ERR_INVALID_ARG;
+  if (!(c->rope_theta > 0.f) || !(c->eps >= 0.f)) return DIT_ERR_INVALID_ARG;
+  return DIT_OK;
+}
+
+struct BlockWorkspace {
+  float* cos_tab;
+  float* sin_tab;
+  uint16_t* h;
+  uint16_t* qkv;
+  uint16_t* o;
+  uint16_t* x1;
+  uint16_t* u;
+  size_t bytes;
+};
+
+BlockWorkspace carve_block(const dit_block_config* c, int batch, int seq, void* base) {
+  BlockWorkspace w{};
+  const size_t M = static_cast<size_t>(batch) * seq;
+  const size_t d = c->d_model, F = c->d_mlp, half = c->head_dim / 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t o_cos = take(seq * half * 4), o_sin = take(seq * half * 4);
+  const size_t o_h = take(M * d * 2), o_qkv = take(M * 3 * d * 2), o_o = take(M * d * 2), o_x1 = take(M * d * 2);
+  const size_t o_u = take(M * F * 2);
+  w.bytes = off;
+  if (base != nullptr) {
+    uint8_t* b = static_cast<uint8_t*>(base);
+    w.cos_tab = reinterpret_cast<float*>(b + o_cos);
+    w.sin_tab = reinterpret_cast<float*>(b + o_sin);
+    w.h = reinterpret_cast<uint16_t*>(b + o_h);
+    w.qkv = reinterpret_cast<uint16_t*>(b + o_qkv);
+    w.o = reinterpret_cast<uint16_t*>(b + o_o);
+    w.x1 = reinterpret_cast<uint16_t*>(b + o_x1);
+    w.u = reinterpret_cast<uint16_t*>(b + o_u);
+  }
+  return w;
+}
+
+bool shape_ok(int batch, int n_text, int grid_h, int grid_w) {
+  if (batch <= 0 || n_text < 0 || grid_h < 0 || grid_w < 0) return false;
+  const int64_t S = static_cast<int64_t>(n_text) + static_cast<int64_t>(grid_h) * grid_w;
+  return S > 0 && S * batch < (1ll << 31) / 16;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dit_abi_version(void) { return 1; }
+
+const char* dit_status_str(int s) {
+  switch (s) {
+    case DIT_OK: return "ok";
+    case DIT_ERR_INVALID_ARG: return "invalid argument";
+    case DIT_ERR_UNSUPPORTED: return "unsupported size";
+    case DIT_ERR_WORKSPACE: return "workspace missing or too small";
+    case DIT_ERR_CUDA: return "CUDA error";
+    case DIT_ERR_TIMEOUT: return "device-side bounded wait timed out";
+    case DIT_ERR_DEVICE: return "device-side error";
+    default: return "unknown status";
+  }
+}
+
+int dit_set_wait_timeout_ms(uint32_t ms) {
+  if (ms == 0) return DIT_ERR_INVALID_ARG;
+  g_timeout_ns.store(static_cast<uint64_t>(ms) * 1000000ull);
+  return DIT_OK;
+}
+
+int dit_poll_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return DIT_ERR_CUDA;
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return DIT_ERR_CUDA;
+  if (v == 0) return DIT_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return DIT_ERR_CUDA;
+  return (v & 0xF00u) == 0x100u ? DIT_ERR_TIMEOUT : DIT_ERR_DEVICE;
+}
+
+int dit_e4m3_to_bf16(const uint8_t* codes, void* out, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (codes == nullptr || out == nullptr))) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(out)) return DIT_ERR_INVALID_ARG;
+  return from_cuda(launch_e4m3_to_bf16(codes, static_cast<uint16_t*>(out), n, as_stream(stream)));
+}
+
+int dit_rmsnorm_rows(const void* x, const void* g, void* y, int64_t rows, int64_t cols, float eps, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 8 != 0 || rows > (1ll << 31) - 1) return DIT_ERR_INVALID_ARG;
+  if (rows > 0 && (x == nullptr || g == nullptr || y == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(g) || !aligned16(y)) return DIT_ERR_INVALID_ARG;
+  return from_cuda(launch_rmsnorm(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g),
+                                  static_cast<uint16_t*>(y), rows, cols, eps, as_stream(stream)));
+}
+
+int euler_cfg_step(float* x, const void* v_cond, const void* v_uncond, int64_t n, float guidance, float dt,
+                   void* stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || v_cond == nullptr || v_uncond == nullptr))) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(v_cond) || !aligned16(v_uncond)) return DIT_ERR_INVALID_ARG;
+  return from_cuda(launch_euler_cfg(x, static_cast<const uint16_t*>(v_cond), static_cast<const uint16_t*>(v_uncond),
+                                    n, guidance, dt, as_stream(stream)));
+}
+
+int dit_mrope_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos_out, void* stream) {
+  if (!shape_ok(1, n_text, grid_h, grid_w) || pos_out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (t_img < 0) t_img = n_text;
+  return from_cuda(launch_positions(n_text, grid_h, grid_w, t_img, pos_out, as_stream(stream)));
+}
+
+int dit_gemm_w8a16(const void* a, const uint8_t* w8, const float* scale, void* y, const void* residual, int M, int N,
+                   int K, int epilogue, int gelu_tanh, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0) return DIT_ERR_INVALID_ARG;
+  if (N % 32 != 0 || K % 16 != 0) return DIT_ERR_UNSUPPORTED;
+  if (epilogue < 0 || epilogue > 2) return DIT_ERR_INVALID_ARG;
+  if (M == 0) return DIT_OK;
+  if (a == nullptr || w8 == nullptr || scale == nullptr || y == nullptr) return DIT_ERR_INVALID_ARG;
+  if (epilogue == EPI_RESIDUAL && residual == nullptr) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w8) || !aligned16(y) || !aligned16(residual)) return DIT_ERR_INVALID_ARG;
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  GemmArgs args{static_cast<const uint16_t*>(a), w8, scale, static_cast<uint16_t*>(y),
+                static_cast<const uint16_t*>(residual), M, N, K, epilogue, gelu_tanh};
+  return from_cuda(launch_gemm_w8a16(args, g, as_stream(stream)));
+}
+
+int dit_qknorm_mrope(void* qkv, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
+                     const dit_block_config* cfg, const void* g_q, const void* g_k, void* workspace, size_t ws_bytes,
+                     void* stream) {
+  int st = check_config(cfg);
+  if (st != DIT_OK) return st;
+  if (!shape_ok(batch, n_text, grid_h, grid_w) || qkv == nullptr || g_q == nullptr || g_k == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  const int S = n_text + grid_h * grid_w;
+  const size_t need = 2 * align256(static_cast<size_t>(S) * (cfg->head_dim / 2) * 4);
+  if (workspace == nullptr || ws_bytes < need) return DIT_ERR_WORKSPACE;
+  float* cos_tab = static_cast<float*>(workspace);
+  float* sin_tab = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + need / 2);
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections,
+                                    cfg->rope_theta, cos_tab, sin_tab, s);
+  if (e != cudaSuccess) return DIT_ERR_CUDA;
+  return from_cuda(launch_qknorm_mrope(static_cast<uint16_t*>(qkv), batch, S, cfg->n_heads, cfg->head_dim, cos_tab,
+                                       sin_tab, static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k),
+                                       cfg->eps, s));
+}
+
+int dit_joint_attention(const void* qkv, void* out, int batch, int seq, int n_heads, int head_dim, void* stream) {
+  if (batch <= 0 || seq <= 0 || n_heads <= 0 || qkv == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return DIT_ERR_UNSUPPORTED;
+  if (!aligned16(qkv) || !aligned16(out)) return DIT_ERR_INVALID_ARG;
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  return from_cuda(launch_attention(static_cast<const uint16_t*>(qkv), static_cast<uint16_t*>(out), batch, seq,
+                                    n_heads, head_dim, g, as_stream(stream)));
+}
+
+size_t dit_block_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w) {
+  if (check_config(cfg) != DIT_OK || !shape_ok(batch, n_text, grid_h, grid_w)) return 0;
+  return carve_block(cfg, batch, n_text + grid_h * grid_w, nullptr).bytes;
+}
+
+int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in, void* x_out,
+                      int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  int st = check_config(cfg);
+  if (st != DIT_OK) return st;
+  if (w == nullptr || x_in == nullptr || x_out == nullptr || x_in == x_out) return DIT_ERR_INVALID_ARG;
+  if (!shape_ok(batch, n_text, grid_h, grid_w)) return DIT_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->w_qkv, w->w_o, w->w_up, w->w_down, w->s_qkv, w->s_o, w->s_up, w->s_down, w->g_norm1,
+                        w->g_norm2, w->g_q, w->g_k};
+  for (const void* p : ptrs)
+    if (p == nullptr) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(w->w_qkv) || !aligned16(w->w_o) || !aligned16(w->w_up) ||
+      !aligned16(w->w_down) || !aligned16(w->g_norm1) || !aligned16(w->g_norm2))
+    return DIT_ERR_INVALID_ARG;
+  const int S = n_text + grid_h * grid_w;
+  BlockWorkspace ws = carve_block(cfg, batch, S, nullptr);
+  if (workspace == nullptr || ws_bytes < ws.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return DIT_ERR_WORKSPACE;
+  ws = carve_block(cfg, batch, S, workspace);
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const int M = batch * S, d = cfg->d_model, F = cfg->d_mlp;
+  const uint16_t* x = static_cast<const uint16_t*>(x_in);
+  uint16_t* y = static_cast<uint16_t*>(x_out);
+
+#define JAB_TRY(expr)                               \
+  do {                                              \
+    if ((expr) != cudaSuccess) return DIT_ERR_CUDA; \
+  } while (0)
+  JAB_TRY(launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections, cfg->rope_theta,
+                            ws.cos_tab, ws.sin_tab, s));
+  JAB_TRY(launch_rmsnorm(x, static_cast<const uint16_t*>(w->g_norm1), ws.h, M, d, cfg->eps, s));
+  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.h, w->w_qkv, w->s_qkv, ws.qkv, nullptr, M, 3 * d, d, EPI_NONE, 0}, g, s));
+  JAB_TRY(launch_qknorm_mrope(ws.qkv, batch, S, cfg->n_heads, cfg->head_dim, ws.cos_tab, ws.sin_tab,
+                              static_cast<const uint16_t*>(w->g_q), static_cast<const uint16_t*>(w->g_k), cfg->eps,
+                              s));
+  JAB_TRY(launch_attention(ws.qkv, ws.o, batch, S, cfg->n_heads, cfg->head_dim, g, s));
+  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.o, w->w_o, w->s_o, ws.x1, x, M, d, d, EPI_RESIDUAL, 0}, g, s));
+  JAB_TRY(launch_rmsnorm(ws.x1, static_cast<const uint16_t*>(w->g_norm2), ws.h, M, d, cfg->eps, s));
+  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.h, w->w_up, w->s_up, ws.u, nullptr, M, F, d, EPI_GELU, cfg->gelu_tanh}, g,
+                            s));
+  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.u, w->w_down, w->s_down, y, ws.x1, M, d, F, EPI_RESIDUAL, 0}, g, s));
+#undef JAB_TRY
+  return DIT_OK;
+}
+
+size_t cond_proj_workspace_bytes(int n_tok, int n_layers, int hidden, int d_out) {
+  if (n_tok <= 0 || n_layers <= 0 || hidden <= 0 || d_out <= 0) return 0;
+  return align256(static_cast<size_t>(n_tok) * n_layers * hidden * 2);
+}
+
+int cond_proj_forward(const void* feats, int n_tok, int n_layers, int hidden, const void* g_norm, float eps,
+                      const uint8_t* w, const float* scale, int d_out, void* out, void* workspace, size_t ws_bytes,
+                      void* stream) {
+  if (n_tok <= 0 || n_layers <= 0 || hidden <= 0 || d_out <= 0) return DIT_ERR_INVALID_ARG;
+  const int64_t K = static_cast<int64_t>(n_layers) * hidden;
+  if (K % 256 != 0 || d_out % 256 != 0 || K > (1 << 30)) return DIT_ERR_UNSUPPORTED;
+  if (feats == nullptr || g_norm == nullptr || w == nullptr || scale == nullptr || out == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  if (!aligned16(feats) || !aligned16(g_norm) || !aligned16(w) || !aligned16(out)) return DIT_ERR_INVALID_ARG;
+  const size_t need = cond_proj_workspace_bytes(n_tok, n_layers, hidden, d_out);
+  if (workspace == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return DIT_ERR_WORKSPACE;
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  uint16_t* normed = static_cast<uint16_t*>(workspace);
+  if (launch_rmsnorm(static_cast<const uint16_t*>(feats), static_cast<const uint16_t*>(g_norm), normed, n_tok, K, eps,
+                     s) != cudaSuccess)
+    return DIT_ERR_CUDA;
+  return from_cuda(launch_gemm_w8a16(
+      GemmArgs{normed, w, scale, static_cast<uint16_t*>(out), nullptr, n_tok, d_out, static_cast<int>(K), EPI_NONE, 0},
+      g, s));
+}
+
+}  // extern "C"

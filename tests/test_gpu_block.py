@@ -1,0 +1,114 @@
+"""Whole-call parity: dit_block_forward, cond_proj_forward against the fp64 oracle (needs a B200).
+
+Small shapes are compared element by element; the full 1024 px and 2048 px blocks
+and the full conditioning projection are compared on sampled rows that the oracle
+computes one by one (K and V still span every token).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from joint_attention_block_b200 import ops, synth
+from gpu_util import as_f64, assert_close, dev, empty_bf16, workspace
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_errors():
+    yield
+    assert ops.poll_error() == 0, "a kernel recorded a device-side error"
+
+
+def run_block(shape, inp, n_text=None, gh=None, gw=None, t_img=-1, pos=None):
+    n_text = shape.n_text if n_text is None else n_text
+    gh = shape.grid_h if gh is None else gh
+    gw = shape.grid_w if gw is None else gw
+    cfg = ops.make_config(shape)
+    wd = {k: dev(v) for k, v in inp.items() if k != "x"}
+    weights = ops.make_weights(wd)
+    x = dev(inp["x"])
+    out = torch.empty_like(x)
+    ws = workspace(ops.block_workspace_bytes(cfg, x.shape[0], n_text, gh, gw))
+    ops.dit_block_forward(cfg, weights, x, out, n_text, gh, gw, ws, t_img=t_img,
+                          pos=None if pos is None else dev(pos.astype(np.int32)))
+    torch.cuda.synchronize()
+    return as_f64(out)
+
+
+def test_block_tiny_full():
+    s = synth.TINY
+    inp = synth.block_inputs(s)
+    got = run_block(s, inp)
+    ref = oracle.dit_block_forward(s, inp, inp["x"], s.n_text, s.grid_h, s.grid_w)
+    assert_close(got, ref, what="tiny block")
+
+
+@pytest.mark.parametrize("n_text,gh,gw,batch", [(0, 8, 8, 1), (1, 1, 1, 1), (16, 1, 1, 1), (5, 7, 9, 2), (130, 3, 3, 1), (16, 0, 0, 1)])
+def test_block_edge_shapes(n_text, gh, gw, batch):
+    s = dataclasses.replace(synth.TINY, n_text=n_text, grid_h=gh, grid_w=gw, batch=batch)
+    inp = synth.block_inputs(s)
+    got = run_block(s, inp)
+    ref = oracle.dit_block_forward(s, inp, inp["x"], n_text, gh, gw)
+    assert_close(got, ref, what=f"tiny block {n_text}+{gh}x{gw} b{batch}")
+
+
+def test_block_explicit_positions_and_t_img():
+    s = synth.TINY
+    inp = synth.block_inputs(s)
+    got = run_block(s, inp, t_img=3)
+    ref = oracle.dit_block_forward(s, inp, inp["x"], s.n_text, s.grid_h, s.grid_w, t_img=3)
+    assert_close(got, ref, what="t_img=3")
+    pos = np.random.default_rng(0).integers(0, 50, size=(s.seq, 3))
+    got = run_block(s, inp, pos=pos)
+    ref = oracle.dit_block_forward(s, inp, inp["x"], s.n_text, s.grid_h, s.grid_w, pos=pos)
+    assert_close(got, ref, what="explicit positions")
+
+
+def test_block_tiny_tanh_gelu():
+    s = dataclasses.replace(synth.TINY, gelu_tanh=1)
+    inp = synth.block_inputs(s)
+    assert_close(run_block(s, inp), oracle.dit_block_forward(s, inp, inp["x"], s.n_text, s.grid_h, s.grid_w), what="tanh")
+
+
+def _sampled(shape, inp, n_rows, seed, **kw):
+    got = run_block(shape, inp, **kw)
+    rows = np.sort(np.random.default_rng(seed).choice(shape.seq, size=n_rows, replace=False))
+    rows = np.unique(np.concatenate([rows, [0, shape.n_text - 1 if shape.n_text else 0, shape.n_text, shape.seq - 1]]))
+    ref = oracle.dit_block_forward(shape, inp, inp["x"], shape.n_text, shape.grid_h, shape.grid_w, rows=rows)
+    return got[:, rows], ref
+
+
+def test_block_1024px_sampled_rows():
+    s = synth.C1024
+    got, ref = _sampled(s, synth.block_inputs(s), 24, seed=1)
+    assert_close(got, ref, what="c1024 sampled")
+
+
+def test_uncond_block_1024px_zero_text_sampled_rows():
+    s = synth.UNCOND1024
+    got, ref = _sampled(s, synth.block_inputs(s, zero_text=True), 16, seed=2)
+    assert_close(got, ref, what="uncond 32+4096, zero text")
+
+
+@pytest.mark.slow
+def test_block_2048px_sampled_rows():
+    s = synth.C2048
+    got, ref = _sampled(s, synth.block_inputs(s), 12, seed=3)
+    assert_close(got, ref, what="c2048 sampled")
+
+
+@pytest.mark.parametrize("n_tok", [40, 512])
+def test_cond_proj(n_tok):
+    c = synth.COND
+    inp = synth.cond_inputs(c, n_tok=n_tok)
+    out = empty_bf16(n_tok, c.d_out)
+    ws = workspace(ops.cond_proj_workspace_bytes(n_tok, c.n_layers, c.hidden, c.d_out))
+    ops.cond_proj_forward(dev(inp["feats"]), c.n_layers, c.hidden, dev(inp["g"]), c.eps, dev(inp["w"]),
+                          dev(inp["scale"]), out, ws)
+    rows = np.arange(n_tok) if n_tok <= 64 else np.sort(np.random.default_rng(4).choice(n_tok, 48, replace=False))
+    ref = oracle.cond_proj_forward(inp["feats"][rows], inp["g"], c.eps, inp["w"], inp["scale"])
+    assert_close(as_f64(out)[rows], ref, what=f"cond_proj {n_tok}")
