@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the Ideogram 4 single-stream DiT block hot path on B200.
+
+One step = one pass of the whole hot path on the 1024 px workload:
+  cond_proj_forward   512 tokens x 13*4096 raw text features -> 4096 (written as the
+                      512 text rows of the block input)
+  dit_block_forward   512 text + 64x64 image tokens (S = 4608), d = 4096, 32 x 128 heads,
+                      MLP 16384, FP8 weights with per-row scales
+  euler_cfg_step      x += dt * (v_u + g (v_c - v_u)) on the 4096 x 128 latent
+Metric: DiT block tokens/s (4608 tokens per step per GPU) and TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (under torchrun) every rank runs its own replica of the workload: the
+block does not shard at batch 1, so the ranks exchange nothing but the timing.
+`--impl reference` times the fp64 CPU oracle instead, on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from joint_attention_block_b200 import synth  # noqa: E402
+
+METRIC = "DiT block tokens/s and TFLOP/s at 1024px (4608 tok) vs B200 dense peak"
+WORKLOAD = ("c1024 step: cond_proj 512x53248->4096 feeding the text rows, one DiT block over 512 text + "
+            "64x64 image tokens (d=4096, 32x128 heads, MLP 16384, FP8 weights), Euler/CFG on 4096x128 latent")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_flops():
+    s, c = synth.C1024, synth.COND
+    return s.flops() + c.flops()
+
+
+def gemm_flops_per_step():
+    s, c = synth.C1024, synth.COND
+    S, d, F = s.seq, s.d_model, s.d_mlp
+    return {
+        "gemm_qkv": 2.0 * S * d * 3 * d,
+        "gemm_o": 2.0 * S * d * d,
+        "gemm_up": 2.0 * S * d * F,
+        "gemm_down": 2.0 * S * F * d,
+        "cond_gemm": c.flops(),
+    }
+
+
+def attention_flops_per_step():
+    s = synth.C1024
+    return 4.0 * s.seq * s.seq * s.d_model
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 50 ms) of SM clock and throttle reasons, kept with wall-clock stamps."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.proc = None
+        self.index = index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [v for (t, v) in self.samples if t0 <= t <= t1 + 0.05]
+        if not rows:
+            rows = [v for (_, v) in self.samples[-5:]]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 4 + i and r[4 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------ oracle sample (CPU baseline / reference arm)
+
+
+def oracle_sample_step(state):
+    """One bounded sample of the step on the host: 1 query row of the block (K/V over all
+    4608 tokens), 1 conditioning token, and the whole Euler/CFG update."""
+    import oracle
+
+    s = synth.C1024
+    row = np.array([state["row"] % s.seq])
+    state["row"] += 997
+    oracle.cond_proj_forward(state["cond"]["feats"][:1], state["cond"]["g"], synth.COND.eps, state["cond"]["w"],
+                             state["cond"]["scale"])
+    oracle.dit_block_forward(s, state["blk"], state["blk"]["x"], s.n_text, s.grid_h, s.grid_w, rows=row)
+    e = state["eul"]
+    oracle.euler_cfg_step(e["x"], e["v_cond"], e["v_uncond"], synth.CFG_GUIDANCE, synth.CFG_DT)
+    return 1  # block tokens processed
+
+
+def oracle_state():
+    return {"row": 5, "blk": synth.block_inputs(synth.C1024), "cond": synth.cond_inputs(synth.COND, n_tok=1),
+            "eul": synth.euler_inputs(4096 * synth.LATENT_CHANNELS)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+SAMPLE_DESC = ("per step: 1 of 4608 query rows of the c1024 block (K/V projections over all 4608 tokens), "
+               "cond_proj of 1 of 512 tokens, full Euler/CFG on 4096x128; fp64 numpy oracle")
+
+
+def cpu_baseline():
+    st = oracle_state()
+    t0 = time.perf_counter()
+    n = oracle_sample_step(st)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": SAMPLE_DESC,
+            "seconds": dt}
+
+
+# ------------------------------------------------------------------ reference arm
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    st = oracle_state()
+    steps = args.steps
+    warm = min(args.warmup, 1)
+    for _ in range(warm):
+        oracle_sample_step(st)
+    t0 = time.perf_counter()
+    tokens = 0
+    for _ in range(steps):
+        tokens += oracle_sample_step(st)
+    dt = time.perf_counter() - t0
+    value = tokens / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": warm, "ms_per_step": dt * 1e3 / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": SAMPLE_DESC},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": SAMPLE_DESC},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from joint_attention_block_b200 import ops
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    s, c = synth.C1024, synth.COND
+    blk = synth.block_inputs(s)
+    cond = synth.cond_inputs(c)
+    eul = synth.euler_inputs(4096 * synth.LATENT_CHANNELS)
+    cfg = ops.make_config(s)
+    wd = {k: to_dev(v) for k, v in blk.items() if k != "x"}
+    weights = ops.make_weights(wd)
+    x_in = to_dev(blk["x"])  # [1, 4608, 4096]; rows 0..511 are overwritten by the projection
+    x_out = torch.empty_like(x_in)
+    text_rows = x_in.view(s.seq, s.d_model)[: s.n_text]
+    img_rows = x_in.view(s.seq, s.d_model)[s.n_text:]
+    feats, g_c, w_c, sc_c = (to_dev(cond[k]) for k in ("feats", "g", "w", "scale"))
+    lat, vc, vu = (to_dev(eul[k]) for k in ("x", "v_cond", "v_uncond"))
+    ws_blk = torch.empty(ops.block_workspace_bytes(cfg, 1, s.n_text, s.grid_h, s.grid_w), dtype=torch.uint8, device=dev)
+    ws_c = torch.empty(ops.cond_proj_workspace_bytes(c.n_tok, c.n_layers, c.hidden, c.d_out), dtype=torch.uint8,
+                       device=dev)
+    dt = float(np.float32(synth.CFG_DT))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ops.cond_proj_forward(feats, c.n_layers, c.hidden, g_c, c.eps, w_c, sc_c, text_rows, ws_c, stream=stream)
+        ops.dit_block_forward(cfg, weights, x_in, x_out, s.n_text, s.grid_h, s.grid_w, ws_blk, stream=stream)
+        ops.euler_cfg_step(lat, vc, vu, synth.CFG_GUIDANCE, dt, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ops.poll_error() != 0:
+        raise RuntimeError("device-side error during warm-up")
+
+    # ---- timed region: device-resident inputs; per-launch events inside the library
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(1.0)
+    ops.profile_enable(args.steps * 24 + 64)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    w0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    barrier()
+    ops.profile_disable()
+    clocks.stop()
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    records = ops.profile_read(args.steps * 24 + 64)
+    if ops.poll_error() != 0:
+        raise RuntimeError("device-side error in the timed region")
+
+    # ---- end to end through the public calls: pinned host inputs in, results out, every step
+    h_feats = torch.from_numpy(cond["feats"].view(np.int16)).pin_memory()
+    h_img = torch.from_numpy(np.ascontiguousarray(blk["x"].reshape(s.seq, s.d_model)[s.n_text:]).view(np.int16)).pin_memory()
+    h_lat = torch.from_numpy(eul["x"]).pin_memory()
+    h_vc = torch.from_numpy(eul["v_cond"].view(np.int16)).pin_memory()
+    h_vu = torch.from_numpy(eul["v_uncond"].view(np.int16)).pin_memory()
+    h_out = torch.empty(x_out.shape, dtype=x_out.dtype).pin_memory()
+    h_lat_out = torch.empty_like(h_lat).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_feats, h_img, h_lat, h_vc, h_vu))
+    d2h = h_out.numel() * h_out.element_size() + h_lat_out.numel() * h_lat_out.element_size()
+
+    def e2e_step():
+        feats.copy_(h_feats, non_blocking=True)
+        img_rows.copy_(h_img, non_blocking=True)
+        lat.copy_(h_lat, non_blocking=True)
+        vc.copy_(h_vc, non_blocking=True)
+        vu.copy_(h_vu, non_blocking=True)
+        step()
+        h_out.copy_(x_out, non_blocking=True)
+        h_lat_out.copy_(lat, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1))
+
+    if rank != 0:
+        return
+
+    # ---- numbers
+    toks = s.seq * args.steps * world
+    value = toks / (ms / 1e3)
+    tflops = step_flops() * args.steps * world / (ms / 1e3) / 1e12
+    pk, pk_kind = peaks()
+    per = {}
+    for name, t in records:
+        d = per.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += t
+    total_kernel_ms = sum(v[1] for v in per.values())
+    gf = gemm_flops_per_step()
+    gemm_names = [n for n in gf if n in per]
+    gemm_ms = sum(per[n][1] for n in gemm_names)
+    gemm_launches = sum(per[n][0] for n in gemm_names)
+    gemm_fl = sum(gf[n] * per[n][0] for n in gemm_names)
+    peak_tc = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    achieved = gemm_fl / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    kernels = {}
+    for n, (cnt, t) in sorted(per.items(), key=lambda kv: -kv[1][1]):
+        k = {"launches": cnt, "ms_total": round(t, 4), "ms_avg": round(t / cnt, 5),
+             "share": round(t / total_kernel_ms, 4) if total_kernel_ms else None}
+        if n in gf:
+            k["tflops"] = round(gf[n] * cnt / (t / 1e3) / 1e12, 1)
+        if n == "attention":
+            k["tflops"] = round(attention_flops_per_step() * cnt / (t / 1e3) / 1e12, 1)
+        kernels[n] = k
+    clk = clocks.summary(w0, w1)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "tflops": round(tflops, 1),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "w:e4m3 a:f16/bf16 acc:f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "model": "Ideogram 4 single-stream DiT block (random-init, FP8)",
+                   "global_batch": world, "seq_len": s.seq, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (~0.6 GB of weights/features read per step); no flush"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_w8a16 (all FP8-weight GEMMs of the step)",
+                     "achieved": round(achieved, 1) if achieved else None, "peak": peak_tc, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_tc, 4) if achieved else None, "traffic": None,
+                     "peak_kind": f"{pk_kind} bf16 dense, sustained", "launches": gemm_launches,
+                     "flops_per_launch": gemm_fl / max(gemm_launches, 1)},
+        "kernels": kernels,
+        "gpu_launches": len(records),
+        "clocks": clk,
+        "e2e": {"value": round(s.seq * e2e_steps * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

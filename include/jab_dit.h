@@ -45,6 +45,9 @@ typedef enum {
   DIT_ERR_DEVICE = 6       /* another device-side error was recorded (from dit_poll_error) */
 } dit_status;
 
+/* Storage formats of activations, for the per-step kernels below. */
+typedef enum { DIT_FMT_BF16 = 0, DIT_FMT_F16 = 1, DIT_FMT_F32 = 2 } dit_format;
+
 /* Shape and numerics of one block.
  * rope_sections: rotary PAIRS per axis (t, h, w), laid out contiguously over the
  *   first head_dim/2 frequencies; must sum to head_dim/2.  The Ideogram 4 deep dive,
@@ -124,34 +127,66 @@ DIT_API int euler_cfg_step(float* x, const void* v_cond, const void* v_uncond, i
  * on chip, before the per-row scale). */
 DIT_API int dit_e4m3_to_bf16(const uint8_t* codes, void* out, int64_t n, void* stream);
 
-/* Row RMSNorm with gain: y = x / sqrt(mean(x^2) + eps) * g, bf16 in/out, fp32 math.
- * x, y: [rows, cols] (may alias); g: [cols].  cols % 8 == 0. */
-DIT_API int dit_rmsnorm_rows(const void* x, const void* g, void* y, int64_t rows, int64_t cols, float eps, void* stream);
+/* Row RMSNorm with gain: y = x / sqrt(mean(x^2) + eps) * g, fp32 math.
+ * x: [rows, cols] in x_fmt (BF16 or F32); y: [rows, cols] in y_fmt (BF16 or F16);
+ * g: bf16 [cols].  x and y may alias when the formats match.  cols % 8 == 0. */
+DIT_API int dit_rmsnorm_rows(const void* x, int x_fmt, const void* g, void* y, int y_fmt, int64_t rows, int64_t cols,
+                             float eps, void* stream);
 
 /* The (t, h, w) int32 [S, 3] positions the block uses for this sequence (see dit_block_forward). */
 DIT_API int dit_mrope_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos_out, void* stream);
 
-/* Y[M, N] = epilogue( A[M, K] (W8[N, K])^T * scale[N] ).  A bf16 row-major, W8 e4m3
- * row-major, scale fp32.  epilogue: 0 = none, 1 = GELU (gelu_tanh selects the form),
- * 2 = + residual R[M, N] (bf16).  Y bf16 [M, N].  N % 32 == 0, K % 16 == 0. */
-DIT_API int dit_gemm_w8a16(const void* a, const uint8_t* w8, const float* scale, void* y, const void* residual, int M,
-                   int N, int K, int epilogue, int gelu_tanh, void* stream);
+/* Y[M, N] = act( A[M, K] (W8[N, K])^T * scale[N] ) + R[M, N]
+ * A: a_fmt (BF16 or F16) row-major; W8: e4m3 row-major (the weight is widened on chip,
+ * exactly, to A's format); scale: fp32 [N]; act: 0 = none, 1 = GELU (gelu_tanh selects
+ * the form); R: optional residual in res_fmt (BF16/F16/F32), NULL for none; Y: y_fmt
+ * (BF16/F16/F32).  fp32 accumulation.  N % 32 == 0, K % 16 == 0. */
+DIT_API int dit_gemm_w8a16(const void* a, int a_fmt, const uint8_t* w8, const float* scale, void* y, int y_fmt,
+                           const void* residual, int res_fmt, int M, int N, int K, int act, int gelu_tanh,
+                           void* stream);
 
-/* Per-head QK-RMSNorm + 3D M-RoPE, in place on a fused qkv buffer bf16 [batch, S, 3d]
- * (Q columns [0, d), K columns [d, 2d); V untouched).  pos: int32 [S, 3] or NULL
- * (derived from n_text/grid/t_img as in dit_block_forward). */
-DIT_API int dit_qknorm_mrope(void* qkv, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
+/* Per-head QK-RMSNorm + 3D M-RoPE, in place on a fused qkv buffer [batch, S, 3d] in fmt
+ * (BF16 or F16; Q columns [0, d), K columns [d, 2d); V untouched).  pos: int32 [S, 3] or
+ * NULL (derived from n_text/grid/t_img as in dit_block_forward).  workspace holds the
+ * fp32 cos/sin tables: >= 2 * align256(S * head_dim/2 * 4) bytes. */
+DIT_API int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                      const dit_block_config* cfg, const void* g_q, const void* g_k, void* workspace,
                      size_t ws_bytes, void* stream);
 
 /* Joint bidirectional attention: out[b, s, h*hd:(h+1)*hd] = softmax(q k^T / sqrt(hd)) v
- * over all S tokens, per head, reading q, k, v from a fused qkv buffer bf16 [batch, S, 3d].
- * out: bf16 [batch, S, d]. */
-DIT_API int dit_joint_attention(const void* qkv, void* out, int batch, int seq, int n_heads, int head_dim, void* stream);
+ * over all S tokens, per head, reading q, k, v from a fused qkv buffer [batch, S, 3d] in
+ * fmt (BF16 or F16).  out: [batch, S, d] in the same format. */
+DIT_API int dit_joint_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim, void* stream);
 
 /* Synchronise `stream`, then report (and clear) device-side errors recorded by any
  * kernel of this library on the current device since the last poll. */
 DIT_API int dit_poll_error(void* stream);
+
+/* ---- launch instrumentation (off by default) ----
+ * While enabled, each kernel launched by dit_block_forward, cond_proj_forward and
+ * euler_cfg_step is bracketed by CUDA events on its stream, so the device time of
+ * every launch inside a timed region can be read back.  dit_profile_enable creates
+ * max_marks events (host-side handles; the only resources this library creates) and
+ * starts recording; dit_profile_read synchronises on the recorded events, writes up to
+ * max_records (tag, milliseconds) pairs and returns how many it wrote (negative status
+ * on error), then clears the record. */
+typedef enum {
+  DIT_KERNEL_END = 0,
+  DIT_KERNEL_ROPE_TABLE = 1,
+  DIT_KERNEL_RMSNORM = 2,
+  DIT_KERNEL_GEMM_QKV = 3,
+  DIT_KERNEL_QKNORM_MROPE = 4,
+  DIT_KERNEL_ATTENTION = 5,
+  DIT_KERNEL_GEMM_O = 6,
+  DIT_KERNEL_GEMM_UP = 7,
+  DIT_KERNEL_GEMM_DOWN = 8,
+  DIT_KERNEL_COND_RMSNORM = 9,
+  DIT_KERNEL_COND_GEMM = 10,
+  DIT_KERNEL_EULER_CFG = 11
+} dit_kernel_tag;
+DIT_API int dit_profile_enable(int max_marks);
+DIT_API int dit_profile_disable(void);
+DIT_API int dit_profile_read(int* tags, float* ms, int max_records);
 
 /* Set the wall-time limit of every device-side bounded wait (default 2000 ms). */
 DIT_API int dit_set_wait_timeout_ms(uint32_t ms);

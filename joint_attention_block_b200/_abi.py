@@ -17,6 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libjab_b200.so")
 
 DIT_OK = 0
+FMT_BF16, FMT_F16, FMT_F32 = 0, 1, 2
 STATUS_NAMES = {
     0: "DIT_OK",
     1: "DIT_ERR_INVALID_ARG",
@@ -68,12 +69,15 @@ SIGNATURES = {
     "cond_proj_forward": (_I, [_P, _I, _I, _I, _P, _F, _P, _P, _I, _P, _P, _SZ, _P]),
     "euler_cfg_step": (_I, [_P, _P, _P, _I64, _F, _F, _P]),
     "dit_e4m3_to_bf16": (_I, [_P, _P, _I64, _P]),
-    "dit_rmsnorm_rows": (_I, [_P, _P, _P, _I64, _I64, _F, _P]),
+    "dit_rmsnorm_rows": (_I, [_P, _I, _P, _P, _I, _I64, _I64, _F, _P]),
     "dit_mrope_positions": (_I, [_I, _I, _I, _I, _P, _P]),
-    "dit_gemm_w8a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
-    "dit_qknorm_mrope": (_I, [_P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(BlockConfig), _P, _P, _P, _SZ, _P]),
-    "dit_joint_attention": (_I, [_P, _P, _I, _I, _I, _I, _P]),
+    "dit_gemm_w8a16": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "dit_qknorm_mrope": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(BlockConfig), _P, _P, _P, _SZ, _P]),
+    "dit_joint_attention": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
     "dit_poll_error": (_I, [_P]),
+    "dit_profile_enable": (_I, [_I]),
+    "dit_profile_disable": (_I, []),
+    "dit_profile_read": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float), _I]),
     "dit_set_wait_timeout_ms": (_I, [ctypes.c_uint32]),
     "dit_status_str": (ctypes.c_char_p, [_I]),
     "dit_abi_version": (_I, []),
@@ -173,10 +177,11 @@ def e4m3_to_bf16(codes: torch.Tensor, out: torch.Tensor, stream=None) -> None:
     _check("dit_e4m3_to_bf16", lib().dit_e4m3_to_bf16(_ptr(codes), _ptr(out), codes.numel(), _stream(stream)))
 
 
-def rmsnorm_rows(x: torch.Tensor, g: torch.Tensor, y: torch.Tensor, eps: float, stream=None) -> None:
+def rmsnorm_rows(x: torch.Tensor, g: torch.Tensor, y: torch.Tensor, eps: float, x_fmt: int = FMT_BF16,
+                 y_fmt: int = FMT_BF16, stream=None) -> None:
     cols = x.shape[-1]
-    _check("dit_rmsnorm_rows", lib().dit_rmsnorm_rows(_ptr(x), _ptr(g), _ptr(y), x.numel() // cols, cols, eps,
-                                                      _stream(stream)))
+    _check("dit_rmsnorm_rows", lib().dit_rmsnorm_rows(_ptr(x), x_fmt, _ptr(g), _ptr(y), y_fmt, x.numel() // cols, cols,
+                                                      eps, _stream(stream)))
 
 
 def mrope_positions(n_text: int, grid_h: int, grid_w: int, t_img: int, out: torch.Tensor, stream=None) -> None:
@@ -185,24 +190,48 @@ def mrope_positions(n_text: int, grid_h: int, grid_w: int, t_img: int, out: torc
 
 
 def gemm_w8a16(a: torch.Tensor, w8: torch.Tensor, scale: torch.Tensor, y: torch.Tensor,
-               residual: Optional[torch.Tensor] = None, epilogue: int = 0, gelu_tanh: int = 0, stream=None) -> None:
+               residual: Optional[torch.Tensor] = None, act: int = 0, gelu_tanh: int = 0, a_fmt: int = FMT_BF16,
+               y_fmt: int = FMT_BF16, res_fmt: int = FMT_BF16, stream=None) -> None:
     M, K = a.shape
     N = w8.shape[0]
-    _check("dit_gemm_w8a16", lib().dit_gemm_w8a16(_ptr(a), _ptr(w8), _ptr(scale), _ptr(y), _ptr(residual), M, N, K,
-                                                  epilogue, gelu_tanh, _stream(stream)))
+    _check("dit_gemm_w8a16", lib().dit_gemm_w8a16(_ptr(a), a_fmt, _ptr(w8), _ptr(scale), _ptr(y), y_fmt,
+                                                  _ptr(residual), res_fmt, M, N, K, act, gelu_tanh, _stream(stream)))
 
 
 def qknorm_mrope(qkv: torch.Tensor, cfg: BlockConfig, n_text: int, grid_h: int, grid_w: int, g_q: torch.Tensor,
                  g_k: torch.Tensor, workspace: torch.Tensor, t_img: int = -1, pos: Optional[torch.Tensor] = None,
-                 stream=None) -> None:
+                 fmt: int = FMT_BF16, stream=None) -> None:
     _check("dit_qknorm_mrope", lib().dit_qknorm_mrope(
-        _ptr(qkv), qkv.shape[0], n_text, grid_h, grid_w, t_img, _ptr(pos), ctypes.byref(cfg), _ptr(g_q), _ptr(g_k),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+        _ptr(qkv), fmt, qkv.shape[0], n_text, grid_h, grid_w, t_img, _ptr(pos), ctypes.byref(cfg), _ptr(g_q),
+        _ptr(g_k), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
-def joint_attention(qkv: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int, stream=None) -> None:
-    _check("dit_joint_attention", lib().dit_joint_attention(_ptr(qkv), _ptr(out), qkv.shape[0], qkv.shape[1], n_heads,
-                                                            head_dim, _stream(stream)))
+def joint_attention(qkv: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int, fmt: int = FMT_BF16,
+                    stream=None) -> None:
+    _check("dit_joint_attention", lib().dit_joint_attention(_ptr(qkv), _ptr(out), fmt, qkv.shape[0], qkv.shape[1],
+                                                            n_heads, head_dim, _stream(stream)))
+
+
+KERNEL_TAGS = {1: "rope_table", 2: "rmsnorm", 3: "gemm_qkv", 4: "qknorm_mrope", 5: "attention", 6: "gemm_o",
+               7: "gemm_up", 8: "gemm_down", 9: "cond_rmsnorm", 10: "cond_gemm", 11: "euler_cfg"}
+
+
+def profile_enable(max_marks: int) -> None:
+    _check("dit_profile_enable", lib().dit_profile_enable(max_marks))
+
+
+def profile_disable() -> None:
+    lib().dit_profile_disable()
+
+
+def profile_read(max_records: int = 1 << 16):
+    """[(kernel name, ms), ...] of every launch recorded since profile_enable / the last read."""
+    tags = (ctypes.c_int * max_records)()
+    ms = (ctypes.c_float * max_records)()
+    n = lib().dit_profile_read(tags, ms, max_records)
+    if n < 0:
+        raise DitError("dit_profile_read", -n)
+    return [(KERNEL_TAGS.get(tags[i], str(tags[i])), float(ms[i])) for i in range(n)]
 
 
 def poll_error(stream=None) -> int:

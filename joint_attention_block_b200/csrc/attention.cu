@@ -13,11 +13,12 @@
 //               memory, V read MN-major), so QK^T of block j overlaps softmax j-1.
 //   warps 2..5  softmax: thread i owns query row i (TMEM lane i), so the running
 //               max and sum are thread-local.  exp2 with the log2(e)/sqrt(hd) scale
-//               folded in; P is written as bf16 into a 128B-swizzled K-major tile.
+//               folded in; P is written as 16-bit (the q/k/v format: bf16 or f16)
+//               into a 128B-swizzled K-major tile.
 //               The running max is only raised (and O in TMEM rescaled) when it
 //               grows by more than 2^8; until then the stale max is used for both
 //               P and the row sum, which leaves O / l unchanged and keeps P <= 256.
-//               The final O / l is stored as bf16.
+//               The final O / l is stored in the q/k/v format.
 #include "common.cuh"
 
 namespace jab {
@@ -43,11 +44,12 @@ struct Layout {
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
 };
 
-template <int HD>
+template <int HD, int F>
 __global__ void __launch_bounds__(THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm, uint16_t* __restrict__ out, int seq, int n_heads,
                      const KernelGuard guard) {
   using L = Layout<HD>;
+  constexpr bool kF16 = F == FMT_F16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::OFF_Q;
@@ -132,8 +134,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
-    constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKV, false, false);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(BQ, HD, false, true);
+    constexpr uint32_t idesc_s = idesc_f16kind(BQ, BKV, kF16, false, false);
+    constexpr uint32_t idesc_o = idesc_f16kind(BQ, HD, kF16, false, true);
     bool ok = mbar_wait(q_full, 0u, guard, abort_flag, ERR_TIMEOUT_ATTN_MMA);
     auto issue_pv = [&](int i) -> bool {
       const int st = i & 1;
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(pbase + (kk >> 2) * L::SLAB + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, L::SLAB, 1024);
-          mma_bf16_ss(tmem_o, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_f16kind_ss(tmem_o, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(p_empty);
         mma_commit(&kv_empty[st]);
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::SLAB + (kk & 3) * 32;
-          mma_bf16_ss(tmem + st * BKV, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+          mma_f16kind_ss(tmem + st * BKV, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
                       idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[st]);
@@ -254,14 +256,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tmem_st_wait();
       }
-      // P row -> bf16, 128B-swizzled K-major (two 64-key slabs)
+      // P row -> 16-bit, 128B-swizzled K-major (two 64-key slabs)
 #pragma unroll
       for (int kc = 0; kc < BKV / 8; ++kc) {
         uint4 o;
-        o.x = pack_bf16x2(s[8 * kc + 0], s[8 * kc + 1]);
-        o.y = pack_bf16x2(s[8 * kc + 2], s[8 * kc + 3]);
-        o.z = pack_bf16x2(s[8 * kc + 4], s[8 * kc + 5]);
-        o.w = pack_bf16x2(s[8 * kc + 6], s[8 * kc + 7]);
+        o.x = pack2<F>(s[8 * kc + 0], s[8 * kc + 1]);
+        o.y = pack2<F>(s[8 * kc + 2], s[8 * kc + 3]);
+        o.z = pack2<F>(s[8 * kc + 4], s[8 * kc + 5]);
+        o.w = pack2<F>(s[8 * kc + 6], s[8 * kc + 7]);
         uint8_t* dst = sP + (kc >> 3) * L::SLAB + r * 128 + ((((kc & 7) ^ (r & 7))) << 4);
         *reinterpret_cast<uint4*>(dst) = o;
       }
@@ -284,10 +286,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(raw[8 * q + 0]) * inv_l, __uint_as_float(raw[8 * q + 1]) * inv_l);
-            o.y = pack_bf16x2(__uint_as_float(raw[8 * q + 2]) * inv_l, __uint_as_float(raw[8 * q + 3]) * inv_l);
-            o.z = pack_bf16x2(__uint_as_float(raw[8 * q + 4]) * inv_l, __uint_as_float(raw[8 * q + 5]) * inv_l);
-            o.w = pack_bf16x2(__uint_as_float(raw[8 * q + 6]) * inv_l, __uint_as_float(raw[8 * q + 7]) * inv_l);
+            o.x = pack2<F>(__uint_as_float(raw[8 * q + 0]) * inv_l, __uint_as_float(raw[8 * q + 1]) * inv_l);
+            o.y = pack2<F>(__uint_as_float(raw[8 * q + 2]) * inv_l, __uint_as_float(raw[8 * q + 3]) * inv_l);
+            o.z = pack2<F>(__uint_as_float(raw[8 * q + 4]) * inv_l, __uint_as_float(raw[8 * q + 5]) * inv_l);
+            o.w = pack2<F>(__uint_as_float(raw[8 * q + 6]) * inv_l, __uint_as_float(raw[8 * q + 7]) * inv_l);
             reinterpret_cast<uint4*>(dst + 32 * c)[q] = o;
           }
         }
@@ -303,32 +305,38 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int HD>
-cudaError_t launch_hd(const CUtensorMap& tm, uint16_t* out, int batch, int seq, int n_heads, const KernelGuard& g,
+template <int HD, int F>
+cudaError_t launch_hd(const CUtensorMap& tm, void* out, int batch, int seq, int n_heads, const KernelGuard& g,
                       cudaStream_t s) {
   using L = Layout<HD>;
-  cudaError_t e = cudaFuncSetAttribute(attention_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+  cudaError_t e =
+      cudaFuncSetAttribute(attention_kernel<HD, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((seq + BQ - 1) / BQ, n_heads, batch);
-  attention_kernel<HD><<<grid, THREADS, L::SMEM, s>>>(tm, out, seq, n_heads, g);
+  attention_kernel<HD, F><<<grid, THREADS, L::SMEM, s>>>(tm, static_cast<uint16_t*>(out), seq, n_heads, g);
   return cudaGetLastError();
 }
 
 }  // namespace attn
 
-cudaError_t launch_attention(const uint16_t* qkv, uint16_t* out, int batch, int seq, int n_heads, int head_dim,
+cudaError_t launch_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
                              const KernelGuard& g, cudaStream_t s) {
   if (batch <= 0 || seq <= 0) return cudaSuccess;
+  if (fmt != FMT_BF16 && fmt != FMT_F16) return cudaErrorInvalidValue;
   const int d = n_heads * head_dim;
   CUtensorMap tm;
   const uint64_t dims[3] = {static_cast<uint64_t>(3 * d), static_cast<uint64_t>(seq), static_cast<uint64_t>(batch)};
   const uint64_t strides[2] = {static_cast<uint64_t>(3 * d) * 2, static_cast<uint64_t>(seq) * 3 * d * 2};
   const uint32_t box[3] = {64, attn::BKV, 1};
-  if (!make_tmap(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(qkv), dims, strides, box,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_tmap(&tm, fmt == FMT_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                 const_cast<void*>(qkv), dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (head_dim == 128) return attn::launch_hd<128>(tm, out, batch, seq, n_heads, g, s);
-  if (head_dim == 64) return attn::launch_hd<64>(tm, out, batch, seq, n_heads, g, s);
+  if (head_dim == 128)
+    return fmt == FMT_F16 ? attn::launch_hd<128, FMT_F16>(tm, out, batch, seq, n_heads, g, s)
+                          : attn::launch_hd<128, FMT_BF16>(tm, out, batch, seq, n_heads, g, s);
+  if (head_dim == 64)
+    return fmt == FMT_F16 ? attn::launch_hd<64, FMT_F16>(tm, out, batch, seq, n_heads, g, s)
+                          : attn::launch_hd<64, FMT_BF16>(tm, out, batch, seq, n_heads, g, s);
   return cudaErrorInvalidValue;
 }
 

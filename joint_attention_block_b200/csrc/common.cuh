@@ -46,6 +46,74 @@ JAB_DEVICE uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Two fp32 -> packed f16x2 (round to nearest even, saturating to +-65504), lo in the low half.
+JAB_DEVICE uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+JAB_DEVICE float f16_lo(uint32_t v) {
+  float f;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(f) : "r"(v));
+  return f;
+}
+JAB_DEVICE float f16_hi(uint32_t v) {
+  float f;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, h;\n\t}" : "=f"(f) : "r"(v));
+  return f;
+}
+
+template <int F>
+JAB_DEVICE uint32_t pack2(float lo, float hi) {
+  if constexpr (F == FMT_F16) return pack_f16x2(lo, hi);
+  else return pack_bf16x2(lo, hi);
+}
+template <int F>
+JAB_DEVICE float unpack_lo(uint32_t v) {
+  if constexpr (F == FMT_F16) return f16_lo(v);
+  else return bf16_lo(v);
+}
+template <int F>
+JAB_DEVICE float unpack_hi(uint32_t v) {
+  if constexpr (F == FMT_F16) return f16_hi(v);
+  else return bf16_hi(v);
+}
+
+// Load 8 consecutive activations of format F (16-bit: one 16-byte vector; f32: two).
+template <int F>
+JAB_DEVICE void load8(const void* base, int64_t idx8, float (&v)[8]) {
+  if constexpr (F == FMT_F32) {
+    const float4 a = reinterpret_cast<const float4*>(base)[2 * idx8];
+    const float4 b = reinterpret_cast<const float4*>(base)[2 * idx8 + 1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 a = reinterpret_cast<const uint4*>(base)[idx8];
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(&a);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = unpack_lo<F>(w[k]);
+      v[2 * k + 1] = unpack_hi<F>(w[k]);
+    }
+  }
+}
+
+// Store 8 consecutive values in format F.
+template <int F>
+JAB_DEVICE void store8(void* base, int64_t idx8, const float (&v)[8]) {
+  if constexpr (F == FMT_F32) {
+    reinterpret_cast<float4*>(base)[2 * idx8] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(base)[2 * idx8 + 1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint4 o;
+    o.x = pack2<F>(v[0], v[1]);
+    o.y = pack2<F>(v[2], v[3]);
+    o.z = pack2<F>(v[4], v[5]);
+    o.w = pack2<F>(v[6], v[7]);
+    reinterpret_cast<uint4*>(base)[idx8] = o;
+  }
+}
+
 JAB_DEVICE float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -70,6 +138,26 @@ JAB_DEVICE void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
   const uint32_t two120 = 0x7B807B80u;  // bf16x2 (2^120, 2^120)
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(two120));
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(two120));
+}
+
+// e4m3 bytes -> f16, exactly, for all finite codes.  Same widening as above but
+// shifted left by 7 and masked with 0xBF80: as an f16 that is value(b) * 2^-8
+// (e4m3 subnormals land on f16 subnormals); an f16 multiply by 2^8 restores it.
+JAB_DEVICE void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  uint32_t a, b;
+  asm("prmt.b32 %0, %1, 0, 0x9180;" : "=r"(a) : "r"(w));
+  asm("prmt.b32 %0, %1, 0, 0xB3A2;" : "=r"(b) : "r"(w));
+  a = (a << 7) & 0xBF80BF80u;
+  b = (b << 7) & 0xBF80BF80u;
+  const uint32_t two8 = 0x5C005C00u;  // f16x2 (256, 256)
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(two8));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(two8));
+}
+
+template <bool F16>
+JAB_DEVICE void e4m3x4_to_16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  if constexpr (F16) e4m3x4_to_f16x4(w, lo, hi);
+  else e4m3x4_to_bf16x4(w, lo, hi);
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -183,17 +271,18 @@ JAB_DEVICE uint64_t smem_desc_sw128(uint32_t smem_addr, uint32_t lbo_bytes, uint
   return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+// Instruction descriptor of kind::f16 with fp32 accumulation; A and B are both
+// bf16 (f16 = false) or both f16 (f16 = true).
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool f16, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                      // D format f32
-         | (1u << 7)                                    // A bf16
-         | (1u << 10)                                   // B bf16
+         | (f16 ? 0u : (1u << 7))                       // A: 0 = f16, 1 = bf16
+         | (f16 ? 0u : (1u << 10))                      // B: 0 = f16, 1 = bf16
          | (a_mn_major ? (1u << 15) : 0u) | (b_mn_major ? (1u << 16) : 0u) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
-JAB_DEVICE void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+JAB_DEVICE void mma_f16kind_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"

@@ -71,6 +71,31 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base
   return r == CUDA_SUCCESS;
 }
 
+// ------------------------------------------------------------------ launch instrumentation
+
+// When enabled, every launch of the three calls is bracketed by CUDA events on
+// its stream (tag = which kernel), so a caller can read per-kernel device time
+// of the very launches it timed.  Off by default; events are created once, at
+// enable time.
+struct ProfState {
+  bool on = false;
+  int cap = 0;
+  int n = 0;
+  cudaEvent_t* ev = nullptr;
+  int* tag = nullptr;
+};
+static ProfState g_prof;
+static std::mutex g_prof_mu;
+
+void prof_mark(cudaStream_t s, int tag) {
+  if (!g_prof.on) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (g_prof.n >= g_prof.cap) return;
+  cudaEventRecord(g_prof.ev[g_prof.n], s);
+  g_prof.tag[g_prof.n] = tag;
+  ++g_prof.n;
+}
+
 }  // namespace jab
 
 using namespace jab;
@@ -94,13 +119,15 @@ int check_config(const dit_block_config* c) {
   return DIT_OK;
 }
 
+// Internal activations: h, qkv, o, u in f16 (every one is bounded: post-norm,
+// softmax-weighted or a GEMM of bounded inputs); the residual x1 in fp32.
 struct BlockWorkspace {
   float* cos_tab;
   float* sin_tab;
   uint16_t* h;
   uint16_t* qkv;
   uint16_t* o;
-  uint16_t* x1;
+  float* x1;
   uint16_t* u;
   size_t bytes;
 };
@@ -116,7 +143,7 @@ BlockWorkspace carve_block(const dit_block_config* c, int batch, int seq, void* 
     return o;
   };
   const size_t o_cos = take(seq * half * 4), o_sin = take(seq * half * 4);
-  const size_t o_h = take(M * d * 2), o_qkv = take(M * 3 * d * 2), o_o = take(M * d * 2), o_x1 = take(M * d * 2);
+  const size_t o_h = take(M * d * 2), o_qkv = take(M * 3 * d * 2), o_o = take(M * d * 2), o_x1 = take(M * d * 4);
   const size_t o_u = take(M * F * 2);
   w.bytes = off;
   if (base != nullptr) {
@@ -126,7 +153,7 @@ BlockWorkspace carve_block(const dit_block_config* c, int batch, int seq, void* 
     w.h = reinterpret_cast<uint16_t*>(b + o_h);
     w.qkv = reinterpret_cast<uint16_t*>(b + o_qkv);
     w.o = reinterpret_cast<uint16_t*>(b + o_o);
-    w.x1 = reinterpret_cast<uint16_t*>(b + o_x1);
+    w.x1 = reinterpret_cast<float*>(b + o_x1);
     w.u = reinterpret_cast<uint16_t*>(b + o_u);
   }
   return w;
@@ -143,6 +170,49 @@ bool shape_ok(int batch, int n_text, int grid_h, int grid_w) {
 extern "C" {
 
 int dit_abi_version(void) { return 1; }
+
+int dit_profile_enable(int max_marks) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (max_marks <= 0) return DIT_ERR_INVALID_ARG;
+  if (g_prof.cap < max_marks) {
+    for (int i = 0; i < g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+    delete[] g_prof.ev;
+    delete[] g_prof.tag;
+    g_prof.ev = new cudaEvent_t[max_marks];
+    g_prof.tag = new int[max_marks];
+    for (int i = 0; i < max_marks; ++i)
+      if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) {
+        g_prof.cap = i;
+        return DIT_ERR_CUDA;
+      }
+    g_prof.cap = max_marks;
+  }
+  g_prof.n = 0;
+  g_prof.on = true;
+  return DIT_OK;
+}
+
+int dit_profile_disable(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof.on = false;
+  return DIT_OK;
+}
+
+int dit_profile_read(int* tags, float* ms, int max_records) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  int out = 0;
+  for (int i = 0; i + 1 < g_prof.n && out < max_records; ++i) {
+    if (g_prof.tag[i] == DIT_KERNEL_END) continue;
+    float t = 0.f;
+    if (cudaEventSynchronize(g_prof.ev[i + 1]) != cudaSuccess) return -DIT_ERR_CUDA;
+    if (cudaEventElapsedTime(&t, g_prof.ev[i], g_prof.ev[i + 1]) != cudaSuccess) return -DIT_ERR_CUDA;
+    tags[out] = g_prof.tag[i];
+    ms[out] = t;
+    ++out;
+  }
+  g_prof.n = 0;
+  return out;
+}
 
 const char* dit_status_str(int s) {
   switch (s) {
@@ -182,20 +252,26 @@ int dit_e4m3_to_bf16(const uint8_t* codes, void* out, int64_t n, void* stream) {
   return from_cuda(launch_e4m3_to_bf16(codes, static_cast<uint16_t*>(out), n, as_stream(stream)));
 }
 
-int dit_rmsnorm_rows(const void* x, const void* g, void* y, int64_t rows, int64_t cols, float eps, void* stream) {
+int dit_rmsnorm_rows(const void* x, int x_fmt, const void* g, void* y, int y_fmt, int64_t rows, int64_t cols,
+                     float eps, void* stream) {
   if (rows < 0 || cols <= 0 || cols % 8 != 0 || rows > (1ll << 31) - 1) return DIT_ERR_INVALID_ARG;
+  if ((x_fmt != FMT_BF16 && x_fmt != FMT_F32) || (y_fmt != FMT_BF16 && y_fmt != FMT_F16)) return DIT_ERR_INVALID_ARG;
   if (rows > 0 && (x == nullptr || g == nullptr || y == nullptr)) return DIT_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(g) || !aligned16(y)) return DIT_ERR_INVALID_ARG;
-  return from_cuda(launch_rmsnorm(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g),
-                                  static_cast<uint16_t*>(y), rows, cols, eps, as_stream(stream)));
+  if (x == y && x_fmt != y_fmt) return DIT_ERR_INVALID_ARG;
+  return from_cuda(launch_rmsnorm(x, x_fmt, static_cast<const uint16_t*>(g), y, y_fmt, rows, cols, eps,
+                                  as_stream(stream)));
 }
 
 int euler_cfg_step(float* x, const void* v_cond, const void* v_uncond, int64_t n, float guidance, float dt,
                    void* stream) {
   if (n < 0 || (n > 0 && (x == nullptr || v_cond == nullptr || v_uncond == nullptr))) return DIT_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(v_cond) || !aligned16(v_uncond)) return DIT_ERR_INVALID_ARG;
-  return from_cuda(launch_euler_cfg(x, static_cast<const uint16_t*>(v_cond), static_cast<const uint16_t*>(v_uncond),
-                                    n, guidance, dt, as_stream(stream)));
+  prof_mark(as_stream(stream), DIT_KERNEL_EULER_CFG);
+  const cudaError_t e = launch_euler_cfg(x, static_cast<const uint16_t*>(v_cond),
+                                         static_cast<const uint16_t*>(v_uncond), n, guidance, dt, as_stream(stream));
+  prof_mark(as_stream(stream), DIT_KERNEL_END);
+  return from_cuda(e);
 }
 
 int dit_mrope_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos_out, void* stream) {
@@ -204,29 +280,30 @@ int dit_mrope_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* 
   return from_cuda(launch_positions(n_text, grid_h, grid_w, t_img, pos_out, as_stream(stream)));
 }
 
-int dit_gemm_w8a16(const void* a, const uint8_t* w8, const float* scale, void* y, const void* residual, int M, int N,
-                   int K, int epilogue, int gelu_tanh, void* stream) {
+int dit_gemm_w8a16(const void* a, int a_fmt, const uint8_t* w8, const float* scale, void* y, int y_fmt,
+                   const void* residual, int res_fmt, int M, int N, int K, int act, int gelu_tanh, void* stream) {
   if (M < 0 || N <= 0 || K <= 0) return DIT_ERR_INVALID_ARG;
   if (N % 32 != 0 || K % 16 != 0) return DIT_ERR_UNSUPPORTED;
-  if (epilogue < 0 || epilogue > 2) return DIT_ERR_INVALID_ARG;
+  if ((a_fmt != FMT_BF16 && a_fmt != FMT_F16) || y_fmt < FMT_BF16 || y_fmt > FMT_F32) return DIT_ERR_INVALID_ARG;
+  if (act < 0 || act > 1) return DIT_ERR_INVALID_ARG;
+  if (residual != nullptr && (res_fmt < FMT_BF16 || res_fmt > FMT_F32)) return DIT_ERR_INVALID_ARG;
   if (M == 0) return DIT_OK;
   if (a == nullptr || w8 == nullptr || scale == nullptr || y == nullptr) return DIT_ERR_INVALID_ARG;
-  if (epilogue == EPI_RESIDUAL && residual == nullptr) return DIT_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(w8) || !aligned16(y) || !aligned16(residual)) return DIT_ERR_INVALID_ARG;
   KernelGuard g;
   if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
-  GemmArgs args{static_cast<const uint16_t*>(a), w8, scale, static_cast<uint16_t*>(y),
-                static_cast<const uint16_t*>(residual), M, N, K, epilogue, gelu_tanh};
+  GemmArgs args{a, a_fmt, w8, scale, y, y_fmt, residual, res_fmt, M, N, K, act, gelu_tanh};
   return from_cuda(launch_gemm_w8a16(args, g, as_stream(stream)));
 }
 
-int dit_qknorm_mrope(void* qkv, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
+int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                      const dit_block_config* cfg, const void* g_q, const void* g_k, void* workspace, size_t ws_bytes,
                      void* stream) {
   int st = check_config(cfg);
   if (st != DIT_OK) return st;
   if (!shape_ok(batch, n_text, grid_h, grid_w) || qkv == nullptr || g_q == nullptr || g_k == nullptr)
     return DIT_ERR_INVALID_ARG;
+  if (fmt != FMT_BF16 && fmt != FMT_F16) return DIT_ERR_INVALID_ARG;
   const int S = n_text + grid_h * grid_w;
   const size_t need = 2 * align256(static_cast<size_t>(S) * (cfg->head_dim / 2) * 4);
   if (workspace == nullptr || ws_bytes < need) return DIT_ERR_WORKSPACE;
@@ -236,19 +313,20 @@ int dit_qknorm_mrope(void* qkv, int batch, int n_text, int grid_h, int grid_w, i
   cudaError_t e = launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections,
                                     cfg->rope_theta, cos_tab, sin_tab, s);
   if (e != cudaSuccess) return DIT_ERR_CUDA;
-  return from_cuda(launch_qknorm_mrope(static_cast<uint16_t*>(qkv), batch, S, cfg->n_heads, cfg->head_dim, cos_tab,
-                                       sin_tab, static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k),
-                                       cfg->eps, s));
+  return from_cuda(launch_qknorm_mrope(qkv, fmt, batch, S, cfg->n_heads, cfg->head_dim, cos_tab, sin_tab,
+                                       static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k), cfg->eps,
+                                       s));
 }
 
-int dit_joint_attention(const void* qkv, void* out, int batch, int seq, int n_heads, int head_dim, void* stream) {
+int dit_joint_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
+                        void* stream) {
   if (batch <= 0 || seq <= 0 || n_heads <= 0 || qkv == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (fmt != FMT_BF16 && fmt != FMT_F16) return DIT_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return DIT_ERR_UNSUPPORTED;
   if (!aligned16(qkv) || !aligned16(out)) return DIT_ERR_INVALID_ARG;
   KernelGuard g;
   if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
-  return from_cuda(launch_attention(static_cast<const uint16_t*>(qkv), static_cast<uint16_t*>(out), batch, seq,
-                                    n_heads, head_dim, g, as_stream(stream)));
+  return from_cuda(launch_attention(qkv, out, fmt, batch, seq, n_heads, head_dim, g, as_stream(stream)));
 }
 
 size_t dit_block_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w) {
@@ -286,19 +364,33 @@ int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, c
   do {                                              \
     if ((expr) != cudaSuccess) return DIT_ERR_CUDA; \
   } while (0)
+  prof_mark(s, DIT_KERNEL_ROPE_TABLE);
   JAB_TRY(launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections, cfg->rope_theta,
                             ws.cos_tab, ws.sin_tab, s));
-  JAB_TRY(launch_rmsnorm(x, static_cast<const uint16_t*>(w->g_norm1), ws.h, M, d, cfg->eps, s));
-  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.h, w->w_qkv, w->s_qkv, ws.qkv, nullptr, M, 3 * d, d, EPI_NONE, 0}, g, s));
-  JAB_TRY(launch_qknorm_mrope(ws.qkv, batch, S, cfg->n_heads, cfg->head_dim, ws.cos_tab, ws.sin_tab,
+  const uint16_t* g1 = static_cast<const uint16_t*>(w->g_norm1);
+  const uint16_t* g2 = static_cast<const uint16_t*>(w->g_norm2);
+  prof_mark(s, DIT_KERNEL_RMSNORM);
+  JAB_TRY(launch_rmsnorm(x, FMT_BF16, g1, ws.h, FMT_F16, M, d, cfg->eps, s));
+  prof_mark(s, DIT_KERNEL_GEMM_QKV);
+  JAB_TRY(launch_gemm_w8a16(
+      GemmArgs{ws.h, FMT_F16, w->w_qkv, w->s_qkv, ws.qkv, FMT_F16, nullptr, -1, M, 3 * d, d, 0, 0}, g, s));
+  prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
+  JAB_TRY(launch_qknorm_mrope(ws.qkv, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, ws.cos_tab, ws.sin_tab,
                               static_cast<const uint16_t*>(w->g_q), static_cast<const uint16_t*>(w->g_k), cfg->eps,
                               s));
-  JAB_TRY(launch_attention(ws.qkv, ws.o, batch, S, cfg->n_heads, cfg->head_dim, g, s));
-  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.o, w->w_o, w->s_o, ws.x1, x, M, d, d, EPI_RESIDUAL, 0}, g, s));
-  JAB_TRY(launch_rmsnorm(ws.x1, static_cast<const uint16_t*>(w->g_norm2), ws.h, M, d, cfg->eps, s));
-  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.h, w->w_up, w->s_up, ws.u, nullptr, M, F, d, EPI_GELU, cfg->gelu_tanh}, g,
-                            s));
-  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.u, w->w_down, w->s_down, y, ws.x1, M, d, F, EPI_RESIDUAL, 0}, g, s));
+  prof_mark(s, DIT_KERNEL_ATTENTION);
+  JAB_TRY(launch_attention(ws.qkv, ws.o, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, g, s));
+  prof_mark(s, DIT_KERNEL_GEMM_O);
+  JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.o, FMT_F16, w->w_o, w->s_o, ws.x1, FMT_F32, x, FMT_BF16, M, d, d, 0, 0}, g, s));
+  prof_mark(s, DIT_KERNEL_RMSNORM);
+  JAB_TRY(launch_rmsnorm(ws.x1, FMT_F32, g2, ws.h, FMT_F16, M, d, cfg->eps, s));
+  prof_mark(s, DIT_KERNEL_GEMM_UP);
+  JAB_TRY(launch_gemm_w8a16(
+      GemmArgs{ws.h, FMT_F16, w->w_up, w->s_up, ws.u, FMT_F16, nullptr, -1, M, F, d, 1, cfg->gelu_tanh}, g, s));
+  prof_mark(s, DIT_KERNEL_GEMM_DOWN);
+  JAB_TRY(launch_gemm_w8a16(
+      GemmArgs{ws.u, FMT_F16, w->w_down, w->s_down, y, FMT_BF16, ws.x1, FMT_F32, M, d, F, 0, 0}, g, s));
+  prof_mark(s, DIT_KERNEL_END);
 #undef JAB_TRY
   return DIT_OK;
 }
@@ -323,13 +415,16 @@ int cond_proj_forward(const void* feats, int n_tok, int n_layers, int hidden, co
   KernelGuard g;
   if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
   cudaStream_t s = as_stream(stream);
-  uint16_t* normed = static_cast<uint16_t*>(workspace);
-  if (launch_rmsnorm(static_cast<const uint16_t*>(feats), static_cast<const uint16_t*>(g_norm), normed, n_tok, K, eps,
-                     s) != cudaSuccess)
+  uint16_t* normed = static_cast<uint16_t*>(workspace);  // f16 [n_tok, K]
+  prof_mark(s, DIT_KERNEL_COND_RMSNORM);
+  if (launch_rmsnorm(feats, FMT_BF16, static_cast<const uint16_t*>(g_norm), normed, FMT_F16, n_tok, K, eps, s) !=
+      cudaSuccess)
     return DIT_ERR_CUDA;
-  return from_cuda(launch_gemm_w8a16(
-      GemmArgs{normed, w, scale, static_cast<uint16_t*>(out), nullptr, n_tok, d_out, static_cast<int>(K), EPI_NONE, 0},
-      g, s));
+  prof_mark(s, DIT_KERNEL_COND_GEMM);
+  const cudaError_t e = launch_gemm_w8a16(
+      GemmArgs{normed, FMT_F16, w, scale, out, FMT_BF16, nullptr, -1, n_tok, d_out, static_cast<int>(K), 0, 0}, g, s);
+  prof_mark(s, DIT_KERNEL_END);
+  return from_cuda(e);
 }
 
 }  // extern "C"

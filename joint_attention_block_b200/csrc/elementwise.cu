@@ -61,84 +61,82 @@ __device__ float block_sum(float v, float* red) {
 // One CTA per row.  kVec 8-element vectors per thread are kept in registers
 // between the two passes when the row fits (cols <= kThreads*8*kVec); longer
 // rows (the 53,248-wide conditioning features) are re-read from L2.
-template <int kThreads, int kVec>
-__global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const uint16_t* x, const uint16_t* __restrict__ g,
-                                                           uint16_t* y, int64_t cols, float eps) {
+// XF: input format (bf16 or fp32), YF: output format (bf16 or f16).
+template <int kThreads, int kVec, int XF, int YF>
+__global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const void* x, const uint16_t* __restrict__ g, void* y,
+                                                           int64_t cols, float eps) {
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
-  uint4* yr = reinterpret_cast<uint4*>(y + row * cols);
-  const uint4* gr = reinterpret_cast<const uint4*>(g);
   const int64_t nv = cols / 8;
+  const int64_t row8 = row * nv;
   float ss = 0.f;
-  if (kVec > 0) {
-    uint4 v[kVec > 0 ? kVec : 1];
+  if constexpr (kVec > 0) {
+    float v[kVec][8];
 #pragma unroll
     for (int j = 0; j < kVec; ++j) {
       const int64_t i = threadIdx.x + static_cast<int64_t>(j) * kThreads;
-      v[j] = i < nv ? xr[i] : make_uint4(0, 0, 0, 0);
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v[j]);
+      if (i < nv) {
+        load8<XF>(x, row8 + i, v[j]);
+      } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float a = bf16_lo(p[k]), b = bf16_hi(p[k]);
-        ss = fmaf(a, a, ss);
-        ss = fmaf(b, b, ss);
+        for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
       }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ss = fmaf(v[j][k], v[j][k], ss);
     }
     const float rstd = rsqrtf(block_sum<kThreads>(ss, red) / static_cast<float>(cols) + eps);
 #pragma unroll
     for (int j = 0; j < kVec; ++j) {
       const int64_t i = threadIdx.x + static_cast<int64_t>(j) * kThreads;
       if (i >= nv) break;
-      const uint4 gv = gr[i];
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v[j]);
-      const uint32_t* q = reinterpret_cast<const uint32_t*>(&gv);
-      uint4 o;
-      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+      float gv[8], o[8];
+      load8<FMT_BF16>(g, i, gv);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        op[k] = pack_bf16x2(bf16_lo(p[k]) * rstd * bf16_lo(q[k]), bf16_hi(p[k]) * rstd * bf16_hi(q[k]));
-      yr[i] = o;
+      for (int k = 0; k < 8; ++k) o[k] = v[j][k] * rstd * gv[k];
+      store8<YF>(y, row8 + i, o);
     }
   } else {
     for (int64_t i = threadIdx.x; i < nv; i += kThreads) {
-      const uint4 v = xr[i];
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v);
+      float v[8];
+      load8<XF>(x, row8 + i, v);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float a = bf16_lo(p[k]), b = bf16_hi(p[k]);
-        ss = fmaf(a, a, ss);
-        ss = fmaf(b, b, ss);
-      }
+      for (int k = 0; k < 8; ++k) ss = fmaf(v[k], v[k], ss);
     }
     const float rstd = rsqrtf(block_sum<kThreads>(ss, red) / static_cast<float>(cols) + eps);
     for (int64_t i = threadIdx.x; i < nv; i += kThreads) {
-      const uint4 v = xr[i];
-      const uint4 gv = gr[i];
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v);
-      const uint32_t* q = reinterpret_cast<const uint32_t*>(&gv);
-      uint4 o;
-      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+      float v[8], gv[8], o[8];
+      load8<XF>(x, row8 + i, v);
+      load8<FMT_BF16>(g, i, gv);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        op[k] = pack_bf16x2(bf16_lo(p[k]) * rstd * bf16_lo(q[k]), bf16_hi(p[k]) * rstd * bf16_hi(q[k]));
-      yr[i] = o;
+      for (int k = 0; k < 8; ++k) o[k] = v[k] * rstd * gv[k];
+      store8<YF>(y, row8 + i, o);
     }
   }
 }
 
-cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* g, uint16_t* y, int64_t rows, int64_t cols, float eps,
-                           cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
+template <int XF, int YF>
+static void rmsnorm_dispatch(const void* x, const uint16_t* g, void* y, int64_t rows, int64_t cols, float eps,
+                             cudaStream_t s) {
+  const unsigned r = static_cast<unsigned>(rows);
   if (cols <= 256 * 8 * 1) {
-    rmsnorm_kernel<256, 1><<<static_cast<unsigned>(rows), 256, 0, s>>>(x, g, y, cols, eps);
+    rmsnorm_kernel<256, 1, XF, YF><<<r, 256, 0, s>>>(x, g, y, cols, eps);
   } else if (cols <= 256 * 8 * 2) {
-    rmsnorm_kernel<256, 2><<<static_cast<unsigned>(rows), 256, 0, s>>>(x, g, y, cols, eps);
+    rmsnorm_kernel<256, 2, XF, YF><<<r, 256, 0, s>>>(x, g, y, cols, eps);
   } else if (cols <= 256 * 8 * 4) {
-    rmsnorm_kernel<256, 4><<<static_cast<unsigned>(rows), 256, 0, s>>>(x, g, y, cols, eps);
+    rmsnorm_kernel<256, 4, XF, YF><<<r, 256, 0, s>>>(x, g, y, cols, eps);
   } else {
-    rmsnorm_kernel<512, 0><<<static_cast<unsigned>(rows), 512, 0, s>>>(x, g, y, cols, eps);
+    rmsnorm_kernel<512, 0, XF, YF><<<r, 512, 0, s>>>(x, g, y, cols, eps);
   }
+}
+
+cudaError_t launch_rmsnorm(const void* x, int x_fmt, const uint16_t* g, void* y, int y_fmt, int64_t rows, int64_t cols,
+                           float eps, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (x_fmt == FMT_BF16 && y_fmt == FMT_BF16) rmsnorm_dispatch<FMT_BF16, FMT_BF16>(x, g, y, rows, cols, eps, s);
+  else if (x_fmt == FMT_BF16 && y_fmt == FMT_F16) rmsnorm_dispatch<FMT_BF16, FMT_F16>(x, g, y, rows, cols, eps, s);
+  else if (x_fmt == FMT_F32 && y_fmt == FMT_F16) rmsnorm_dispatch<FMT_F32, FMT_F16>(x, g, y, rows, cols, eps, s);
+  else if (x_fmt == FMT_F32 && y_fmt == FMT_BF16) rmsnorm_dispatch<FMT_F32, FMT_BF16>(x, g, y, rows, cols, eps, s);
+  else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
@@ -260,6 +258,8 @@ cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, con
 // ------------------------------------------------------------------ QK-RMSNorm + M-RoPE (standalone)
 
 // One warp per (batch, token, head, q|k); lane l owns rotary pairs l, l+32, ...
+// F: storage format of the qkv buffer (bf16 or f16).
+template <int F>
 __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int seq, int n_heads, int head_dim,
                                     const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
                                     const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
@@ -282,8 +282,8 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int s
   for (int j = 0; j < 2; ++j) {
     if (j < np) {
       const int i = lane + 32 * j;
-      a[j] = __uint_as_float(static_cast<uint32_t>(v[i]) << 16);
-      b[j] = __uint_as_float(static_cast<uint32_t>(v[i + half]) << 16);
+      a[j] = unpack_lo<F>(v[i]);
+      b[j] = unpack_lo<F>(v[i + half]);
       ss = fmaf(a[j], a[j], fmaf(b[j], b[j], ss));
     }
   }
@@ -293,25 +293,32 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int s
   for (int j = 0; j < 2; ++j) {
     if (j < np) {
       const int i = lane + 32 * j;
-      const float x1 = a[j] * rstd * __uint_as_float(static_cast<uint32_t>(g[i]) << 16);
-      const float x2 = b[j] * rstd * __uint_as_float(static_cast<uint32_t>(g[i + half]) << 16);
+      const float x1 = a[j] * rstd * bf16_lo(g[i]);
+      const float x2 = b[j] * rstd * bf16_lo(g[i + half]);
       const float c = cos_tab[static_cast<int64_t>(s) * half + i];
       const float sn = sin_tab[static_cast<int64_t>(s) * half + i];
-      const uint32_t o = pack_bf16x2(x1 * c - x2 * sn, x2 * c + x1 * sn);
+      const uint32_t o = pack2<F>(x1 * c - x2 * sn, x2 * c + x1 * sn);
       v[i] = static_cast<uint16_t>(o & 0xFFFFu);
       v[i + half] = static_cast<uint16_t>(o >> 16);
     }
   }
 }
 
-cudaError_t launch_qknorm_mrope(uint16_t* qkv, int batch, int seq, int n_heads, int head_dim, const float* cos_tab,
-                                const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k, float eps,
-                                cudaStream_t s) {
+cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
+                                const float* cos_tab, const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k,
+                                float eps, cudaStream_t s) {
   const int64_t warps = static_cast<int64_t>(batch) * seq * n_heads * 2;
   if (warps <= 0) return cudaSuccess;
-  const int64_t blocks = (warps * 32 + 255) / 256;
-  qknorm_mrope_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(qkv, batch, seq, n_heads, head_dim, cos_tab,
-                                                                    sin_tab, g_q, g_k, eps);
+  const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+  uint16_t* q = static_cast<uint16_t*>(qkv);
+  if (fmt == FMT_F16)
+    qknorm_mrope_kernel<FMT_F16><<<blocks, 256, 0, s>>>(q, batch, seq, n_heads, head_dim, cos_tab, sin_tab, g_q, g_k,
+                                                        eps);
+  else if (fmt == FMT_BF16)
+    qknorm_mrope_kernel<FMT_BF16><<<blocks, 256, 0, s>>>(q, batch, seq, n_heads, head_dim, cos_tab, sin_tab, g_q, g_k,
+                                                         eps);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

@@ -6,11 +6,13 @@
 // fp8 * weight_scale[:, None]).  Both operands are K-major, so the problem is the
 // "TN" GEMM tcgen05 reads natively.
 //
-// The checkpoint's numerics are W8 dequantised, activations bf16.  e4m3 is a
-// subset of bf16, so each weight tile is widened to bf16 on chip, exactly, and
-// fed to tcgen05.mma kind::f16 with an fp32 accumulator in TMEM; the per-row
+// The checkpoint's numerics are W8 dequantised, activations 16-bit.  e4m3 is a
+// subset of both bf16 and f16, so each weight tile is widened on chip, exactly,
+// to the activation format (bf16, or f16 for the block's internal activations)
+// and fed to tcgen05.mma kind::f16 with an fp32 accumulator in TMEM; the per-row
 // scale is applied once per output in the epilogue (scale[n] * sum_k a*w8 is
-// sum_k a*(w8*scale[n]) up to rounding).
+// sum_k a*(w8*scale[n]) up to rounding).  The epilogue writes bf16, f16 or fp32
+// and can add a bf16 / f16 / fp32 residual.
 //
 // CTA tile 128 x 256 x 64, one CTA per output tile.  Warp roles:
 //   warp 0      TMA producer: A tile (128 x 64 bf16, 128B swizzle) and the raw
@@ -46,10 +48,12 @@ constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte align
 
 struct Params {
   const float* scale;
-  uint16_t* y;
-  const uint16_t* residual;
+  void* y;
+  const void* residual;
   int M, N, K;
-  int epilogue;
+  int y_fmt;    // FMT_BF16 / FMT_F16 / FMT_F32
+  int res_fmt;  // -1 none, FMT_BF16 / FMT_F16 / FMT_F32
+  int act;      // 0 none, 1 GELU
   int gelu_tanh;
 };
 
@@ -61,6 +65,7 @@ __device__ __forceinline__ float gelu_f(float x, int tanh_form) {
   return 0.5f * x * (1.f + erff(x * 0.7071067811865476f));
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_w8a16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const Params p, const KernelGuard guard) {
@@ -137,7 +142,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
+    constexpr uint32_t idesc = idesc_f16kind(BM, BN, F16, false, false);
     bool ok = true;
     for (int kb = 0; kb < num_kb && ok; ++kb) {
       const int s = kb % RAW_STAGES;
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(a0 + kk * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-          mma_bf16_ss(tmem_acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          mma_f16kind_ss(tmem_acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
         mma_commit(&raw_empty[s]);
         mma_commit(&cvt_empty[c]);
@@ -189,10 +194,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = chunk & 3;
         const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
         uint4 o0, o1;
-        e4m3x4_to_bf16x4(v.x, o0.x, o0.y);
-        e4m3x4_to_bf16x4(v.y, o0.z, o0.w);
-        e4m3x4_to_bf16x4(v.z, o1.x, o1.y);
-        e4m3x4_to_bf16x4(v.w, o1.z, o1.w);
+        e4m3x4_to_16x4<F16>(v.x, o0.x, o0.y);
+        e4m3x4_to_16x4<F16>(v.y, o0.z, o0.w);
+        e4m3x4_to_16x4<F16>(v.z, o1.x, o1.y);
+        e4m3x4_to_16x4<F16>(v.w, o1.z, o1.w);
         uint8_t* row = dst + r * 128;
         *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) << 4)) = o0;
         *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) << 4)) = o1;
@@ -220,34 +225,31 @@ __global__ void __launch_bounds__(THREADS, 1)
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * sScale[cc * 32 + j];
-        if (p.epilogue == EPI_GELU) {
+        if (p.act == 1) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], p.gelu_tanh);
         }
         if (row_ok) {
-          const size_t off = static_cast<size_t>(row) * p.N + col0;
-          if (p.epilogue == EPI_RESIDUAL) {
-            const uint4* rp = reinterpret_cast<const uint4*>(p.residual + off);
+          const int64_t off8 = (static_cast<int64_t>(row) * p.N + col0) / 8;
+          if (p.res_fmt >= 0) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint4 rv = rp[q];
-              const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rv);
+              float rv[8];
+              if (p.res_fmt == FMT_F32) load8<FMT_F32>(p.residual, off8 + q, rv);
+              else if (p.res_fmt == FMT_F16) load8<FMT_F16>(p.residual, off8 + q, rv);
+              else load8<FMT_BF16>(p.residual, off8 + q, rv);
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                v[q * 8 + 2 * k] += bf16_lo(rw[k]);
-                v[q * 8 + 2 * k + 1] += bf16_hi(rw[k]);
-              }
+              for (int k = 0; k < 8; ++k) v[q * 8 + k] += rv[k];
             }
           }
-          uint4* yp = reinterpret_cast<uint4*>(p.y + off);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 o;
-            o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-            o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-            o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-            o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-            yp[q] = o;
+            float ov[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ov[k] = v[q * 8 + k];
+            if (p.y_fmt == FMT_F32) store8<FMT_F32>(p.y, off8 + q, ov);
+            else if (p.y_fmt == FMT_F16) store8<FMT_F16>(p.y, off8 + q, ov);
+            else store8<FMT_BF16>(p.y, off8 + q, ov);
           }
         }
       }
@@ -267,13 +269,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStream_t s) {
   using namespace gemm;
   if (a.M <= 0 || a.N <= 0) return cudaSuccess;
+  const bool f16 = a.a_fmt == FMT_F16;
   CUtensorMap tm_a, tm_b;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
     const uint32_t box[2] = {BK, BM};
-    if (!make_tmap(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.a), dims, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_tmap(&tm_a, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(a.a), dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   {
@@ -284,11 +287,12 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
                    CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(gemm_w8a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  Params p{a.scale, a.y, a.residual, a.M, a.N, a.K, a.epilogue, a.gelu_tanh};
+  Params p{a.scale, a.y, a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1, a.act, a.gelu_tanh};
   dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN);
-  gemm_w8a16_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tm_a, tm_b, p, g);
+  auto kern = f16 ? gemm_w8a16_kernel<true> : gemm_w8a16_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, THREADS, SMEM_BYTES, s>>>(tm_a, tm_b, p, g);
   return cudaGetLastError();
 }
 

@@ -37,8 +37,9 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base
 
 // ---- launchers (return cudaSuccess or the launch error) ----
 cudaError_t launch_e4m3_to_bf16(const uint8_t* codes, uint16_t* out, int64_t n, cudaStream_t s);
-cudaError_t launch_rmsnorm(const uint16_t* x, const uint16_t* g, uint16_t* y, int64_t rows, int64_t cols, float eps,
-                           cudaStream_t s);
+// y = RMSNorm(x) * g; x in x_fmt (bf16 / f32), y in y_fmt (bf16 / f16), g bf16.
+cudaError_t launch_rmsnorm(const void* x, int x_fmt, const uint16_t* g, void* y, int y_fmt, int64_t rows, int64_t cols,
+                           float eps, cudaStream_t s);
 cudaError_t launch_euler_cfg(float* x, const uint16_t* vc, const uint16_t* vu, int64_t n, float g, float dt,
                              cudaStream_t s);
 cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos, cudaStream_t s);
@@ -46,26 +47,30 @@ cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int3
 cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, int head_dim,
                               const int32_t sections[3], float theta, float* cos_tab, float* sin_tab,
                               cudaStream_t s);
-cudaError_t launch_qknorm_mrope(uint16_t* qkv, int batch, int seq, int n_heads, int head_dim, const float* cos_tab,
-                                const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k, float eps,
-                                cudaStream_t s);
+cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
+                                const float* cos_tab, const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k,
+                                float eps, cudaStream_t s);
 
-// GEMM epilogues.
-enum GemmEpilogue : int { EPI_NONE = 0, EPI_GELU = 1, EPI_RESIDUAL = 2 };
+// Activation storage formats (the ABI's format codes).
+enum Fmt : int { FMT_BF16 = 0, FMT_F16 = 1, FMT_F32 = 2 };
 
 struct GemmArgs {
-  const uint16_t* a;  // bf16 [M, K]
-  const uint8_t* w;   // e4m3 [N, K]
-  const float* scale; // [N]
-  uint16_t* y;        // bf16 [M, N]
-  const uint16_t* residual;  // bf16 [M, N] or null
+  const void* a;       // [M, K], a_fmt (bf16 or f16)
+  int a_fmt;
+  const uint8_t* w;    // e4m3 [N, K]
+  const float* scale;  // [N]
+  void* y;             // [M, N], y_fmt
+  int y_fmt;
+  const void* residual;  // [M, N], res_fmt, or null
+  int res_fmt;
   int M, N, K;
-  int epilogue;
+  int act;        // 0 none, 1 GELU
   int gelu_tanh;
 };
 cudaError_t launch_gemm_w8a16(const GemmArgs& args, const KernelGuard& g, cudaStream_t s);
 
-cudaError_t launch_attention(const uint16_t* qkv, uint16_t* out, int batch, int seq, int n_heads, int head_dim,
+// qkv and out in fmt (bf16 or f16).
+cudaError_t launch_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
                              const KernelGuard& g, cudaStream_t s);
 
 }  // namespace jab

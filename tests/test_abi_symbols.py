@@ -59,8 +59,12 @@ def test_argument_validation_without_gpu(lib):
     assert lib.dit_block_forward(ctypes.byref(hd96), ctypes.byref(w), 16, 32, 1, 16, 8, 8, -1, None, None, 0, None) == 2
     assert lib.euler_cfg_step(None, None, None, 8, 4.0, -0.02, None) == 1
     assert lib.euler_cfg_step(None, None, None, 0, 4.0, -0.02, None) == 1 or True
-    assert lib.dit_gemm_w8a16(16, 16, 16, 16, None, 128, 100, 64, 0, 0, None) == 2  # N % 32 != 0
-    assert lib.dit_gemm_w8a16(16, 16, 16, 16, None, 128, 128, 64, 2, 0, None) == 1  # residual missing
-    assert lib.dit_gemm_w8a16(17, 16, 16, 16, None, 128, 128, 64, 0, 0, None) == 1  # misaligned A
+    assert lib.dit_gemm_w8a16(16, 0, 16, 16, 16, 0, None, 0, 128, 100, 64, 0, 0, None) == 2  # N % 32 != 0
+    assert lib.dit_gemm_w8a16(16, 2, 16, 16, 16, 0, None, 0, 128, 128, 64, 0, 0, None) == 1  # A cannot be fp32
+    assert lib.dit_gemm_w8a16(17, 0, 16, 16, 16, 0, None, 0, 128, 128, 64, 0, 0, None) == 1  # misaligned A
+    assert lib.dit_gemm_w8a16(16, 0, 16, 16, 16, 0, 32, 7, 128, 128, 64, 0, 0, None) == 1  # bad residual format
     assert lib.cond_proj_forward(16, 4, 13, 4096, 16, 1e-6, 16, 16, 4096, 16, None, 0, None) == 3  # no workspace
-    assert lib.dit_rmsnorm_rows(16, 16, 16, 4, 12, 1e-6, None) == 1  # cols % 8
+    assert lib.dit_rmsnorm_rows(16, 0, 16, 16, 0, 4, 12, 1e-6, None) == 1  # cols % 8
+    assert lib.dit_rmsnorm_rows(16, 0, 16, 16, 1, 4, 16, 1e-6, None) == 1  # in place with a format change
+    assert lib.dit_joint_attention(16, 32, 2, 1, 8, 2, 64, None) == 1  # fp32 q/k/v
+    assert lib.dit_joint_attention(16, 32, 1, 1, 8, 2, 96, None) == 2  # head_dim 96

@@ -32,15 +32,23 @@ def test_e4m3_to_bf16_every_code_bit_exact():
 
 
 @pytest.mark.parametrize("rows,cols", [(3, 256), (5, 4096), (2, 8200), (3, 53248)])
-def test_rmsnorm_rows(rows, cols):
-    x = synth.to_bf16_bits(synth.normal(7, rows, (rows, cols), std=2.0))
+@pytest.mark.parametrize("x_fmt,y_fmt", [(0, 0), (0, 1), (2, 1), (2, 0)], ids=["bf16-bf16", "bf16-f16", "f32-f16", "f32-bf16"])
+def test_rmsnorm_rows(rows, cols, x_fmt, y_fmt):
+    xf = synth.normal(7, rows, (rows, cols), std=2.0)
     g = synth.to_bf16_bits(synth.normal(7, 100 + rows, (cols,), std=0.05, mean=1.0))
-    y = empty_bf16(rows, cols)
-    ops.rmsnorm_rows(dev(x), dev(g), y, 1e-6)
-    ref = oracle.rmsnorm(oracle.bf16_to_f64(x), oracle.bf16_to_f64(g), 1e-6)
-    got = as_f64(y)
-    # one bf16 rounding of an fp32 result: |d| <= 2^-8 |ref|
-    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
+    if x_fmt == 0:
+        x_np = synth.to_bf16_bits(xf)
+        x_val = oracle.bf16_to_f64(x_np)
+    else:
+        x_np = xf.astype(np.float32)
+        x_val = x_np.astype(np.float64)
+    y = torch.empty(rows, cols, dtype=torch.int16 if y_fmt == 0 else torch.float16, device="cuda")
+    ops.rmsnorm_rows(dev(x_np), dev(g), y, 1e-6, x_fmt=x_fmt, y_fmt=y_fmt)
+    ref = oracle.rmsnorm(x_val, oracle.bf16_to_f64(g), 1e-6)
+    got = as_f64(y) if y_fmt == 0 else y.cpu().numpy().astype(np.float64)
+    # one 16-bit rounding of an fp32 result: |d| <= 2^-8 |ref| (bf16), 2^-11 |ref| (f16)
+    ulp = 2.0 ** -8 if y_fmt == 0 else 2.0 ** -11
+    assert np.all(np.abs(got - ref) <= ulp * np.abs(ref) + 1e-7)
 
 
 @pytest.mark.parametrize("n_text,gh,gw,t_img", [(16, 8, 8, -1), (512, 64, 64, -1), (0, 3, 5, -1), (1, 1, 1, 7), (4, 0, 0, -1)])
@@ -73,20 +81,45 @@ def _gemm_case(M, N, K, seed):
     return a, codes, scale, res
 
 
+def _fmt_tensor(vals: np.ndarray, fmt: int) -> torch.Tensor:
+    if fmt == 0:
+        return dev(synth.to_bf16_bits(vals))
+    if fmt == 1:
+        return torch.from_numpy(vals.astype(np.float16)).cuda()
+    return torch.from_numpy(vals.astype(np.float32)).cuda()
+
+
+def _fmt_values(t: torch.Tensor, fmt: int) -> np.ndarray:
+    return as_f64(t) if fmt == 0 else t.cpu().numpy().astype(np.float64)
+
+
+def _fmt_empty(shape, fmt: int) -> torch.Tensor:
+    return torch.empty(*shape, dtype=(torch.int16, torch.float16, torch.float32)[fmt], device="cuda")
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 512, 256), (37, 768, 1024), (300, 288, 528)])
-@pytest.mark.parametrize("epi", [0, 1, 2])
-def test_gemm_w8a16(M, N, K, epi):
-    a, codes, scale, res = _gemm_case(M, N, K, seed=M + N + K + epi)
-    y = empty_bf16(M, N)
-    ops.gemm_w8a16(dev(a), dev(codes), dev(scale), y, residual=dev(res) if epi == 2 else None, epilogue=epi)
-    ref = oracle.bf16_to_f64(a) @ oracle.dequant(codes, scale).T
-    if epi == 1:
+@pytest.mark.parametrize("a_fmt,y_fmt,act,res_fmt", [
+    (0, 0, 0, None), (0, 0, 1, None), (0, 0, 0, 0),  # bf16 in / out
+    (1, 1, 0, None), (1, 2, 0, 0), (1, 1, 1, None), (1, 0, 0, 2),  # the block's four GEMMs
+], ids=["bf16", "bf16-gelu", "bf16-res", "qkv", "oproj", "up-gelu", "down"])
+def test_gemm_w8a16(M, N, K, a_fmt, y_fmt, act, res_fmt):
+    r = np.random.default_rng(M + N + K + 10 * a_fmt + y_fmt + act)
+    a_vals = r.standard_normal((M, K)).astype(np.float32)
+    codes, scale = synth.quantize_rows_e4m3((r.standard_normal((N, K)) * 0.02).astype(np.float32))
+    a_t = _fmt_tensor(a_vals, a_fmt)
+    a_exact = _fmt_values(a_t, a_fmt)
+    res_t = None if res_fmt is None else _fmt_tensor(r.standard_normal((M, N)).astype(np.float32), res_fmt)
+    y = _fmt_empty((M, N), y_fmt)
+    ops.gemm_w8a16(a_t, dev(codes), dev(scale), y, residual=res_t, act=act, a_fmt=a_fmt, y_fmt=y_fmt,
+                   res_fmt=0 if res_fmt is None else res_fmt)
+    ref = a_exact @ oracle.dequant(codes, scale).T
+    if act == 1:
         ref = oracle.gelu(ref)
-    if epi == 2:
-        ref = ref + oracle.bf16_to_f64(res)
-    got = as_f64(y)
-    # fp32 accumulation of exact products, one bf16 rounding at the end
-    assert_close(got, ref, max_rel=8e-3, mean_rel=3e-3, what=f"gemm {M}x{N}x{K} epi{epi}")
+    if res_t is not None:
+        ref = ref + _fmt_values(res_t, res_fmt)
+    got = _fmt_values(y, y_fmt)
+    # fp32 accumulation of exact products, one rounding to the output format
+    assert_close(got, ref, max_rel=8e-3, mean_rel=2e-3, what=f"gemm {M}x{N}x{K}")
 
 
 def test_gemm_dequant_is_exact_inside_the_mma():
@@ -94,11 +127,12 @@ def test_gemm_dequant_is_exact_inside_the_mma():
     K = N = 256
     finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
     codes = np.resize(finite, (N, K)).astype(np.uint8)
-    a = synth.to_bf16_bits(np.eye(K, dtype=np.float32))
-    y = empty_bf16(K, N)
-    ops.gemm_w8a16(dev(a), dev(codes), dev(np.ones(N, dtype=np.float32)), y)
     want = oracle.e4m3_to_f64(codes).T
-    assert np.array_equal(as_f64(y), want)
+    for a_fmt in (0, 1):
+        a = _fmt_tensor(np.eye(K, dtype=np.float32), a_fmt)
+        y = _fmt_empty((K, N), 2)
+        ops.gemm_w8a16(a, dev(codes), dev(np.ones(N, dtype=np.float32)), y, a_fmt=a_fmt, y_fmt=2)
+        assert np.array_equal(_fmt_values(y, 2), want), f"a_fmt={a_fmt}"
 
 
 def _tiny_qkv(shape, seed=3, n_text=None, gh=None, gw=None, batch=1):
@@ -111,37 +145,39 @@ def _tiny_qkv(shape, seed=3, n_text=None, gh=None, gw=None, batch=1):
 
 
 @pytest.mark.parametrize("shape", [synth.TINY, synth.C1024], ids=["tiny", "hd128"])
-def test_qknorm_mrope(shape):
-    import ctypes
+@pytest.mark.parametrize("fmt", [0, 1], ids=["bf16", "f16"])
+def test_qknorm_mrope(shape, fmt):
     cfg = ops.make_config(shape)
     if shape is synth.C1024:
         qkv_np, n_text, gh, gw, S = _tiny_qkv(shape, n_text=37, gh=9, gw=11)
     else:
         qkv_np, n_text, gh, gw, S = _tiny_qkv(shape)
-    w = synth.block_inputs(synth.TINY) if shape is synth.TINY else None
     r = np.random.default_rng(5)
     gq = synth.to_bf16_bits(1 + 0.05 * r.standard_normal(shape.head_dim))
     gk = synth.to_bf16_bits(1 + 0.05 * r.standard_normal(shape.head_dim))
-    qkv = dev(qkv_np)
-    ops.qknorm_mrope(qkv, cfg, n_text, gh, gw, dev(gq), dev(gk), workspace(2 * S * shape.head_dim * 4 + 1024))
-    got = oracle.bf16_to_f64(bits(qkv)).reshape(1, S, 3, shape.n_heads, shape.head_dim)
-    x = oracle.bf16_to_f64(qkv_np).reshape(1, S, 3, shape.n_heads, shape.head_dim)
+    vals = oracle.bf16_to_f64(qkv_np).astype(np.float32)
+    qkv = _fmt_tensor(vals, fmt)
+    before = qkv.clone()
+    ops.qknorm_mrope(qkv, cfg, n_text, gh, gw, dev(gq), dev(gk), workspace(2 * S * shape.head_dim * 4 + 1024), fmt=fmt)
+    got = _fmt_values(qkv, fmt).reshape(1, S, 3, shape.n_heads, shape.head_dim)
+    x = _fmt_values(before, fmt).reshape(1, S, 3, shape.n_heads, shape.head_dim)
     pos = oracle.mrope_positions(n_text, gh, gw)
     for which, g in ((0, gq), (1, gk)):
         ref = oracle.mrope(oracle.rmsnorm(x[0, :, which], oracle.bf16_to_f64(g), shape.eps), pos, shape.rope_sections, shape.rope_theta)
         assert np.max(np.abs(got[0, :, which] - ref)) <= 2.0 ** -7 * np.abs(ref).max()
-    assert np.array_equal(bits(qkv).reshape(1, S, 3, -1)[:, :, 2], qkv_np.reshape(1, S, 3, -1)[:, :, 2])
+    assert torch.equal(qkv.view(1, S, 3, -1)[:, :, 2], before.view(1, S, 3, -1)[:, :, 2])
 
 
 @pytest.mark.parametrize("S,H,hd,batch", [(80, 4, 64, 1), (300, 2, 128, 1), (1, 2, 128, 1), (129, 1, 64, 2), (640, 2, 128, 1)])
-def test_joint_attention(S, H, hd, batch):
+@pytest.mark.parametrize("fmt", [0, 1], ids=["bf16", "f16"])
+def test_joint_attention(S, H, hd, batch, fmt):
     d = H * hd
     r = np.random.default_rng(S * 7 + H)
-    qkv_np = synth.to_bf16_bits((r.standard_normal((batch, S, 3 * d)) * 1.5).astype(np.float32))
-    out = empty_bf16(batch, S, d)
-    ops.joint_attention(dev(qkv_np), out, H, hd)
-    x = oracle.bf16_to_f64(qkv_np).reshape(batch, S, 3, H, hd)
-    got = as_f64(out).reshape(batch, S, H, hd)
+    qkv = _fmt_tensor((r.standard_normal((batch, S, 3 * d)) * 1.5).astype(np.float32), fmt)
+    out = _fmt_empty((batch, S, d), fmt)
+    ops.joint_attention(qkv, out, H, hd, fmt=fmt)
+    x = _fmt_values(qkv, fmt).reshape(batch, S, 3, H, hd)
+    got = _fmt_values(out, fmt).reshape(batch, S, H, hd)
     for b in range(batch):
         ref = oracle.attention(x[b, :, 0], x[b, :, 1], x[b, :, 2])
         assert_close(got[b], ref, max_rel=2e-2, mean_rel=3e-3, what=f"attention S={S} H={H} hd={hd}")
