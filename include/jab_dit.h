@@ -101,7 +101,8 @@ DIT_API int dit_block_forward(const dit_block_config* cfg, const dit_block_weigh
                       int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                       void* workspace, size_t ws_bytes, void* stream);
 
-/* Bytes of device workspace cond_proj_forward needs. */
+/* Bytes of device workspace cond_proj_forward needs: the normalised features (f16) and,
+ * when the token count leaves SMs idle, fp32 split-K partial sums of the projection. */
 DIT_API size_t cond_proj_workspace_bytes(int n_tok, int n_layers, int hidden, int d_out);
 
 /* llm_cond_norm + llm_cond_proj (SimpleTuner Ideogram 4 quickstart, "Text Embed Cache"):
@@ -182,7 +183,8 @@ typedef enum {
   DIT_KERNEL_GEMM_DOWN = 8,
   DIT_KERNEL_COND_RMSNORM = 9,
   DIT_KERNEL_COND_GEMM = 10,
-  DIT_KERNEL_EULER_CFG = 11
+  DIT_KERNEL_EULER_CFG = 11,
+  DIT_KERNEL_COND_REDUCE = 12
 } dit_kernel_tag;
 DIT_API int dit_profile_enable(int max_marks);
 DIT_API int dit_profile_disable(void);

@@ -213,7 +213,8 @@ def joint_attention(qkv: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim
 
 
 KERNEL_TAGS = {1: "rope_table", 2: "rmsnorm", 3: "gemm_qkv", 4: "qknorm_mrope", 5: "attention", 6: "gemm_o",
-               7: "gemm_up", 8: "gemm_down", 9: "cond_rmsnorm", 10: "cond_gemm", 11: "euler_cfg"}
+               7: "gemm_up", 8: "gemm_down", 9: "cond_rmsnorm", 10: "cond_gemm", 11: "euler_cfg",
+               12: "cond_reduce"}
 
 
 def profile_enable(max_marks: int) -> None:

@@ -397,7 +397,12 @@ int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, c
 
 size_t cond_proj_workspace_bytes(int n_tok, int n_layers, int hidden, int d_out) {
   if (n_tok <= 0 || n_layers <= 0 || hidden <= 0 || d_out <= 0) return 0;
-  return align256(static_cast<size_t>(n_tok) * n_layers * hidden * 2);
+  const int64_t K = static_cast<int64_t>(n_layers) * hidden;
+  if (K > (1 << 30)) return 0;
+  const int splits = gemm_pick_splits(n_tok, d_out, static_cast<int>(K));
+  size_t bytes = align256(static_cast<size_t>(n_tok) * K * 2);
+  if (splits > 1) bytes += align256(static_cast<size_t>(splits) * n_tok * d_out * 4);
+  return bytes;
 }
 
 int cond_proj_forward(const void* feats, int n_tok, int n_layers, int hidden, const void* g_norm, float eps,
@@ -420,9 +425,24 @@ int cond_proj_forward(const void* feats, int n_tok, int n_layers, int hidden, co
   if (launch_rmsnorm(feats, FMT_BF16, static_cast<const uint16_t*>(g_norm), normed, FMT_F16, n_tok, K, eps, s) !=
       cudaSuccess)
     return DIT_ERR_CUDA;
+  const int splits = gemm_pick_splits(n_tok, d_out, static_cast<int>(K));
   prof_mark(s, DIT_KERNEL_COND_GEMM);
-  const cudaError_t e = launch_gemm_w8a16(
-      GemmArgs{normed, FMT_F16, w, scale, out, FMT_BF16, nullptr, -1, n_tok, d_out, static_cast<int>(K), 0, 0}, g, s);
+  cudaError_t e;
+  if (splits > 1) {
+    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           align256(static_cast<size_t>(n_tok) * K * 2));
+    GemmArgs ga{normed, FMT_F16, w, scale, part, FMT_F32, nullptr, -1, n_tok, d_out, static_cast<int>(K), 0, 0};
+    ga.k_splits = splits;
+    e = launch_gemm_w8a16(ga, g, s);
+    if (e == cudaSuccess) {
+      prof_mark(s, DIT_KERNEL_COND_REDUCE);
+      e = launch_splitk_reduce(part, static_cast<uint16_t*>(out), static_cast<int64_t>(n_tok) * d_out, splits, s);
+    }
+  } else {
+    e = launch_gemm_w8a16(
+        GemmArgs{normed, FMT_F16, w, scale, out, FMT_BF16, nullptr, -1, n_tok, d_out, static_cast<int>(K), 0, 0}, g,
+        s);
+  }
   prof_mark(s, DIT_KERNEL_END);
   return from_cuda(e);
 }

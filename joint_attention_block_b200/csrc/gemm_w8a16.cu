@@ -15,12 +15,14 @@
 // and can add a bf16 / f16 / fp32 residual.
 //
 // CTA tile 128 x 256 x 64, one CTA per output tile.  Warp roles:
-//   warp 0      TMA producer: A tile (128 x 64 bf16, 128B swizzle) and the raw
-//               W8 tile (256 x 64 bytes) into a 4-stage ring.
+//   warp 0      TMA producer: A tile (128 x 64, 128B swizzle) and the raw W8 tile
+//               (256 x 64 bytes) into a 4-stage ring.
 //   warp 1      TMEM allocation; one lane issues the MMAs (4 x K=16 per stage).
-//   warps 2..5  convert W8 -> bf16 into the 128B-swizzled K-major layout the MMA
-//               reads (2-stage ring), then run the epilogue: tcgen05.ld of the
-//               accumulator, scale, optional GELU / residual, bf16 stores.
+//   warps 2..9  convert W8 -> 16-bit into the 128B-swizzled K-major layout the MMA
+//               reads (2-stage ring; two converter warps per scheduler to hide the
+//               conversion latency), then run the epilogue: tcgen05.ld of the
+//               accumulator (warp w reads TMEM lanes 32*(w%4).., column half
+//               (w-2)/4), scale, optional GELU / residual, stores.
 #include "common.cuh"
 
 namespace jab {
@@ -34,7 +36,8 @@ constexpr int CVT_STAGES = 2;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B8_BYTES = BN * BK;
 constexpr int B16_BYTES = BN * BK * 2;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
+constexpr int CVT_WARPS = 8;
 constexpr int TMEM_COLS = 256;
 
 constexpr int OFF_A = 0;
@@ -55,6 +58,8 @@ struct Params {
   int res_fmt;  // -1 none, FMT_BF16 / FMT_F16 / FMT_F32
   int act;      // 0 none, 1 GELU
   int gelu_tanh;
+  int kb_per_split;          // k-blocks per split (grid.z splits); all of K when not split
+  int64_t y_split_stride;    // elements between the fp32 partial outputs of consecutive splits
 };
 
 __device__ __forceinline__ float gelu_f(float x, int tanh_form) {
@@ -89,15 +94,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int lane = static_cast<int>(lane_id());
   const int tile_m = blockIdx.x;
   const int tile_n = blockIdx.y;
-  const int num_kb = (p.K + BK - 1) / BK;
+  const int kb_total = (p.K + BK - 1) / BK;
+  const int kb0 = blockIdx.z * p.kb_per_split;
+  const int num_kb = min(kb_total - kb0, p.kb_per_split);
+  void* const y_out = static_cast<char*>(p.y) + blockIdx.z * p.y_split_stride * 4;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < RAW_STAGES; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], 1 + 4);  // MMA commit + 4 converter warps
+      mbar_init(&raw_empty[s], 1 + CVT_WARPS);  // MMA commit + converter warps
     }
     for (int c = 0; c < CVT_STAGES; ++c) {
-      mbar_init(&cvt_full[c], 4);
+      mbar_init(&cvt_full[c], CVT_WARPS);
       mbar_init(&cvt_empty[c], 1);
     }
     mbar_init(acc_full, 1);
@@ -128,8 +136,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!mbar_wait(&raw_empty[s], (it & 1u) ^ 1u, guard, abort_flag, ERR_TIMEOUT_GEMM_PRODUCER)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&raw_full[s], A_BYTES + B8_BYTES);
-        tma_load_2d(sA + s * A_BYTES, &tm_a, &raw_full[s], kb * BK, tile_m * BM);
-        tma_load_2d(sB8 + s * B8_BYTES, &tm_b, &raw_full[s], kb * BK, tile_n * BN);
+        tma_load_2d(sA + s * A_BYTES, &tm_a, &raw_full[s], (kb0 + kb) * BK, tile_m * BM);
+        tma_load_2d(sB8 + s * B8_BYTES, &tm_b, &raw_full[s], (kb0 + kb) * BK, tile_n * BN);
       }
       __syncwarp();
       issued = kb + 1;
@@ -174,8 +182,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
     mbar_wait(drain_bar, 0u, guard, abort_flag, ERR_TIMEOUT_GEMM_DRAIN, true);
   } else {
-    // ---------------- converters (warps 2..5), then the epilogue
-    const int ct = threadIdx.x - 64;  // 0..127
+    // ---------------- converters (warps 2..9), then the epilogue
+    const int ct = threadIdx.x - 64;  // 0..255
     bool ok = true;
     for (int kb = 0; kb < num_kb && ok; ++kb) {
       const int s = kb % RAW_STAGES;
@@ -187,9 +195,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       const uint8_t* src = sB8 + s * B8_BYTES;
       uint8_t* dst = sB16 + c * B16_BYTES;
-#pragma unroll 4
-      for (int i = 0; i < (BN * BK / 16) / 128; ++i) {
-        const int chunk = i * 128 + ct;
+#pragma unroll
+      for (int i = 0; i < (BN * BK / 16) / (32 * CVT_WARPS); ++i) {
+        const int chunk = i * (32 * CVT_WARPS) + ct;
         const int r = chunk >> 2;
         const int q = chunk & 3;
         const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
@@ -214,9 +222,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok && mbar_wait(acc_full, 0u, guard, abort_flag, ERR_TIMEOUT_GEMM_EPILOGUE)) {
       tc_fence_after();
       const int quarter = warp & 3;
+      const int half = (warp - 2) >> 2;
       const int row = tile_m * BM + quarter * 32 + lane;
       const bool row_ok = row < p.M;
-      for (int cc = 0; cc < BN / 32; ++cc) {
+      for (int cc = half * (BN / 64); cc < (half + 1) * (BN / 64); ++cc) {
         const int col0 = tile_n * BN + cc * 32;
         if (col0 >= p.N) break;
         uint32_t r[32];
@@ -247,9 +256,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             float ov[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) ov[k] = v[q * 8 + k];
-            if (p.y_fmt == FMT_F32) store8<FMT_F32>(p.y, off8 + q, ov);
-            else if (p.y_fmt == FMT_F16) store8<FMT_F16>(p.y, off8 + q, ov);
-            else store8<FMT_BF16>(p.y, off8 + q, ov);
+            if (p.y_fmt == FMT_F32) store8<FMT_F32>(y_out, off8 + q, ov);
+            else if (p.y_fmt == FMT_F16) store8<FMT_F16>(y_out, off8 + q, ov);
+            else store8<FMT_BF16>(y_out, off8 + q, ov);
           }
         }
       }
@@ -264,7 +273,38 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// out[i] = sum over splits of part[z][i], as bf16; 8 elements per thread.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, uint16_t* __restrict__ out, int64_t n,
+                                     int splits) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i >= n / 8) return;
+  float v[8];
+  load8<FMT_F32>(part, i, v);
+  for (int z = 1; z < splits; ++z) {
+    float w[8];
+    load8<FMT_F32>(part + z * n, i, w);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] += w[k];
+  }
+  store8<FMT_BF16>(out, i, v);
+}
+
 }  // namespace gemm
+
+int gemm_pick_splits(int M, int N, int K) {
+  const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
+  const int kb = (K + gemm::BK - 1) / gemm::BK;
+  int s = 148 / tiles;
+  if (s > 8) s = 8;
+  if (s > kb / 16) s = kb / 16;  // keep at least 16 k-blocks per split
+  return s < 1 ? 1 : s;
+}
+
+cudaError_t launch_splitk_reduce(const float* part, uint16_t* out, int64_t n, int splits, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  gemm::splitk_reduce_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s>>>(part, out, n, splits);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStream_t s) {
   using namespace gemm;
@@ -287,8 +327,13 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
                    CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  Params p{a.scale, a.y, a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1, a.act, a.gelu_tanh};
-  dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN);
+  const int kb_total = (a.K + BK - 1) / BK;
+  const int splits = a.k_splits > 1 ? a.k_splits : 1;
+  const int kb_per = (kb_total + splits - 1) / splits;
+  Params p{a.scale, a.y, a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1, a.act, a.gelu_tanh,
+           kb_per, static_cast<int64_t>(a.M) * a.N};
+  if (splits > 1 && (a.y_fmt != FMT_F32 || a.residual != nullptr || a.act != 0)) return cudaErrorInvalidValue;
+  dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN, (kb_total + kb_per - 1) / kb_per);
   auto kern = f16 ? gemm_w8a16_kernel<true> : gemm_w8a16_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;

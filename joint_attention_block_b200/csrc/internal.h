@@ -66,8 +66,13 @@ struct GemmArgs {
   int M, N, K;
   int act;        // 0 none, 1 GELU
   int gelu_tanh;
+  int k_splits = 1;  // > 1: y is fp32 [k_splits, M, N] partial sums (scale applied; no act / residual)
 };
 cudaError_t launch_gemm_w8a16(const GemmArgs& args, const KernelGuard& g, cudaStream_t s);
+// Split count that fills the SMs for an M x N x K problem (1 when the tile grid already does).
+int gemm_pick_splits(int M, int N, int K);
+// out (bf16, n elements) = sum of `splits` fp32 partials laid out [splits, n]; n % 8 == 0.
+cudaError_t launch_splitk_reduce(const float* part, uint16_t* out, int64_t n, int splits, cudaStream_t s);
 
 // qkv and out in fmt (bf16 or f16).
 cudaError_t launch_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
