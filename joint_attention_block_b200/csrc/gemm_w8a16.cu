@@ -1,55 +1,59 @@
-// Y = epilogue( A (W8)^T * scale ) on the 5th-generation tensor cores.
+// Y = act( A (W8)^T * scale ) + R on the 5th-generation tensor cores.
 //
-// A: bf16 activations [M, K] row-major.  W8: e4m3 weights [N, K] row-major with an
-// fp32 per-output-row scale, the storage of the Ideogram 4 FP8 checkpoint
-// (unsloth diffusion_ideogram4.py commit log, fp8 loader commit: the real weight is
-// fp8 * weight_scale[:, None]).  Both operands are K-major, so the problem is the
-// "TN" GEMM tcgen05 reads natively.
+// A: 16-bit activations [M, K] row-major (M = tokens).  W8: e4m3 weights [N, K]
+// row-major with an fp32 per-output-row scale, the storage of the Ideogram 4 FP8
+// checkpoint (unsloth diffusion_ideogram4.py commit log, fp8 loader commit: the real
+// weight is fp8 * weight_scale[:, None]).
 //
 // The checkpoint's numerics are W8 dequantised, activations 16-bit.  e4m3 is a
-// subset of both bf16 and f16, so each weight tile is widened on chip, exactly,
-// to the activation format (bf16, or f16 for the block's internal activations)
-// and fed to tcgen05.mma kind::f16 with an fp32 accumulator in TMEM; the per-row
-// scale is applied once per output in the epilogue (scale[n] * sum_k a*w8 is
-// sum_k a*(w8*scale[n]) up to rounding).  The epilogue writes bf16, f16 or fp32
-// and can add a bf16 / f16 / fp32 residual.
+// subset of both bf16 and f16, so the weights are widened on chip, exactly, to the
+// activation format and fed to tcgen05.mma kind::f16 with an fp32 accumulator; the
+// per-row scale is applied once per output in the epilogue (scale[n] * sum_k a*w8
+// is sum_k a*(w8*scale[n]) up to rounding).
 //
-// CTA tile 128 x 256 x 64, one CTA per output tile.  Warp roles:
-//   warp 0      TMA producer: A tile (128 x 64, 128B swizzle) and the raw W8 tile
-//               (256 x 64 bytes) into a 4-stage ring.
-//   warp 1      TMEM allocation; one lane issues the MMAs (4 x K=16 per stage).
-//   warps 2..9  convert W8 -> 16-bit into the 128B-swizzled K-major layout the MMA
-//               reads (2-stage ring; two converter warps per scheduler to hide the
-//               conversion latency), then run the epilogue: tcgen05.ld of the
-//               accumulator (warp w reads TMEM lanes 32*(w%4).., column half
-//               (w-2)/4), scale, optional GELU / residual, stores.
+// The kernel computes the transposed tile D = W8_tile * A_tile^T (128 output
+// channels x 256 tokens) so that the widened weights are the MMA's A operand and
+// live in TENSOR MEMORY: each converter thread owns one weight row (one TMEM lane),
+// loads its e4m3 bytes straight from global memory (L2) a few stages ahead,
+// widens them in registers and writes them with tcgen05.st.  The converted weights
+// never touch shared memory, so shared memory carries only the TMA-fed activation
+// tile the MMA reads; and a 128-row weight tile is widened once per 256 tokens.
+//
+// CTA tile 128 (channels) x 256 (tokens) x 64 (K); one CTA per tile (grid.z = K splits).
+//   warp 0      TMA producer: activation tile 256 x 64 (128B swizzle), 4-stage ring.
+//   warp 1      TMEM allocation; one lane issues 4 MMAs (M=128, N=256, K=16) per stage.
+//   warps 2..9  converters: warp w owns TMEM lanes 32*(w%4).. (channels) and half of
+//               each stage's 64 K-columns; 4-stage TMEM ring for the widened weights.
+//               Then the epilogue: tcgen05.ld of the accumulator (lane = channel,
+//               column = token), scale, optional GELU, a transpose through shared
+//               memory, optional residual, and row-contiguous stores.
 #include "common.cuh"
 
 namespace jab {
 namespace gemm {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 256;  // tokens per tile (MMA N)
+constexpr int BN = 128;  // output channels per tile (MMA M)
 constexpr int BK = 64;
-constexpr int RAW_STAGES = 4;
-constexpr int CVT_STAGES = 2;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B8_BYTES = BN * BK;
-constexpr int B16_BYTES = BN * BK * 2;
+constexpr int STAGES = 4;
+constexpr int X_BYTES = BM * BK * 2;
 constexpr int THREADS = 320;
 constexpr int CVT_WARPS = 8;
-constexpr int TMEM_COLS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COL = 0;      // accumulator: columns [0, 256)
+constexpr int A_COL = 256;      // widened weights: stage s at 256 + 32 * s
+constexpr int EPI_BYTES = 32 * 32 * 4;  // per-warp transpose buffer
 
-constexpr int OFF_A = 0;
-constexpr int OFF_B8 = OFF_A + RAW_STAGES * A_BYTES;
-constexpr int OFF_B16 = OFF_B8 + RAW_STAGES * B8_BYTES;
-constexpr int OFF_SCALE = OFF_B16 + CVT_STAGES * B16_BYTES;
+constexpr int OFF_X = 0;
+constexpr int OFF_EPI = OFF_X + STAGES * X_BYTES;
+constexpr int OFF_SCALE = OFF_EPI + CVT_WARPS * EPI_BYTES;
 constexpr int OFF_BAR = OFF_SCALE + BN * 4;
-constexpr int NUM_BARS = 2 * RAW_STAGES + 2 * CVT_STAGES + 2;
+constexpr int NUM_BARS = 4 * STAGES + 2;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 
 struct Params {
+  const uint8_t* w;
   const float* scale;
   void* y;
   const void* residual;
@@ -58,8 +62,8 @@ struct Params {
   int res_fmt;  // -1 none, FMT_BF16 / FMT_F16 / FMT_F32
   int act;      // 0 none, 1 GELU
   int gelu_tanh;
-  int kb_per_split;          // k-blocks per split (grid.z splits); all of K when not split
-  int64_t y_split_stride;    // elements between the fp32 partial outputs of consecutive splits
+  int kb_per_split;        // k-blocks per split (grid.z splits); all of K when not split
+  int64_t y_split_stride;  // elements between the fp32 partial outputs of consecutive splits
 };
 
 __device__ __forceinline__ float gelu_f(float x, int tanh_form) {
@@ -70,53 +74,58 @@ __device__ __forceinline__ float gelu_f(float x, int tanh_form) {
   return 0.5f * x * (1.f + erff(x * 0.7071067811865476f));
 }
 
+// The 32 weight bytes a converter thread widens for k-block kb (zero past N or K).
+__device__ __forceinline__ void load_w(const Params& p, int n, int kb, int kh, uint4 (&v)[2]) {
+  const int k = kb * BK + kh * 32;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (n < p.N && k + 16 * i < p.K) {
+      v[i] = __ldg(reinterpret_cast<const uint4*>(p.w + static_cast<size_t>(n) * p.K + k + 16 * i));
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
 template <bool F16>
 __global__ void __launch_bounds__(THREADS, 1)
-    gemm_w8a16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                      const Params p, const KernelGuard guard) {
+    gemm_w8a16_kernel(const __grid_constant__ CUtensorMap tm_x, const Params p, const KernelGuard guard) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem + OFF_A;
-  uint8_t* sB8 = smem + OFF_B8;
-  uint8_t* sB16 = smem + OFF_B16;
+  uint8_t* sX = smem + OFF_X;
   float* sScale = reinterpret_cast<float*>(smem + OFF_SCALE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* raw_full = bars;
-  uint64_t* raw_empty = bars + RAW_STAGES;
-  uint64_t* cvt_full = bars + 2 * RAW_STAGES;
-  uint64_t* cvt_empty = bars + 2 * RAW_STAGES + CVT_STAGES;
-  uint64_t* acc_full = bars + 2 * RAW_STAGES + 2 * CVT_STAGES;
+  uint64_t* x_full = bars;
+  uint64_t* x_empty = bars + STAGES;
+  uint64_t* a_full = bars + 2 * STAGES;
+  uint64_t* a_empty = bars + 3 * STAGES;
+  uint64_t* acc_full = bars + 4 * STAGES;
   uint64_t* drain_bar = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
 
   const int warp = static_cast<int>(warp_id());
   const int lane = static_cast<int>(lane_id());
-  const int tile_m = blockIdx.x;
-  const int tile_n = blockIdx.y;
+  const int tile_m = blockIdx.x;  // tokens
+  const int tile_n = blockIdx.y;  // channels
   const int kb_total = (p.K + BK - 1) / BK;
   const int kb0 = blockIdx.z * p.kb_per_split;
   const int num_kb = min(kb_total - kb0, p.kb_per_split);
   void* const y_out = static_cast<char*>(p.y) + blockIdx.z * p.y_split_stride * 4;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < RAW_STAGES; ++s) {
-      mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], 1 + CVT_WARPS);  // MMA commit + converter warps
-    }
-    for (int c = 0; c < CVT_STAGES; ++c) {
-      mbar_init(&cvt_full[c], CVT_WARPS);
-      mbar_init(&cvt_empty[c], 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1);
+      mbar_init(&a_full[s], CVT_WARPS);
+      mbar_init(&a_empty[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
-  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_x);
   if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
   for (int i = threadIdx.x; i < BN; i += THREADS) {
     const int n = tile_n * BN + i;
@@ -125,53 +134,48 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_acc = *tmem_slot;
+  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer (activation tiles)
     int issued = 0;
     for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % RAW_STAGES;
-      const uint32_t it = static_cast<uint32_t>(kb / RAW_STAGES);
-      if (!mbar_wait(&raw_empty[s], (it & 1u) ^ 1u, guard, abort_flag, ERR_TIMEOUT_GEMM_PRODUCER)) break;
+      const int s = kb % STAGES;
+      const uint32_t it = static_cast<uint32_t>(kb / STAGES);
+      if (!mbar_wait(&x_empty[s], (it & 1u) ^ 1u, guard, abort_flag, ERR_TIMEOUT_GEMM_PRODUCER)) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&raw_full[s], A_BYTES + B8_BYTES);
-        tma_load_2d(sA + s * A_BYTES, &tm_a, &raw_full[s], (kb0 + kb) * BK, tile_m * BM);
-        tma_load_2d(sB8 + s * B8_BYTES, &tm_b, &raw_full[s], (kb0 + kb) * BK, tile_n * BN);
+        mbar_arrive_expect_tx(&x_full[s], X_BYTES);
+        tma_load_2d(sX + s * X_BYTES, &tm_x, &x_full[s], (kb0 + kb) * BK, tile_m * BM);
       }
       __syncwarp();
       issued = kb + 1;
     }
     // Never leave with copies in flight: wait for the last load of every stage.
-    for (int s = 0; s < RAW_STAGES && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / RAW_STAGES) * RAW_STAGES;
-      const uint32_t it = static_cast<uint32_t>(last / RAW_STAGES);
-      mbar_wait(&raw_full[s], it & 1u, guard, abort_flag, ERR_TIMEOUT_GEMM_DRAIN, true);
+    for (int s = 0; s < STAGES && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
+      mbar_wait(&x_full[s], static_cast<uint32_t>(last / STAGES) & 1u, guard, abort_flag, ERR_TIMEOUT_GEMM_DRAIN,
+                true);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
-    constexpr uint32_t idesc = idesc_f16kind(BM, BN, F16, false, false);
+    constexpr uint32_t idesc = idesc_f16kind(BN, BM, F16, false, false);
     bool ok = true;
     for (int kb = 0; kb < num_kb && ok; ++kb) {
-      const int s = kb % RAW_STAGES;
-      const int c = kb % CVT_STAGES;
-      ok = mbar_wait(&raw_full[s], static_cast<uint32_t>(kb / RAW_STAGES) & 1u, guard, abort_flag,
-                     ERR_TIMEOUT_GEMM_MMA) &&
-           mbar_wait(&cvt_full[c], static_cast<uint32_t>(kb / CVT_STAGES) & 1u, guard, abort_flag,
-                     ERR_TIMEOUT_GEMM_MMA);
+      const int s = kb % STAGES;
+      const uint32_t par = static_cast<uint32_t>(kb / STAGES) & 1u;
+      ok = mbar_wait(&x_full[s], par, guard, abort_flag, ERR_TIMEOUT_GEMM_MMA) &&
+           mbar_wait(&a_full[s], par, guard, abort_flag, ERR_TIMEOUT_GEMM_MMA);
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a0 = smem_u32(sA + s * A_BYTES);
-        const uint32_t b0 = smem_u32(sB16 + c * B16_BYTES);
+        const uint32_t x0 = smem_u32(sX + s * X_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(a0 + kk * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-          mma_f16kind_ss(tmem_acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(x0 + kk * 32, 16, 1024);
+          mma_f16kind_ts(tmem + ACC_COL, tmem + A_COL + 32 * s + 8 * kk, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
-        mma_commit(&raw_empty[s]);
-        mma_commit(&cvt_empty[c]);
+        mma_commit(&x_empty[s]);
+        mma_commit(&a_empty[s]);
       }
       __syncwarp();
     }
@@ -182,80 +186,96 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
     mbar_wait(drain_bar, 0u, guard, abort_flag, ERR_TIMEOUT_GEMM_DRAIN, true);
   } else {
-    // ---------------- converters (warps 2..9), then the epilogue
-    const int ct = threadIdx.x - 64;  // 0..255
-    bool ok = true;
-    for (int kb = 0; kb < num_kb && ok; ++kb) {
-      const int s = kb % RAW_STAGES;
-      const int c = kb % CVT_STAGES;
-      ok = mbar_wait(&raw_full[s], static_cast<uint32_t>(kb / RAW_STAGES) & 1u, guard, abort_flag,
-                     ERR_TIMEOUT_GEMM_CONVERT) &&
-           mbar_wait(&cvt_empty[c], (static_cast<uint32_t>(kb / CVT_STAGES) & 1u) ^ 1u, guard, abort_flag,
-                     ERR_TIMEOUT_GEMM_CONVERT);
-      if (!ok) break;
-      const uint8_t* src = sB8 + s * B8_BYTES;
-      uint8_t* dst = sB16 + c * B16_BYTES;
+    // ---------------- converters (warps 2..9): thread = weight row, half a stage of K each
+    const int quarter = warp & 3;
+    const int kh = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;  // TMEM lane = channel within the tile
+    const int n = tile_n * BN + row;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    constexpr int PF = STAGES;  // weight bytes held in registers ahead of conversion
+    uint4 pf[PF][2];
 #pragma unroll
-      for (int i = 0; i < (BN * BK / 16) / (32 * CVT_WARPS); ++i) {
-        const int chunk = i * (32 * CVT_WARPS) + ct;
-        const int r = chunk >> 2;
-        const int q = chunk & 3;
-        const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
-        uint4 o0, o1;
-        e4m3x4_to_16x4<F16>(v.x, o0.x, o0.y);
-        e4m3x4_to_16x4<F16>(v.y, o0.z, o0.w);
-        e4m3x4_to_16x4<F16>(v.z, o1.x, o1.y);
-        e4m3x4_to_16x4<F16>(v.w, o1.z, o1.w);
-        uint8_t* row = dst + r * 128;
-        *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) << 4)) = o0;
-        *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) << 4)) = o1;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&cvt_full[c]);
-        mbar_arrive(&raw_empty[s]);
+    for (int i = 0; i < PF; ++i) {
+      if (i < num_kb) load_w(p, n, kb0 + i, kh, pf[i]);
+    }
+    bool ok = true;
+    for (int kbase = 0; kbase < num_kb && ok; kbase += PF) {
+#pragma unroll
+      for (int i = 0; i < PF; ++i) {
+        const int kb = kbase + i;
+        if (kb >= num_kb) break;
+        const uint4 c0 = pf[i][0], c1 = pf[i][1];
+        if (kb + PF < num_kb) load_w(p, n, kb0 + kb + PF, kh, pf[i]);
+        uint32_t h[16];
+        e4m3x4_to_16x4<F16>(c0.x, h[0], h[1]);
+        e4m3x4_to_16x4<F16>(c0.y, h[2], h[3]);
+        e4m3x4_to_16x4<F16>(c0.z, h[4], h[5]);
+        e4m3x4_to_16x4<F16>(c0.w, h[6], h[7]);
+        e4m3x4_to_16x4<F16>(c1.x, h[8], h[9]);
+        e4m3x4_to_16x4<F16>(c1.y, h[10], h[11]);
+        e4m3x4_to_16x4<F16>(c1.z, h[12], h[13]);
+        e4m3x4_to_16x4<F16>(c1.w, h[14], h[15]);
+        const int s = kb % STAGES;
+        if (!mbar_wait(&a_empty[s], (static_cast<uint32_t>(kb / STAGES) & 1u) ^ 1u, guard, abort_flag,
+                       ERR_TIMEOUT_GEMM_CONVERT)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(tmem + lane_off + A_COL + 32 * s + 16 * kh, h);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[s]);
       }
     }
 
-    // ---------------- epilogue: warp (w % 4) owns TMEM lanes 32*(w%4) .. +31
+    // ---------------- epilogue: lane = channel, TMEM column = token
     if (ok && mbar_wait(acc_full, 0u, guard, abort_flag, ERR_TIMEOUT_GEMM_EPILOGUE)) {
       tc_fence_after();
-      const int quarter = warp & 3;
-      const int half = (warp - 2) >> 2;
-      const int row = tile_m * BM + quarter * 32 + lane;
-      const bool row_ok = row < p.M;
-      for (int cc = half * (BN / 64); cc < (half + 1) * (BN / 64); ++cc) {
-        const int col0 = tile_n * BN + cc * 32;
-        if (col0 >= p.N) break;
+      float* buf = reinterpret_cast<float*>(smem + OFF_EPI + (warp - 2) * EPI_BYTES);
+      const float sc = sScale[row];
+      const int ch0 = tile_n * BN + quarter * 32;  // first channel of this warp
+      const bool warp_has_channels = ch0 < p.N;
+      for (int c = 0; c < 4; ++c) {
+        const int tcol = kh * 128 + c * 32;  // first token column of this chunk
         uint32_t r[32];
-        tmem_ld32(tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16) + cc * 32, r);
+        tmem_ld32(tmem + lane_off + ACC_COL + tcol, r);
         tmem_ld_wait();
-        float v[32];
+        // r[j] = D[channel = lane][token j] -> transpose: buf row j = token, column = channel
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * sScale[cc * 32 + j];
-        if (p.act == 1) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = gelu_f(v[j], p.gelu_tanh);
+        for (int j = 0; j < 32; ++j) {
+          float v = __uint_as_float(r[j]) * sc;
+          if (p.act == 1) v = gelu_f(v, p.gelu_tanh);
+          buf[j * 32 + ((((lane >> 2) ^ (j & 7))) << 2) + (lane & 3)] = v;
         }
-        if (row_ok) {
-          const int64_t off8 = (static_cast<int64_t>(row) * p.N + col0) / 8;
-          if (p.res_fmt >= 0) {
+        __syncwarp();
+        float o[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 8; ++q) {
+          const float4 t = *reinterpret_cast<const float4*>(buf + lane * 32 + ((q ^ (lane & 7)) << 2));
+          o[4 * q] = t.x;
+          o[4 * q + 1] = t.y;
+          o[4 * q + 2] = t.z;
+          o[4 * q + 3] = t.w;
+        }
+        __syncwarp();
+        const int tok = tile_m * BM + tcol + lane;
+        if (warp_has_channels && tok < p.M) {
+          const int64_t off8 = (static_cast<int64_t>(tok) * p.N + ch0) / 8;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float ov[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ov[k] = o[8 * q + k];
+            if (p.res_fmt >= 0) {
               float rv[8];
               if (p.res_fmt == FMT_F32) load8<FMT_F32>(p.residual, off8 + q, rv);
               else if (p.res_fmt == FMT_F16) load8<FMT_F16>(p.residual, off8 + q, rv);
               else load8<FMT_BF16>(p.residual, off8 + q, rv);
 #pragma unroll
-              for (int k = 0; k < 8; ++k) v[q * 8 + k] += rv[k];
+              for (int k = 0; k < 8; ++k) ov[k] += rv[k];
             }
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float ov[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) ov[k] = v[q * 8 + k];
             if (p.y_fmt == FMT_F32) store8<FMT_F32>(y_out, off8 + q, ov);
             else if (p.y_fmt == FMT_F16) store8<FMT_F16>(y_out, off8 + q, ov);
             else store8<FMT_BF16>(y_out, off8 + q, ov);
@@ -269,7 +289,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_acc, TMEM_COLS);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -310,34 +330,26 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
   using namespace gemm;
   if (a.M <= 0 || a.N <= 0) return cudaSuccess;
   const bool f16 = a.a_fmt == FMT_F16;
-  CUtensorMap tm_a, tm_b;
+  CUtensorMap tm_x;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
     const uint32_t box[2] = {BK, BM};
-    if (!make_tmap(&tm_a, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+    if (!make_tmap(&tm_x, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(a.a), dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  }
-  {
-    const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.N)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(a.K)};
-    const uint32_t box[2] = {BK, BN};
-    if (!make_tmap(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.w), dims, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
   const int kb_total = (a.K + BK - 1) / BK;
   const int splits = a.k_splits > 1 ? a.k_splits : 1;
   const int kb_per = (kb_total + splits - 1) / splits;
-  Params p{a.scale, a.y, a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1, a.act, a.gelu_tanh,
-           kb_per, static_cast<int64_t>(a.M) * a.N};
   if (splits > 1 && (a.y_fmt != FMT_F32 || a.residual != nullptr || a.act != 0)) return cudaErrorInvalidValue;
+  Params p{a.w,   a.scale,     a.y,    a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1,
+           a.act, a.gelu_tanh, kb_per, static_cast<int64_t>(a.M) * a.N};
   dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN, (kb_total + kb_per - 1) / kb_per);
   auto kern = f16 ? gemm_w8a16_kernel<true> : gemm_w8a16_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, THREADS, SMEM_BYTES, s>>>(tm_a, tm_b, p, g);
+  kern<<<grid, THREADS, SMEM_BYTES, s>>>(tm_x, p, g);
   return cudaGetLastError();
 }
 
