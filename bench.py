@@ -250,11 +250,13 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    for _ in range(args.warmup):
+    for i in range(args.warmup):
         step()
+        if i == 0 and ops.poll_error() != 0:  # fail fast: a broken step must not be repeated
+            raise RuntimeError(f"device-side error in the first step: {ops.last_device_error():#x}")
     torch.cuda.synchronize(dev)
     if ops.poll_error() != 0:
-        raise RuntimeError("device-side error during warm-up")
+        raise RuntimeError(f"device-side error during warm-up: {ops.last_device_error():#x}")
 
     # ---- timed region: device-resident inputs; per-launch events inside the library
     clocks = ClockSampler(local_rank)
@@ -277,7 +279,7 @@ def run_ours(args, rank, world, local_rank):
     ms = max_over_ranks(ev0.elapsed_time(ev1))
     records = ops.profile_read(args.steps * 24 + 64)
     if ops.poll_error() != 0:
-        raise RuntimeError("device-side error in the timed region")
+        raise RuntimeError(f"device-side error in the timed region: {ops.last_device_error():#x}")
 
     # ---- end to end through the public calls: pinned host inputs in, results out, every step
     h_feats = torch.from_numpy(cond["feats"].view(np.int16)).pin_memory()

@@ -190,6 +190,11 @@ DIT_API int dit_profile_enable(int max_marks);
 DIT_API int dit_profile_disable(void);
 DIT_API int dit_profile_read(int* tags, float* ms, int max_records);
 
+/* Raw device error word seen by the last dit_poll_error() that reported an error:
+ * bits 0..11 name the wait that gave up (0x1xx = bounded-wait timeout), bits 12..15 the
+ * CTA's rank in its cluster, bits 16..31 the k-block / loop index. */
+DIT_API uint32_t dit_last_device_error(void);
+
 /* Set the wall-time limit of every device-side bounded wait (default 2000 ms). */
 DIT_API int dit_set_wait_timeout_ms(uint32_t ms);
 

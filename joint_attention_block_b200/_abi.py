@@ -79,6 +79,7 @@ SIGNATURES = {
     "dit_profile_disable": (_I, []),
     "dit_profile_read": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float), _I]),
     "dit_set_wait_timeout_ms": (_I, [ctypes.c_uint32]),
+    "dit_last_device_error": (ctypes.c_uint32, []),
     "dit_status_str": (ctypes.c_char_p, [_I]),
     "dit_abi_version": (_I, []),
 }
@@ -237,6 +238,10 @@ def profile_read(max_records: int = 1 << 16):
 
 def poll_error(stream=None) -> int:
     return int(lib().dit_poll_error(_stream(stream)))
+
+
+def last_device_error() -> int:
+    return int(lib().dit_last_device_error())
 
 
 def set_wait_timeout_ms(ms: int) -> None:

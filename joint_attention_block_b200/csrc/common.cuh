@@ -32,8 +32,14 @@ JAB_DEVICE uint64_t global_timer_ns() {
 }
 
 // Record an error code (first one wins) in the library's device error word.
+// Bits 0..11: which wait; bits 12..15: CTA rank in its cluster; bits 16..31: k-block
+// or loop index where it gave up (see where_code()).
 JAB_DEVICE void record_error(uint32_t* err, uint32_t code) {
   if (err != nullptr) atomicCAS(err, 0u, code);
+}
+
+JAB_DEVICE uint32_t where_code(uint32_t where, uint32_t rank, uint32_t index) {
+  return (where & 0xFFFu) | ((rank & 0xFu) << 12) | ((index < 0xFFFFu ? index : 0xFFFFu) << 16);
 }
 
 JAB_DEVICE float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -216,6 +222,10 @@ JAB_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, const KernelGuard& g, 
     if (mbar_try_wait(bar, parity)) return true;
     if (((++spins) & 63u) == 0) {
       if (!drain && *abort_flag) return false;
+      if (!drain && g.err != nullptr && *reinterpret_cast<volatile uint32_t*>(g.err) != 0u) {
+        *abort_flag = 1u;  // another CTA already failed: give up at once
+        return false;
+      }
       if (global_timer_ns() - t0 > g.timeout_ns) {
         *abort_flag = 1u;
         record_error(g.err, where);
@@ -223,6 +233,108 @@ JAB_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, const KernelGuard& g, 
       }
     }
   }
+}
+
+// ------------------------------------------------------------------ CTA pairs (clusters of 2)
+
+JAB_DEVICE uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+JAB_DEVICE uint32_t mapa_shared(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+
+// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.
+JAB_DEVICE void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+JAB_DEVICE bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire, for barriers that CTAs of the pair arrive on.
+JAB_DEVICE bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const KernelGuard& g, volatile uint32_t* abort_flag,
+                                  uint32_t where) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (((++spins) & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (g.err != nullptr && *reinterpret_cast<volatile uint32_t*>(g.err) != 0u) {
+        *abort_flag = 1u;
+        return false;
+      }
+      if (global_timer_ns() - t0 > g.timeout_ns) {
+        *abort_flag = 1u;
+        record_error(g.err, where);
+        return false;
+      }
+    }
+  }
+}
+
+JAB_DEVICE void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// TMA tile load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (given by its shared::cluster address).
+JAB_DEVICE void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster_addr, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+
+JAB_DEVICE void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+JAB_DEVICE void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Pair MMA issued by the leader CTA: D (M=256 over both CTAs' TMEM) (+)= A (TMEM of
+// both CTAs) * B (shared memory of both CTAs, N/2 rows each)^T.
+JAB_DEVICE void mma_f16kind_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                    uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the mbarrier at this shared-memory offset in every CTA of `cta_mask`
+// once all pair MMAs issued so far by this thread are done.
+JAB_DEVICE void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
 }
 
 // ------------------------------------------------------------------ proxies / fences

@@ -233,6 +233,10 @@ int dit_set_wait_timeout_ms(uint32_t ms) {
   return DIT_OK;
 }
 
+static std::atomic<uint32_t> g_last_device_error{0};
+
+uint32_t dit_last_device_error(void) { return g_last_device_error.load(); }
+
 int dit_poll_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize(as_stream(stream));
   if (e != cudaSuccess) return DIT_ERR_CUDA;
@@ -241,6 +245,7 @@ int dit_poll_error(void* stream) {
   uint32_t v = 0;
   if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return DIT_ERR_CUDA;
   if (v == 0) return DIT_OK;
+  g_last_device_error.store(v);
   const uint32_t zero = 0;
   if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return DIT_ERR_CUDA;
   return (v & 0xF00u) == 0x100u ? DIT_ERR_TIMEOUT : DIT_ERR_DEVICE;

@@ -11,43 +11,55 @@
 // per-row scale is applied once per output in the epilogue (scale[n] * sum_k a*w8
 // is sum_k a*(w8*scale[n]) up to rounding).
 //
-// The kernel computes the transposed tile D = W8_tile * A_tile^T (128 output
-// channels x 256 tokens) so that the widened weights are the MMA's A operand and
-// live in TENSOR MEMORY: each converter thread owns one weight row (one TMEM lane),
-// loads its e4m3 bytes straight from global memory (L2) a few stages ahead,
-// widens them in registers and writes them with tcgen05.st.  The converted weights
-// never touch shared memory, so shared memory carries only the TMA-fed activation
-// tile the MMA reads; and a 128-row weight tile is widened once per 256 tokens.
+// The kernel computes the transposed tile D = W8_tile * A_tile^T so that the
+// widened weights are the MMA's A operand and live in TENSOR MEMORY: each converter
+// thread owns one weight row (one TMEM lane), loads its e4m3 bytes straight from
+// global memory (L2) a few stages ahead, widens them in registers and writes them
+// with tcgen05.st.  The converted weights never touch shared memory.
 //
-// CTA tile 128 (channels) x 256 (tokens) x 64 (K); one CTA per tile (grid.z = K splits).
-//   warp 0      TMA producer: activation tile 256 x 64 (128B swizzle), 4-stage ring.
-//   warp 1      TMEM allocation; one lane issues 4 MMAs (M=128, N=256, K=16) per stage.
+// Two CTAs on two SMs (a cluster of 2) share one 256 (channels) x 256 (tokens) tile
+// through the pair form of the MMA (tcgen05.mma.cta_group::2, M = 256, N = 256):
+// each CTA widens its own 128 weight rows into its own TMEM (half of A) and
+// TMA-loads its own 128 tokens into its own shared memory (half of B); the leader
+// CTA issues the MMAs, each CTA's TMEM receives its 128 channels x 256 tokens of D.
+// Per SM and K-step this reads half the activation bytes of a one-SM 128 x 256
+// tile, which is what keeps L2 traffic per FLOP low enough for the tensor pipe.
+// Both CTAs' TMA loads count on the leader's barrier, the converters arrive on it
+// remotely, and the leader's MMA commits arrive on both CTAs' barriers.  No TMA
+// load is multicast.
+//
+// Per CTA: 128 channels x 256 tokens x 64 (K) per stage; grid.z = K splits.
+//   warp 0      TMA producer: this CTA's 128 x 64 activation half (128B swizzle).
+//   warp 1      TMEM allocation (pair); in the leader, one lane issues the pair MMAs.
 //   warps 2..9  converters: warp w owns TMEM lanes 32*(w%4).. (channels) and half of
-//               each stage's 64 K-columns; 4-stage TMEM ring for the widened weights.
-//               Then the epilogue: tcgen05.ld of the accumulator (lane = channel,
-//               column = token), scale, optional GELU, a transpose through shared
-//               memory, optional residual, and row-contiguous stores.
+//               each stage's 64 K-columns (TMEM ring of widened weights).  Then the
+//               epilogue: tcgen05.ld of the accumulator (lane = channel, column =
+//               token), scale, optional GELU, a transpose through shared memory,
+//               optional residual, and row-contiguous stores.
 #include "common.cuh"
 
 namespace jab {
 namespace gemm {
 
-constexpr int BM = 256;  // tokens per tile (MMA N)
-constexpr int BN = 128;  // output channels per tile (MMA M)
+constexpr int BM = 256;      // tokens per pair tile (MMA N)
+constexpr int BM_CTA = 128;  // tokens each CTA loads
+constexpr int BN = 256;      // output channels per pair tile (MMA M)
+constexpr int BN_CTA = 128;  // channels each CTA owns (its TMEM lanes)
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int X_BYTES = BM * BK * 2;
+constexpr int STAGES = 6;    // activation (smem) and widened-weight (TMEM) ring depth
+constexpr int PF = 4;        // k-blocks of weight bytes prefetched into registers
+constexpr int X_BYTES = BM_CTA * BK * 2;
 constexpr int THREADS = 320;
 constexpr int CVT_WARPS = 8;
 constexpr int TMEM_COLS = 512;
-constexpr int ACC_COL = 0;      // accumulator: columns [0, 256)
-constexpr int A_COL = 256;      // widened weights: stage s at 256 + 32 * s
+constexpr int ACC_COL = 0;   // accumulator: columns [0, 256)
+constexpr int A_COL = 256;   // widened weights: stage s at 256 + 32 * s
 constexpr int EPI_BYTES = 32 * 32 * 4;  // per-warp transpose buffer
 
 constexpr int OFF_X = 0;
 constexpr int OFF_EPI = OFF_X + STAGES * X_BYTES;
 constexpr int OFF_SCALE = OFF_EPI + CVT_WARPS * EPI_BYTES;
-constexpr int OFF_BAR = OFF_SCALE + BN * 4;
+constexpr int OFF_BAR = OFF_SCALE + BN_CTA * 4;
 constexpr int NUM_BARS = 4 * STAGES + 2;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
@@ -88,16 +100,16 @@ __device__ __forceinline__ void load_w(const Params& p, int n, int kb, int kh, u
 }
 
 template <bool F16>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_w8a16_kernel(const __grid_constant__ CUtensorMap tm_x, const Params p, const KernelGuard guard) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem + OFF_X;
   float* sScale = reinterpret_cast<float*>(smem + OFF_SCALE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* x_full = bars;
-  uint64_t* x_empty = bars + STAGES;
-  uint64_t* a_full = bars + 2 * STAGES;
+  uint64_t* x_full = bars;               // leader: both CTAs' activation halves landed
+  uint64_t* x_empty = bars + STAGES;     // both: the pair MMAs of the stage are done
+  uint64_t* a_full = bars + 2 * STAGES;  // leader: both CTAs' weights widened into TMEM
   uint64_t* a_empty = bars + 3 * STAGES;
   uint64_t* acc_full = bars + 4 * STAGES;
   uint64_t* drain_bar = acc_full + 1;
@@ -106,8 +118,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = static_cast<int>(warp_id());
   const int lane = static_cast<int>(lane_id());
-  const int tile_m = blockIdx.x;  // tokens
-  const int tile_n = blockIdx.y;  // channels
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int tile_m = blockIdx.x >> 1;  // pair tile of 256 tokens
+  const int tile_n = blockIdx.y;       // pair tile of 256 channels
+  const int tok_cta = tile_m * BM + static_cast<int>(rank) * BM_CTA;  // rows of A this CTA loads
+  const int ch_cta = tile_n * BN + static_cast<int>(rank) * BN_CTA;   // channels this CTA owns
   const int kb_total = (p.K + BK - 1) / BK;
   const int kb0 = blockIdx.z * p.kb_per_split;
   const int num_kb = min(kb_total - kb0, p.kb_per_split);
@@ -117,7 +133,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&x_full[s], 1);
       mbar_init(&x_empty[s], 1);
-      mbar_init(&a_full[s], CVT_WARPS);
+      mbar_init(&a_full[s], 2 * CVT_WARPS);
       mbar_init(&a_empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -126,73 +142,79 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_x);
-  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
-  for (int i = threadIdx.x; i < BN; i += THREADS) {
-    const int n = tile_n * BN + i;
+  if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
+  for (int i = threadIdx.x; i < BN_CTA; i += THREADS) {
+    const int n = ch_cta + i;
     sScale[i] = n < p.N ? p.scale[n] : 0.f;
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer (activation tiles)
+    // ---------------- TMA producer: this CTA's activation half, counted on the leader's barrier
     int issued = 0;
     for (int kb = 0; kb < num_kb; ++kb) {
       const int s = kb % STAGES;
       const uint32_t it = static_cast<uint32_t>(kb / STAGES);
-      if (!mbar_wait(&x_empty[s], (it & 1u) ^ 1u, guard, abort_flag, ERR_TIMEOUT_GEMM_PRODUCER)) break;
+      if (!mbar_wait(&x_empty[s], (it & 1u) ^ 1u, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_PRODUCER, rank, kb))) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&x_full[s], X_BYTES);
-        tma_load_2d(sX + s * X_BYTES, &tm_x, &x_full[s], (kb0 + kb) * BK, tile_m * BM);
+        if (leader) mbar_arrive_expect_tx(&x_full[s], 2 * X_BYTES);
+        tma_load_2d_pair(sX + s * X_BYTES, &tm_x, mapa_shared(smem_u32(&x_full[s]), 0), (kb0 + kb) * BK, tok_cta);
       }
       __syncwarp();
       issued = kb + 1;
     }
-    // Never leave with copies in flight: wait for the last load of every stage.
-    for (int s = 0; s < STAGES && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
-      mbar_wait(&x_full[s], static_cast<uint32_t>(last / STAGES) & 1u, guard, abort_flag, ERR_TIMEOUT_GEMM_DRAIN,
-                true);
+    // The leader never leaves with copies in flight (its barrier counts both CTAs' loads);
+    // the peer is held by the final cluster barrier until the leader has drained.
+    if (leader) {
+      for (int s = 0; s < STAGES && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
+        mbar_wait(&x_full[s], static_cast<uint32_t>(last / STAGES) & 1u, guard, abort_flag,
+                  where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, s), true);
+      }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
-    constexpr uint32_t idesc = idesc_f16kind(BN, BM, F16, false, false);
-    bool ok = true;
-    for (int kb = 0; kb < num_kb && ok; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t par = static_cast<uint32_t>(kb / STAGES) & 1u;
-      ok = mbar_wait(&x_full[s], par, guard, abort_flag, ERR_TIMEOUT_GEMM_MMA) &&
-           mbar_wait(&a_full[s], par, guard, abort_flag, ERR_TIMEOUT_GEMM_MMA);
-      if (!ok) break;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t x0 = smem_u32(sX + s * X_BYTES);
+    // ---------------- MMA issuer (leader only)
+    if (leader) {
+      constexpr uint32_t idesc = idesc_f16kind(BN, BM, F16, false, false);
+      bool ok = true;
+      for (int kb = 0; kb < num_kb && ok; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t par = static_cast<uint32_t>(kb / STAGES) & 1u;
+        ok = mbar_wait_cluster(&x_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_MMA_X, rank, kb)) &&
+             mbar_wait_cluster(&a_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_MMA, rank, kb));
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t x0 = smem_u32(sX + s * X_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(x0 + kk * 32, 16, 1024);
-          mma_f16kind_ts(tmem + ACC_COL, tmem + A_COL + 32 * s + 8 * kk, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(x0 + kk * 32, 16, 1024);
+            mma_f16kind_ts_pair(tmem + ACC_COL, tmem + A_COL + 32 * s + 8 * kk, bd, idesc,
+                                (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair(&x_empty[s], 0x3);
+          mma_commit_pair(&a_empty[s], 0x3);
         }
-        mma_commit(&x_empty[s]);
-        mma_commit(&a_empty[s]);
+        __syncwarp();
+      }
+      if (lane == 0) {
+        if (ok) mma_commit_pair(acc_full, 0x3);
+        mma_commit_pair(drain_bar, 0x3);  // all MMAs retired before either CTA frees TMEM
       }
       __syncwarp();
     }
-    if (lane == 0) {
-      if (ok) mma_commit(acc_full);
-      mma_commit(drain_bar);  // all MMAs retired before TMEM is freed
-    }
-    __syncwarp();
-    mbar_wait(drain_bar, 0u, guard, abort_flag, ERR_TIMEOUT_GEMM_DRAIN, true);
+    mbar_wait(drain_bar, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_DRAIN_MMA, rank, 0), true);
   } else {
     // ---------------- converters (warps 2..9): thread = weight row, half a stage of K each
     const int quarter = warp & 3;
     const int kh = (warp - 2) >> 2;
-    const int row = quarter * 32 + lane;  // TMEM lane = channel within the tile
-    const int n = tile_n * BN + row;
+    const int row = quarter * 32 + lane;  // TMEM lane = channel within this CTA's half
+    const int n = ch_cta + row;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    constexpr int PF = STAGES;  // weight bytes held in registers ahead of conversion
     uint4 pf[PF][2];
 #pragma unroll
     for (int i = 0; i < PF; ++i) {
@@ -217,7 +239,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         e4m3x4_to_16x4<F16>(c1.w, h[14], h[15]);
         const int s = kb % STAGES;
         if (!mbar_wait(&a_empty[s], (static_cast<uint32_t>(kb / STAGES) & 1u) ^ 1u, guard, abort_flag,
-                       ERR_TIMEOUT_GEMM_CONVERT)) {
+                       where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, kb))) {
           ok = false;
           break;
         }
@@ -226,16 +248,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[s]);
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[s]), 0));
       }
     }
 
-    // ---------------- epilogue: lane = channel, TMEM column = token
-    if (ok && mbar_wait(acc_full, 0u, guard, abort_flag, ERR_TIMEOUT_GEMM_EPILOGUE)) {
+    // ---------------- epilogue: lane = channel, TMEM column = token of the pair tile
+    if (ok && mbar_wait(acc_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_EPILOGUE, rank, 0))) {
       tc_fence_after();
       float* buf = reinterpret_cast<float*>(smem + OFF_EPI + (warp - 2) * EPI_BYTES);
       const float sc = sScale[row];
-      const int ch0 = tile_n * BN + quarter * 32;  // first channel of this warp
+      const int ch0 = ch_cta + quarter * 32;  // first channel of this warp
       const bool warp_has_channels = ch0 < p.N;
       for (int c = 0; c < 4; ++c) {
         const int tcol = kh * 128 + c * 32;  // first token column of this chunk
@@ -287,9 +309,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair MMAs or remote arrives may touch it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -314,7 +337,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, uint16_t* _
 int gemm_pick_splits(int M, int N, int K) {
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
   const int kb = (K + gemm::BK - 1) / gemm::BK;
-  int s = 148 / tiles;
+  int s = 148 / (2 * tiles);  // a tile occupies a pair of SMs
   if (s > 8) s = 8;
   if (s > kb / 16) s = kb / 16;  // keep at least 16 k-blocks per split
   return s < 1 ? 1 : s;
@@ -345,7 +368,7 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
   if (splits > 1 && (a.y_fmt != FMT_F32 || a.residual != nullptr || a.act != 0)) return cudaErrorInvalidValue;
   Params p{a.w,   a.scale,     a.y,    a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1,
            a.act, a.gelu_tanh, kb_per, static_cast<int64_t>(a.M) * a.N};
-  dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN, (kb_total + kb_per - 1) / kb_per);
+  dim3 grid(2 * ((a.M + BM - 1) / BM), (a.N + BN - 1) / BN, (kb_total + kb_per - 1) / kb_per);
   auto kern = f16 ? gemm_w8a16_kernel<true> : gemm_w8a16_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;

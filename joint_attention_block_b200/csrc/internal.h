@@ -22,6 +22,8 @@ enum : uint32_t {
   ERR_TIMEOUT_GEMM_CONVERT = 0x103,
   ERR_TIMEOUT_GEMM_EPILOGUE = 0x104,
   ERR_TIMEOUT_GEMM_DRAIN = 0x105,
+  ERR_TIMEOUT_GEMM_MMA_X = 0x106,
+  ERR_TIMEOUT_GEMM_DRAIN_MMA = 0x107,
   ERR_TIMEOUT_ATTN_PRODUCER = 0x111,
   ERR_TIMEOUT_ATTN_MMA = 0x112,
   ERR_TIMEOUT_ATTN_SOFTMAX = 0x113,

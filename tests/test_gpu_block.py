@@ -20,7 +20,8 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(autouse=True)
 def _clean_errors():
     yield
-    assert ops.poll_error() == 0, "a kernel recorded a device-side error"
+    st = ops.poll_error()
+    assert st == 0, f"a kernel recorded a device-side error: status {st}, word {ops.last_device_error():#x}"
 
 
 def run_block(shape, inp, n_text=None, gh=None, gw=None, t_img=-1, pos=None):

@@ -15,7 +15,8 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(autouse=True)
 def _clean_errors():
     yield
-    assert ops.poll_error() == 0, "a kernel recorded a device-side error"
+    st = ops.poll_error()
+    assert st == 0, f"a kernel recorded a device-side error: status {st}, word {ops.last_device_error():#x}"
 
 
 def test_e4m3_to_bf16_every_code_bit_exact():
