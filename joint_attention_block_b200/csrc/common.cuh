@@ -250,44 +250,11 @@ JAB_DEVICE uint32_t mapa_shared(uint32_t smem_addr, uint32_t rank) {
   return r;
 }
 
-// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.
-JAB_DEVICE void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-JAB_DEVICE bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait with cluster-scope acquire, for barriers that CTAs of the pair arrive on.
-JAB_DEVICE bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const KernelGuard& g, volatile uint32_t* abort_flag,
-                                  uint32_t where) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  uint32_t spins = 0;
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (((++spins) & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (g.err != nullptr && *reinterpret_cast<volatile uint32_t*>(g.err) != 0u) {
-        *abort_flag = 1u;
-        return false;
-      }
-      if (global_timer_ns() - t0 > g.timeout_ns) {
-        *abort_flag = 1u;
-        record_error(g.err, where);
-        return false;
-      }
-    }
-  }
+// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer
+// CTA), with the default (CTA-scope release) semantics: a cluster-scope release
+// would make the thread wait for all of its outstanding memory operations.
+JAB_DEVICE void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 JAB_DEVICE void cluster_sync() {

@@ -12,10 +12,11 @@
 // is sum_k a*(w8*scale[n]) up to rounding).
 //
 // The kernel computes the transposed tile D = W8_tile * A_tile^T so that the
-// widened weights are the MMA's A operand and live in TENSOR MEMORY: each converter
-// thread owns one weight row (one TMEM lane), loads its e4m3 bytes straight from
-// global memory (L2) a few stages ahead, widens them in registers and writes them
-// with tcgen05.st.  The converted weights never touch shared memory.
+// widened weights are the MMA's A operand and live in TENSOR MEMORY: TMA brings
+// each CTA's e4m3 weight tile (128 rows x 64 bytes) into shared memory, each
+// converter thread owns one weight row (one TMEM lane), widens its bytes in
+// registers and writes them with tcgen05.st.  The 16-bit weights never touch
+// shared memory.
 //
 // Two CTAs on two SMs (a cluster of 2) share one 256 (channels) x 256 (tokens) tile
 // through the pair form of the MMA (tcgen05.mma.cta_group::2, M = 256, N = 256):
@@ -24,12 +25,13 @@
 // CTA issues the MMAs, each CTA's TMEM receives its 128 channels x 256 tokens of D.
 // Per SM and K-step this reads half the activation bytes of a one-SM 128 x 256
 // tile, which is what keeps L2 traffic per FLOP low enough for the tensor pipe.
-// Both CTAs' TMA loads count on the leader's barrier, the converters arrive on it
-// remotely, and the leader's MMA commits arrive on both CTAs' barriers.  No TMA
-// load is multicast.
+// Both CTAs' TMA loads count on the leader's barrier, both CTAs' converter warps
+// arrive on the leader's barrier, and the leader's MMA commits arrive on both CTAs'
+// barriers.  No TMA load is multicast.
 //
 // Per CTA: 128 channels x 256 tokens x 64 (K) per stage; grid.z = K splits.
-//   warp 0      TMA producer: this CTA's 128 x 64 activation half (128B swizzle).
+//   warp 0      TMA producer: this CTA's 128 x 64 activation half (128B swizzle) and
+//               its 128 x 64-byte e4m3 weight tile (64B swizzle), 6-stage rings.
 //   warp 1      TMEM allocation (pair); in the leader, one lane issues the pair MMAs.
 //   warps 2..9  converters: warp w owns TMEM lanes 32*(w%4).. (channels) and half of
 //               each stage's 64 K-columns (TMEM ring of widened weights).  Then the
@@ -47,8 +49,8 @@ constexpr int BN = 256;      // output channels per pair tile (MMA M)
 constexpr int BN_CTA = 128;  // channels each CTA owns (its TMEM lanes)
 constexpr int BK = 64;
 constexpr int STAGES = 6;    // activation (smem) and widened-weight (TMEM) ring depth
-constexpr int PF = 4;        // k-blocks of weight bytes prefetched into registers
-constexpr int X_BYTES = BM_CTA * BK * 2;
+constexpr int X_BYTES = BM_CTA * BK * 2;  // one TMA box of {BK, BM_CTA} 16-bit elements
+constexpr int W_BYTES = BN_CTA * BK;      // one TMA box of {BK, BN_CTA} e4m3 bytes (64-byte swizzle)
 constexpr int THREADS = 320;
 constexpr int CVT_WARPS = 8;
 constexpr int TMEM_COLS = 512;
@@ -57,15 +59,15 @@ constexpr int A_COL = 256;   // widened weights: stage s at 256 + 32 * s
 constexpr int EPI_BYTES = 32 * 32 * 4;  // per-warp transpose buffer
 
 constexpr int OFF_X = 0;
-constexpr int OFF_EPI = OFF_X + STAGES * X_BYTES;
+constexpr int OFF_W = OFF_X + STAGES * X_BYTES;
+constexpr int OFF_EPI = OFF_W + STAGES * W_BYTES;
 constexpr int OFF_SCALE = OFF_EPI + CVT_WARPS * EPI_BYTES;
 constexpr int OFF_BAR = OFF_SCALE + BN_CTA * 4;
-constexpr int NUM_BARS = 4 * STAGES + 2;
+constexpr int NUM_BARS = 5 * STAGES + 2;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 
 struct Params {
-  const uint8_t* w;
   const float* scale;
   void* y;
   const void* residual;
@@ -86,32 +88,22 @@ __device__ __forceinline__ float gelu_f(float x, int tanh_form) {
   return 0.5f * x * (1.f + erff(x * 0.7071067811865476f));
 }
 
-// The 32 weight bytes a converter thread widens for k-block kb (zero past N or K).
-__device__ __forceinline__ void load_w(const Params& p, int n, int kb, int kh, uint4 (&v)[2]) {
-  const int k = kb * BK + kh * 32;
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    if (n < p.N && k + 16 * i < p.K) {
-      v[i] = __ldg(reinterpret_cast<const uint4*>(p.w + static_cast<size_t>(n) * p.K + k + 16 * i));
-    } else {
-      v[i] = make_uint4(0, 0, 0, 0);
-    }
-  }
-}
-
 template <bool F16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    gemm_w8a16_kernel(const __grid_constant__ CUtensorMap tm_x, const Params p, const KernelGuard guard) {
+    gemm_w8a16_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p,
+                      const KernelGuard guard) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem + OFF_X;
+  uint8_t* sW = smem + OFF_W;
   float* sScale = reinterpret_cast<float*>(smem + OFF_SCALE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* x_full = bars;               // leader: both CTAs' activation halves landed
   uint64_t* x_empty = bars + STAGES;     // both: the pair MMAs of the stage are done
   uint64_t* a_full = bars + 2 * STAGES;  // leader: both CTAs' weights widened into TMEM
   uint64_t* a_empty = bars + 3 * STAGES;
-  uint64_t* acc_full = bars + 4 * STAGES;
+  uint64_t* w_full = bars + 4 * STAGES;  // this CTA's e4m3 weight tile landed
+  uint64_t* acc_full = bars + 5 * STAGES;
   uint64_t* drain_bar = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
@@ -133,15 +125,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&x_full[s], 1);
       mbar_init(&x_empty[s], 1);
-      mbar_init(&a_full[s], 2 * CVT_WARPS);
+      mbar_init(&a_full[s], 2 * CVT_WARPS);  // used in the leader: both CTAs' converter warps
       mbar_init(&a_empty[s], 1);
+      mbar_init(&w_full[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_x);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+  }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
   for (int i = threadIdx.x; i < BN_CTA; i += THREADS) {
     const int n = ch_cta + i;
@@ -161,20 +157,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint32_t it = static_cast<uint32_t>(kb / STAGES);
       if (!mbar_wait(&x_empty[s], (it & 1u) ^ 1u, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_PRODUCER, rank, kb))) break;
       if (lane == 0) {
+        // The stage is free once its pair MMAs are done; by then this CTA's converters
+        // have also consumed the weight bytes of the stage.
+        mbar_arrive_expect_tx(&w_full[s], W_BYTES);
+        tma_load_2d(sW + s * W_BYTES, &tm_w, &w_full[s], (kb0 + kb) * BK, ch_cta);
         if (leader) mbar_arrive_expect_tx(&x_full[s], 2 * X_BYTES);
         tma_load_2d_pair(sX + s * X_BYTES, &tm_x, mapa_shared(smem_u32(&x_full[s]), 0), (kb0 + kb) * BK, tok_cta);
       }
       __syncwarp();
       issued = kb + 1;
     }
-    // The leader never leaves with copies in flight (its barrier counts both CTAs' loads);
-    // the peer is held by the final cluster barrier until the leader has drained.
-    if (leader) {
-      for (int s = 0; s < STAGES && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
-        mbar_wait(&x_full[s], static_cast<uint32_t>(last / STAGES) & 1u, guard, abort_flag,
-                  where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, s), true);
-      }
+    // Never leave with copies in flight: every CTA drains its weight loads; the leader's
+    // activation barrier counts both CTAs' activation loads, and the peer is held by the
+    // final cluster barrier until the leader has drained.
+    for (int s = 0; s < STAGES && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
+      const uint32_t par = static_cast<uint32_t>(last / STAGES) & 1u;
+      mbar_wait(&w_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, s), true);
+      if (leader) mbar_wait(&x_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, s), true);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (leader only)
@@ -184,8 +184,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int kb = 0; kb < num_kb && ok; ++kb) {
         const int s = kb % STAGES;
         const uint32_t par = static_cast<uint32_t>(kb / STAGES) & 1u;
-        ok = mbar_wait_cluster(&x_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_MMA_X, rank, kb)) &&
-             mbar_wait_cluster(&a_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_MMA, rank, kb));
+        ok = mbar_wait(&x_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_MMA_X, rank, kb)) &&
+             mbar_wait(&a_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_MMA, rank, kb));
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
@@ -213,43 +213,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int kh = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;  // TMEM lane = channel within this CTA's half
-    const int n = ch_cta + row;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    uint4 pf[PF][2];
-#pragma unroll
-    for (int i = 0; i < PF; ++i) {
-      if (i < num_kb) load_w(p, n, kb0 + i, kh, pf[i]);
-    }
     bool ok = true;
-    for (int kbase = 0; kbase < num_kb && ok; kbase += PF) {
-#pragma unroll
-      for (int i = 0; i < PF; ++i) {
-        const int kb = kbase + i;
-        if (kb >= num_kb) break;
-        const uint4 c0 = pf[i][0], c1 = pf[i][1];
-        if (kb + PF < num_kb) load_w(p, n, kb0 + kb + PF, kh, pf[i]);
-        uint32_t h[16];
-        e4m3x4_to_16x4<F16>(c0.x, h[0], h[1]);
-        e4m3x4_to_16x4<F16>(c0.y, h[2], h[3]);
-        e4m3x4_to_16x4<F16>(c0.z, h[4], h[5]);
-        e4m3x4_to_16x4<F16>(c0.w, h[6], h[7]);
-        e4m3x4_to_16x4<F16>(c1.x, h[8], h[9]);
-        e4m3x4_to_16x4<F16>(c1.y, h[10], h[11]);
-        e4m3x4_to_16x4<F16>(c1.z, h[12], h[13]);
-        e4m3x4_to_16x4<F16>(c1.w, h[14], h[15]);
-        const int s = kb % STAGES;
-        if (!mbar_wait(&a_empty[s], (static_cast<uint32_t>(kb / STAGES) & 1u) ^ 1u, guard, abort_flag,
-                       where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, kb))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_st16(tmem + lane_off + A_COL + 32 * s + 16 * kh, h);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[s]), 0));
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t par = static_cast<uint32_t>(kb / STAGES) & 1u;
+      if (!mbar_wait(&w_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, kb))) {
+        ok = false;
+        break;
       }
+      // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3).
+      const uint8_t* wrow = sW + s * W_BYTES + row * BK;
+      const uint4 c0 = *reinterpret_cast<const uint4*>(wrow + (((2 * kh) ^ ((row >> 1) & 3)) << 4));
+      const uint4 c1 = *reinterpret_cast<const uint4*>(wrow + (((2 * kh + 1) ^ ((row >> 1) & 3)) << 4));
+      uint32_t h[16];
+      e4m3x4_to_16x4<F16>(c0.x, h[0], h[1]);
+      e4m3x4_to_16x4<F16>(c0.y, h[2], h[3]);
+      e4m3x4_to_16x4<F16>(c0.z, h[4], h[5]);
+      e4m3x4_to_16x4<F16>(c0.w, h[6], h[7]);
+      e4m3x4_to_16x4<F16>(c1.x, h[8], h[9]);
+      e4m3x4_to_16x4<F16>(c1.y, h[10], h[11]);
+      e4m3x4_to_16x4<F16>(c1.z, h[12], h[13]);
+      e4m3x4_to_16x4<F16>(c1.w, h[14], h[15]);
+      if (!mbar_wait(&a_empty[s], par ^ 1u, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, kb))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st16(tmem + lane_off + A_COL + 32 * s + 16 * kh, h);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&a_full[s]), 0));
     }
 
     // ---------------- epilogue: lane = channel, TMEM column = token of the pair tile
@@ -353,11 +348,19 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
   using namespace gemm;
   if (a.M <= 0 || a.N <= 0) return cudaSuccess;
   const bool f16 = a.a_fmt == FMT_F16;
-  CUtensorMap tm_x;
+  CUtensorMap tm_x, tm_w;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.N)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(a.K)};
+    const uint32_t box[2] = {BK, BN_CTA};
+    if (!make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.w), dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
-    const uint32_t box[2] = {BK, BM};
+    const uint32_t box[2] = {BK, BM_CTA};  // each CTA of the pair loads its own 128 rows
     if (!make_tmap(&tm_x, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(a.a), dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -366,13 +369,13 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
   const int splits = a.k_splits > 1 ? a.k_splits : 1;
   const int kb_per = (kb_total + splits - 1) / splits;
   if (splits > 1 && (a.y_fmt != FMT_F32 || a.residual != nullptr || a.act != 0)) return cudaErrorInvalidValue;
-  Params p{a.w,   a.scale,     a.y,    a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1,
-           a.act, a.gelu_tanh, kb_per, static_cast<int64_t>(a.M) * a.N};
+  Params p{a.scale, a.y,         a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1,
+           a.act,   a.gelu_tanh, kb_per,     static_cast<int64_t>(a.M) * a.N};
   dim3 grid(2 * ((a.M + BM - 1) / BM), (a.N + BN - 1) / BN, (kb_total + kb_per - 1) / kb_per);
   auto kern = f16 ? gemm_w8a16_kernel<true> : gemm_w8a16_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, THREADS, SMEM_BYTES, s>>>(tm_x, p, g);
+  kern<<<grid, THREADS, SMEM_BYTES, s>>>(tm_x, tm_w, p, g);
   return cudaGetLastError();
 }
 
