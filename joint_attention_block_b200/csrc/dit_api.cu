@@ -7,7 +7,7 @@
 #include <atomic>
 #include <mutex>
 
-#include "../../include/jab_dit.h"
+#include "jab_dit.h"
 #include "internal.h"
 
 namespace jab {
