@@ -5,20 +5,25 @@
 // announcement thread), so every query attends to every key with no mask:
 //   O_h = softmax(q_h k_h^T / sqrt(hd)) v_h.
 //
-// One CTA per (batch, head, 128-query tile), flash-style over 128-key blocks:
-//   warp 0      TMA producer: Q once, then K_j and V_j into a 2-stage ring, read
-//               straight out of the fused qkv buffer [B, S, 3d] (3D tensor map).
-//   warp 1      TMEM allocation; one lane issues S_j = Q K_j^T (kind::f16, into one
-//               of two TMEM S buffers) and O += P_{j-1} V_{j-1} (P from shared
-//               memory, V read MN-major), so QK^T of block j overlaps softmax j-1.
-//   warps 2..5  softmax: thread i owns query row i (TMEM lane i), so the running
-//               max and sum are thread-local.  exp2 with the log2(e)/sqrt(hd) scale
-//               folded in; P is written as 16-bit (the q/k/v format: bf16 or f16)
-//               into a 128B-swizzled K-major tile.
-//               The running max is only raised (and O in TMEM rescaled) when it
-//               grows by more than 2^8; until then the stale max is used for both
-//               P and the row sum, which leaves O / l unchanged and keeps P <= 256.
-//               The final O / l is stored in the q/k/v format.
+// One CTA per (batch, head, 256 queries) as two 128-query tiles A and B, flash-style
+// over 128-key blocks.  Each tile owns 256 TMEM columns: S (128 fp32 columns) and O
+// (hd columns).  The two tiles ping-pong so that the tensor core works on one tile
+// while the other tile's softmax runs:
+//     MMA issue order per key block j:  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
+//   warp 0       TMA producer: Q_A and Q_B once, then K_j and V_j (2-stage ring),
+//                straight from the fused qkv buffer [B, S, 3d] (3D tensor map).
+//   warp 1       TMEM allocation; one lane issues S = Q K^T (both operands in shared
+//                memory) and O += P V with P read from TMEM (the tcgen05 A-from-TMEM
+//                form) and V read MN-major from shared memory.
+//   warps 2..5   softmax of tile A; warps 6..9 softmax of tile B.  Thread i owns query
+//                row i (TMEM lane i), so the running max and sum are thread-local.
+//                exp2 with the log2(e)/sqrt(hd) scale folded in; a quarter of the
+//                exponentials run as a polynomial on the FMA pipe so the MUFU unit is
+//                not the bottleneck.  P is written back over S in TMEM as 16-bit pairs.
+//                The running max is only raised (and O rescaled in TMEM) when it grows
+//                by more than 2^8; until then the stale max is used for both P and the
+//                row sum, which leaves O / l unchanged and keeps P <= 256.  At the end
+//                the same warps store O / l in the q/k/v format.
 #include "common.cuh"
 
 namespace jab {
@@ -26,23 +31,46 @@ namespace attn {
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+constexpr int POLY_FROM = 96;              // keys [96, 128) of a block use the polynomial exp2
 
 template <int HD>
 struct Layout {
-  static constexpr int SLAB = 128 * 128;  // 128 rows x 128 bytes (64 bf16)
+  static constexpr int SLAB = 128 * 128;  // 128 rows x 128 bytes (64 16-bit values)
   static constexpr int TILE = (HD / 64) * SLAB;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE;
-  static constexpr int OFF_V = OFF_K + 2 * TILE;
-  static constexpr int OFF_P = OFF_V + 2 * TILE;
-  static constexpr int OFF_BAR = OFF_P + 2 * SLAB;
+  static constexpr int OFF_Q = 0;                 // [2] tiles A, B
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;  // [2] stages
+  static constexpr int OFF_V = OFF_K + 2 * TILE;  // [2] stages
+  static constexpr int OFF_BAR = OFF_V + 2 * TILE;
   static constexpr int NUM_BARS = 16;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
 };
+
+// 2^x on the FMA pipe, for x <= 8: x = n + f with n = round(x), f in [-1/2, 1/2];
+// 2^f by a degree-4 polynomial (coefficients fitted to 2^f on [-1/2, 1/2] by
+// iteratively reweighted least squares on Chebyshev nodes; max relative error
+// 8.5e-6, below the f16 rounding of P); 2^n by adding n to the exponent field.
+// Adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits, and
+// (bits(t) << 23) adds exactly n << 23 because the constant's low 9 bits are 0.
+// x is clamped at -125: 2^f can sit just below 1 (exponent field 126), so n must
+// stay >= -125 for the exponent field to stay positive; 2^-125 is 0 in f16/bf16 P
+// and masked keys (x = -inf) come out as that.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float magic = 12582912.0f;  // 1.5 * 2^23
+  const float t = x + magic;
+  const float n = t - magic;
+  const float f = x - n;
+  float p = 0.00925496406853199f;
+  p = fmaf(p, f, 0.05585603043437004f);
+  p = fmaf(p, f, 0.24031251668930054f);
+  p = fmaf(p, f, 0.693130612373352f);
+  p = fmaf(p, f, 0.9999977946281433f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
 
 template <int HD, int F>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -55,24 +83,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
-  uint8_t* sP = smem + L::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_full = bars + 1;    // [2] stages
   uint64_t* v_full = bars + 3;    // [2]
   uint64_t* kv_empty = bars + 5;  // [2]
-  uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* s_empty = bars + 9;   // [2]
-  uint64_t* p_full = bars + 11;
-  uint64_t* p_empty = bars + 12;
-  uint64_t* o_full = bars + 13;
-  uint64_t* drain_bar = bars + 14;
+  uint64_t* s_full = bars + 7;    // [2] tiles: S_t(j) ready (and PV_t(j-1) done)
+  uint64_t* p_full = bars + 9;    // [2] tiles: P_t(j) in TMEM, O_t rescaled
+  uint64_t* o_full = bars + 11;   // both tiles' O final
+  uint64_t* drain_bar = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 4);
 
   const int warp = static_cast<int>(warp_id());
   const int lane = static_cast<int>(lane_id());
-  const int q0 = blockIdx.x * BQ;
+  const int q0 = blockIdx.x * 2 * BQ;
   const int head = blockIdx.y;
   const int b = blockIdx.z;
   const int d = n_heads * HD;
@@ -85,10 +110,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(p_empty, 1);
     mbar_init(o_full, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
@@ -100,20 +123,23 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_o = tmem + 256;
 
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, L::TILE);
-      for (int c = 0; c < HD / 64; ++c) tma_load_3d(sQ + c * L::SLAB, &tm, q_full, head * HD + 64 * c, q0, b);
+      mbar_arrive_expect_tx(q_full, 2 * L::TILE);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < HD / 64; ++c)
+          tma_load_3d(sQ + t * L::TILE + c * L::SLAB, &tm, q_full, head * HD + 64 * c, q0 + t * BQ, b);
     }
     __syncwarp();
     int issued = 0;
     for (int j = 0; j < nb; ++j) {
       const int st = j & 1;
       const uint32_t it = static_cast<uint32_t>(j >> 1);
-      if (!mbar_wait(&kv_empty[st], (it & 1u) ^ 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_PRODUCER)) break;
+      if (!mbar_wait(&kv_empty[st], (it & 1u) ^ 1u, guard, abort_flag,
+                     where_code(ERR_TIMEOUT_ATTN_PRODUCER, 0, j)))
+        break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&k_full[st], L::TILE);
         for (int c = 0; c < HD / 64; ++c)
@@ -125,103 +151,120 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       issued = j + 1;
     }
-    mbar_wait(q_full, 0u, guard, abort_flag, ERR_TIMEOUT_ATTN_DRAIN, true);
+    // Never leave with copies in flight.
+    mbar_wait(q_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_DRAIN, 0, 0), true);
     for (int st = 0; st < 2 && st < issued; ++st) {
       const int last = st + ((issued - 1 - st) / 2) * 2;
       const uint32_t it = static_cast<uint32_t>(last >> 1);
-      mbar_wait(&k_full[st], it & 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_DRAIN, true);
-      mbar_wait(&v_full[st], it & 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_DRAIN, true);
+      mbar_wait(&k_full[st], it & 1u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_DRAIN, 0, last), true);
+      mbar_wait(&v_full[st], it & 1u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_DRAIN, 0, last), true);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     constexpr uint32_t idesc_s = idesc_f16kind(BQ, BKV, kF16, false, false);
     constexpr uint32_t idesc_o = idesc_f16kind(BQ, HD, kF16, false, true);
-    bool ok = mbar_wait(q_full, 0u, guard, abort_flag, ERR_TIMEOUT_ATTN_MMA);
-    auto issue_pv = [&](int i) -> bool {
-      const int st = i & 1;
-      if (!mbar_wait(&v_full[st], static_cast<uint32_t>(i >> 1) & 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_MMA))
-        return false;
-      if (!mbar_wait(p_full, static_cast<uint32_t>(i) & 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_MMA)) return false;
+    auto issue_s = [&](int t, int j) {  // S_t(j) = Q_t K_j^T into columns [256 t, 256 t + 128)
+      const uint32_t qbase = smem_u32(sQ + t * L::TILE);
+      const uint32_t kbase = smem_u32(sK + (j & 1) * L::TILE);
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * L::SLAB + (kk & 3) * 32;
+        mma_f16kind_ss(tmem + 256 * t, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                       idesc_s, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(&s_full[t]);
+    };
+    auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P from TMEM (columns [256 t, 256 t + 64))
+      const uint32_t vbase = smem_u32(sV + (j & 1) * L::TILE);
+#pragma unroll
+      for (int kk = 0; kk < BKV / 16; ++kk) {
+        const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, L::SLAB, 1024);
+        mma_f16kind_ts(tmem + 256 * t + 128, tmem + 256 * t + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+    };
+    bool ok = mbar_wait(q_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 0, 0)) &&
+              mbar_wait(&k_full[0], 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 0, 0));
+    if (ok) {
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t pbase = smem_u32(sP);
-        const uint32_t vbase = smem_u32(sV + st * L::TILE);
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(pbase + (kk >> 2) * L::SLAB + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, L::SLAB, 1024);
-          mma_f16kind_ss(tmem_o, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(p_empty);
-        mma_commit(&kv_empty[st]);
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
       __syncwarp();
-      return true;
-    };
+    }
     for (int j = 0; j < nb && ok; ++j) {
       const int st = j & 1;
-      ok = mbar_wait(&k_full[st], static_cast<uint32_t>(j >> 1) & 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_MMA) &&
-           mbar_wait(&s_empty[st], (static_cast<uint32_t>(j >> 1) & 1u) ^ 1u, guard, abort_flag,
-                     ERR_TIMEOUT_ATTN_MMA);
+      const uint32_t par = static_cast<uint32_t>(j) & 1u;
+      const bool next = j + 1 < nb;
+      ok = mbar_wait(&v_full[st], static_cast<uint32_t>(j >> 1) & 1u, guard, abort_flag,
+                     where_code(ERR_TIMEOUT_ATTN_MMA, 1, j)) &&
+           mbar_wait(&p_full[0], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 2, j)) &&
+           (!next || mbar_wait(&k_full[(j + 1) & 1], static_cast<uint32_t>((j + 1) >> 1) & 1u, guard, abort_flag,
+                               where_code(ERR_TIMEOUT_ATTN_MMA, 3, j)));
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t qbase = smem_u32(sQ);
-        const uint32_t kbase = smem_u32(sK + st * L::TILE);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::SLAB + (kk & 3) * 32;
-          mma_f16kind_ss(tmem + st * BKV, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                      idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&s_full[st]);
+        issue_pv(0, j);
+        if (next) issue_s(0, j + 1);  // overwrites P_A(j) only after PV_A(j) has read it (in-order issue)
       }
       __syncwarp();
-      if (j > 0) ok = issue_pv(j - 1);
+      ok = mbar_wait(&p_full[1], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 4, j));
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        issue_pv(1, j);
+        mma_commit(&kv_empty[st]);  // K_j and V_j fully consumed by both tiles
+        if (next) issue_s(1, j + 1);
+      }
+      __syncwarp();
     }
-    if (ok) ok = issue_pv(nb - 1);
     if (lane == 0) {
       if (ok) mma_commit(o_full);
       mma_commit(drain_bar);
     }
     __syncwarp();
-    mbar_wait(drain_bar, 0u, guard, abort_flag, ERR_TIMEOUT_ATTN_DRAIN, true);
+    mbar_wait(drain_bar, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_DRAIN, 1, 0), true);
   } else {
-    // ---------------- softmax (warps 2..5): thread owns query row 32*(warp%4) + lane
+    // ---------------- softmax: warps 2..5 -> tile A, 6..9 -> tile B; thread owns query row
+    const int t = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_col = tmem + lane_off + 256 * t;
+    const uint32_t o_col = s_col + 128;
     const float c_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
     float m_used = -INFINITY;
     float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nb && ok; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&s_full[st], static_cast<uint32_t>(j >> 1) & 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_SOFTMAX)) {
+    for (int j = 0; j < nb; ++j) {
+      if (!mbar_wait(&s_full[t], static_cast<uint32_t>(j) & 1u, guard, abort_flag,
+                     where_code(ERR_TIMEOUT_ATTN_SOFTMAX, t, j))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tmem + lane_off + st * BKV + 32 * c, raw);
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) s[32 * c + k] = __uint_as_float(raw[k]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[st]);
-
       const int valid = seq - j * BKV;  // keys beyond the sequence are masked
+      const bool full = valid >= BKV;    // every block but possibly the last
+      // pass 1: row max of the scaled logits (S read from TMEM 64 columns at a time)
       float mx = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < BKV; ++k) {
-        s[k] = k < valid ? s[k] * c_log2 : -INFINITY;
-        mx = fmaxf(mx, s[k]);
+      for (int c = 0; c < BKV / 64; ++c) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(s_col + 64 * c, r0);
+        tmem_ld32(s_col + 64 * c + 32, r1);
+        tmem_ld_wait();
+        if (full) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fmaxf(__uint_as_float(r0[k]), __uint_as_float(r1[k])));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            if (64 * c + k < valid) mx = fmaxf(mx, __uint_as_float(r0[k]));
+            if (64 * c + 32 + k < valid) mx = fmaxf(mx, __uint_as_float(r1[k]));
+          }
+        }
       }
+      mx *= c_log2;
       float alpha = 1.f;
       bool rescale = false;
       if (mx > m_used + RESCALE_THRESHOLD) {
@@ -229,68 +272,77 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_used = mx;
         rescale = true;
       }
-      float sum = 0.f;
-#pragma unroll
-      for (int k = 0; k < BKV; ++k) {
-        s[k] = ex2_approx(s[k] - m_used);
-        sum += s[k];
-      }
-      l = l * alpha + sum;
-
-      // PV of the previous block must be done: P buffer free, O current.
-      if (j > 0 &&
-          !mbar_wait(p_empty, static_cast<uint32_t>(j - 1) & 1u, guard, abort_flag, ERR_TIMEOUT_ATTN_SOFTMAX)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      // O_t is up to date here: PV_t(j-1) was issued before S_t(j) and s_full covers it.
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t raw[32];
-          tmem_ld32(tmem_o + lane_off + 32 * c, raw);
+          tmem_ld32(o_col + 32 * c, raw);
           tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 32; ++k) raw[k] = __float_as_uint(__uint_as_float(raw[k]) * alpha);
-          tmem_st32(tmem_o + lane_off + 32 * c, raw);
+          tmem_st32(o_col + 32 * c, raw);
         }
-        tmem_st_wait();
       }
-      // P row -> 16-bit, 128B-swizzled K-major (two 64-key slabs)
+      // pass 2, two halves of 64 keys: exponentiate, sum, and write P_t(j) as 16-bit pairs
+      // over the first 64 columns of S_t (the A operand of the PV MMA).  Half h reads S
+      // columns [64h, 64h + 64) and writes P columns [32h, 32h + 32), which hold S values
+      // already consumed.
+      float sum = 0.f;
 #pragma unroll
-      for (int kc = 0; kc < BKV / 8; ++kc) {
-        uint4 o;
-        o.x = pack2<F>(s[8 * kc + 0], s[8 * kc + 1]);
-        o.y = pack2<F>(s[8 * kc + 2], s[8 * kc + 3]);
-        o.z = pack2<F>(s[8 * kc + 4], s[8 * kc + 5]);
-        o.w = pack2<F>(s[8 * kc + 6], s[8 * kc + 7]);
-        uint8_t* dst = sP + (kc >> 3) * L::SLAB + r * 128 + ((((kc & 7) ^ (r & 7))) << 4);
-        *reinterpret_cast<uint4*>(dst) = o;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t raw[64];
+        uint32_t* r0 = raw;
+        uint32_t* r1 = raw + 32;
+        tmem_ld32(s_col + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(r0));
+        tmem_ld32(s_col + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(r1));
+        tmem_ld_wait();
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const int key = 64 * h + k;
+          float x0 = fmaf(__uint_as_float(raw[k]), c_log2, -m_used);
+          float x1 = fmaf(__uint_as_float(raw[k + 1]), c_log2, -m_used);
+          if (!full) {
+            x0 = key < valid ? x0 : -INFINITY;
+            x1 = key + 1 < valid ? x1 : -INFINITY;
+          }
+          float e0, e1;
+          if (key < POLY_FROM) {
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
+          } else {
+            e0 = exp2_poly(x0);
+            e1 = exp2_poly(x1);
+          }
+          sum += e0 + e1;
+          pk[k / 2] = pack2<F>(e0, e1);
+        }
+        tmem_st32(s_col + 32 * h, pk);
       }
-      fence_proxy_async_smem();
+      l = l * alpha + sum;
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait(o_full, 0u, guard, abort_flag, ERR_TIMEOUT_ATTN_SOFTMAX)) {
+    if (ok && mbar_wait(o_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_SOFTMAX, 2 + t, 0))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const int row = q0 + r;
+      const int row = q0 + t * BQ + r;
       uint16_t* dst = out + (static_cast<size_t>(b) * seq + row) * d + head * HD;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t raw[32];
-        tmem_ld32(tmem_o + lane_off + 32 * c, raw);
+        tmem_ld32(o_col + 32 * c, raw);
         tmem_ld_wait();
         if (row < seq) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 o;
-            o.x = pack2<F>(__uint_as_float(raw[8 * q + 0]) * inv_l, __uint_as_float(raw[8 * q + 1]) * inv_l);
-            o.y = pack2<F>(__uint_as_float(raw[8 * q + 2]) * inv_l, __uint_as_float(raw[8 * q + 3]) * inv_l);
-            o.z = pack2<F>(__uint_as_float(raw[8 * q + 4]) * inv_l, __uint_as_float(raw[8 * q + 5]) * inv_l);
-            o.w = pack2<F>(__uint_as_float(raw[8 * q + 6]) * inv_l, __uint_as_float(raw[8 * q + 7]) * inv_l);
-            reinterpret_cast<uint4*>(dst + 32 * c)[q] = o;
+            float v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = __uint_as_float(raw[8 * q + k]) * inv_l;
+            store8<F>(dst + 32 * c, q, v);
           }
         }
       }
@@ -312,7 +364,7 @@ cudaError_t launch_hd(const CUtensorMap& tm, void* out, int batch, int seq, int 
   cudaError_t e =
       cudaFuncSetAttribute(attention_kernel<HD, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((seq + BQ - 1) / BQ, n_heads, batch);
+  dim3 grid((seq + 2 * BQ - 1) / (2 * BQ), n_heads, batch);
   attention_kernel<HD, F><<<grid, THREADS, L::SMEM, s>>>(tm, static_cast<uint16_t*>(out), seq, n_heads, g);
   return cudaGetLastError();
 }
