@@ -195,6 +195,12 @@ DIT_API int dit_profile_read(int* tags, float* ms, int max_records);
  * CTA's rank in its cluster, bits 16..31 the k-block / loop index. */
 DIT_API uint32_t dit_last_device_error(void);
 
+/* Launch a one-thread kernel whose only wait can never complete: it gives up after the
+ * configured limit (dit_set_wait_timeout_ms) and records a timeout, which the next
+ * dit_poll_error() reports as DIT_ERR_TIMEOUT.  Exercises the failure path of every
+ * pipelined kernel here without faulting or hanging the device. */
+DIT_API int dit_wait_selftest(void* stream);
+
 /* Set the wall-time limit of every device-side bounded wait (default 2000 ms). */
 DIT_API int dit_set_wait_timeout_ms(uint32_t ms);
 

@@ -80,6 +80,7 @@ SIGNATURES = {
     "dit_profile_read": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float), _I]),
     "dit_set_wait_timeout_ms": (_I, [ctypes.c_uint32]),
     "dit_last_device_error": (ctypes.c_uint32, []),
+    "dit_wait_selftest": (_I, [_P]),
     "dit_status_str": (ctypes.c_char_p, [_I]),
     "dit_abi_version": (_I, []),
 }
@@ -238,6 +239,10 @@ def profile_read(max_records: int = 1 << 16):
 
 def poll_error(stream=None) -> int:
     return int(lib().dit_poll_error(_stream(stream)))
+
+
+def wait_selftest(stream=None) -> None:
+    _check("dit_wait_selftest", lib().dit_wait_selftest(_stream(stream)))
 
 
 def last_device_error() -> int:

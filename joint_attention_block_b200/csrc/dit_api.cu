@@ -251,6 +251,12 @@ int dit_poll_error(void* stream) {
   return (v & 0xF00u) == 0x100u ? DIT_ERR_TIMEOUT : DIT_ERR_DEVICE;
 }
 
+int dit_wait_selftest(void* stream) {
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  return from_cuda(launch_wait_selftest(g, as_stream(stream)));
+}
+
 int dit_e4m3_to_bf16(const uint8_t* codes, void* out, int64_t n, void* stream) {
   if (n < 0 || (n > 0 && (codes == nullptr || out == nullptr))) return DIT_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(out)) return DIT_ERR_INVALID_ARG;

@@ -324,4 +324,23 @@ cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_he
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ bounded-wait self test
+
+// One thread waits on an mbarrier that nothing arrives on; the bounded wait must give
+// up after the guard's limit and record ERR_TIMEOUT_SELFTEST, leaving the context usable.
+__global__ void wait_selftest_kernel(const KernelGuard guard) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0u;
+  fence_barrier_init();
+  mbar_wait(&bar, 0u, guard, &abort_flag, ERR_TIMEOUT_SELFTEST);
+}
+
+cudaError_t launch_wait_selftest(const KernelGuard& g, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(g);
+  return cudaGetLastError();
+}
+
 }  // namespace jab

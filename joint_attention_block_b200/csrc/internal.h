@@ -28,6 +28,7 @@ enum : uint32_t {
   ERR_TIMEOUT_ATTN_MMA = 0x112,
   ERR_TIMEOUT_ATTN_SOFTMAX = 0x113,
   ERR_TIMEOUT_ATTN_DRAIN = 0x114,
+  ERR_TIMEOUT_SELFTEST = 0x1F0,
 };
 
 // Guard for the current device (error word address + configured timeout).
@@ -77,6 +78,9 @@ int gemm_pick_splits(int M, int N, int K);
 cudaError_t launch_splitk_reduce(const float* part, uint16_t* out, int64_t n, int splits, cudaStream_t s);
 
 // qkv and out in fmt (bf16 or f16).
+// A kernel whose only wait never completes (exercises the bounded-wait path).
+cudaError_t launch_wait_selftest(const KernelGuard& g, cudaStream_t s);
+
 cudaError_t launch_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
                              const KernelGuard& g, cudaStream_t s);
 

@@ -70,3 +70,4 @@ def test_argument_validation_without_gpu(lib):
     assert lib.dit_rmsnorm_rows(16, 0, 16, 16, 1, 4, 16, 1e-6, None) == 1  # in place with a format change
     assert lib.dit_joint_attention(16, 32, 2, 1, 8, 2, 64, None) == 1  # fp32 q/k/v
     assert lib.dit_joint_attention(16, 32, 1, 1, 8, 2, 96, None) == 2  # head_dim 96
+

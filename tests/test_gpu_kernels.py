@@ -187,3 +187,22 @@ def test_joint_attention(S, H, hd, batch, fmt):
 def test_bounded_wait_timeout_is_not_hit_in_normal_runs():
     ops.set_wait_timeout_ms(2000)
     assert ops.poll_error() == 0
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """A wait that nothing completes times out, is reported, and the next kernels still run."""
+    ops.set_wait_timeout_ms(100)
+    try:
+        ops.wait_selftest()
+        assert ops.poll_error() == 5  # DIT_ERR_TIMEOUT
+        assert ops.last_device_error() & 0xFFF == 0x1F0
+        assert ops.poll_error() == 0  # the error word was cleared
+    finally:
+        ops.set_wait_timeout_ms(2000)
+    # the context is still usable: a real kernel after the timeout is exact
+    codes = np.arange(256, dtype=np.uint8)
+    out = empty_bf16(256)
+    ops.e4m3_to_bf16(dev(codes), out)
+    ref = oracle.e4m3_to_f64(codes)
+    fin = ~np.isnan(ref)
+    assert np.array_equal(bits(out)[fin], (ref[fin].astype(np.float32).view(np.uint32) >> 16).astype(np.uint16))
