@@ -227,7 +227,6 @@ def run_reference(args, rank, world):
 
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     from joint_attention_block_b200 import ops
 
@@ -263,16 +262,12 @@ def run_ours(args, rank, world, local_rank):
         ops.dit_block_forward(cfg, weights, x_in, x_out, s.n_text, s.grid_h, s.grid_w, ws_blk, stream=stream)
         ops.euler_cfg_step(lat, vc, vu, synth.CFG_GUIDANCE, dt, stream=stream)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    from joint_attention_block_b200 import replicas
+
+    barrier = replicas.barrier
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, dev)
 
     for i in range(args.warmup):
         step()
