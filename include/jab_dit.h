@@ -101,6 +101,27 @@ DIT_API int dit_block_forward(const dit_block_config* cfg, const dit_block_weigh
                       int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                       void* workspace, size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch behind dit_block_forward_noalloc (32 MiB).  Every GPU
+ * that loads this library holds this much device memory until the process exits. */
+#define DIT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* dit_block_forward for callers that cannot allocate device memory: hosts that reserve all
+ * device memory at start-up, plugin interfaces that pass a kernel only its inputs and outputs,
+ * or latency-critical paths where an allocation (which may synchronise the device) is not
+ * acceptable.  The pages describe no such call; it exists for these integrators.
+ * Same arguments and results as dit_block_forward, minus the workspace: the intermediates live
+ * in a fixed array of DIT_NOALLOC_SCRATCH_BYTES inside the library.  No allocation happens.
+ * Limits and behaviour:
+ *  - shapes whose dit_block_workspace_bytes() exceeds DIT_NOALLOC_SCRATCH_BYTES return
+ *    DIT_ERR_UNSUPPORTED (e.g. the tiny 16 + 8x8 block fits; the 1024 px block does not);
+ *  - the first call on a device looks up the array's device address with that device
+ *    current; make that first call before any stream capture;
+ *  - all calls share the one array and it keeps the last call's contents; calls that
+ *    overlap on the GPU (other streams, other threads) race on it, so serialise them. */
+DIT_API int dit_block_forward_noalloc(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in,
+                                      void* x_out, int batch, int n_text, int grid_h, int grid_w, int t_img,
+                                      const int32_t* pos, void* stream);
+
 /* Bytes of device workspace cond_proj_forward needs: the normalised features (f16) and,
  * when the token count leaves SMs idle, fp32 split-K partial sums of the projection. */
 DIT_API size_t cond_proj_workspace_bytes(int n_tok, int n_layers, int hidden, int d_out);

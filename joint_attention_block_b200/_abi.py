@@ -65,6 +65,8 @@ SIGNATURES = {
     "dit_block_workspace_bytes": (_SZ, [ctypes.POINTER(BlockConfig), _I, _I, _I, _I]),
     "dit_block_forward": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I, _I, _I, _I,
                                _P, _P, _SZ, _P]),
+    "dit_block_forward_noalloc": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I,
+                                       _I, _I, _I, _P, _P]),
     "cond_proj_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "cond_proj_forward": (_I, [_P, _I, _I, _I, _P, _F, _P, _P, _I, _P, _P, _SZ, _P]),
     "euler_cfg_step": (_I, [_P, _P, _P, _I64, _F, _F, _P]),
@@ -153,6 +155,18 @@ def dit_block_forward(cfg: BlockConfig, weights: BlockWeights, x: torch.Tensor, 
     _check("dit_block_forward", lib().dit_block_forward(
         ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
         _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # DIT_NOALLOC_SCRATCH_BYTES
+
+
+def dit_block_forward_noalloc(cfg: BlockConfig, weights: BlockWeights, x: torch.Tensor, out: torch.Tensor,
+                              n_text: int, grid_h: int, grid_w: int, t_img: int = -1,
+                              pos: Optional[torch.Tensor] = None, stream=None) -> None:
+    """dit_block_forward without a workspace: the library's fixed device scratch is used instead."""
+    _check("dit_block_forward_noalloc", lib().dit_block_forward_noalloc(
+        ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
+        _ptr(pos), _stream(stream)))
 
 
 def cond_proj_workspace_bytes(n_tok: int, n_layers: int, hidden: int, d_out: int) -> int:

@@ -71,3 +71,14 @@ def test_argument_validation_without_gpu(lib):
     assert lib.dit_joint_attention(16, 32, 2, 1, 8, 2, 64, None) == 1  # fp32 q/k/v
     assert lib.dit_joint_attention(16, 32, 1, 1, 8, 2, 96, None) == 2  # head_dim 96
 
+
+def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
+    """The 1024 px block needs more than the fixed scratch: rejected before any device work."""
+    from joint_attention_block_b200 import synth
+    s = synth.C1024
+    cfg = _abi.make_config(s)
+    assert lib.dit_block_workspace_bytes(ctypes.byref(cfg), 1, s.n_text, s.grid_h, s.grid_w) > _abi.NOALLOC_SCRATCH_BYTES
+    w = _abi.BlockWeights()
+    rc = lib.dit_block_forward_noalloc(ctypes.byref(cfg), ctypes.byref(w), None, None, 1, s.n_text, s.grid_h,
+                                       s.grid_w, -1, None, None)
+    assert rc == 2  # DIT_ERR_UNSUPPORTED
