@@ -120,6 +120,31 @@ JAB_DEVICE void store8(void* base, int64_t idx8, const float (&v)[8]) {
   }
 }
 
+// Load / store 4 consecutive values of format F (16-bit: one 8-byte vector; f32: 16 bytes).
+template <int F>
+JAB_DEVICE float4 load4(const void* base, int64_t idx4) {
+  if constexpr (F == FMT_F32) {
+    return reinterpret_cast<const float4*>(base)[idx4];
+  } else {
+    const uint2 a = reinterpret_cast<const uint2*>(base)[idx4];
+    return make_float4(unpack_lo<F>(a.x), unpack_hi<F>(a.x), unpack_lo<F>(a.y), unpack_hi<F>(a.y));
+  }
+}
+template <int F>
+JAB_DEVICE void store4(void* base, int64_t idx4, float4 v) {
+  if constexpr (F == FMT_F32) {
+    reinterpret_cast<float4*>(base)[idx4] = v;
+  } else {
+    reinterpret_cast<uint2*>(base)[idx4] = make_uint2(pack2<F>(v.x, v.y), pack2<F>(v.z, v.w));
+  }
+}
+
+JAB_DEVICE float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 JAB_DEVICE float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -294,6 +319,19 @@ JAB_DEVICE void mma_f16kind_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b
       : "memory");
 }
 
+// Pair MMA issued by the leader CTA with both operands in shared memory: D (M=256
+// over both CTAs' TMEM) (+)= A (128 rows in each CTA) * B (N/2 rows in each CTA)^T.
+// Both descriptors give the same shared-memory offsets in the two CTAs.
+JAB_DEVICE void mma_f16kind_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                    uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the mbarrier at this shared-memory offset in every CTA of `cta_mask`
 // once all pair MMAs issued so far by this thread are done.
 JAB_DEVICE void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -331,6 +369,26 @@ JAB_DEVICE void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int3
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// TMA tiled stores from this CTA's shared memory, tracked by bulk groups.
+JAB_DEVICE void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+JAB_DEVICE void tma_store_3d(const CUtensorMap* m, const void* src, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+JAB_DEVICE void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+JAB_DEVICE void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -432,6 +490,19 @@ JAB_DEVICE void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
 
 JAB_DEVICE void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 JAB_DEVICE void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Wait for this thread's TMEM loads, then pass `r` through an empty asm so that no use of
+// the loaded registers can be scheduled above the wait (they are written asynchronously).
+JAB_DEVICE void tmem_ld_wait_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+  asm volatile("" : "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+// Prefetch `bytes` (a multiple of 16, 16-byte aligned address) of global memory into L2.
+JAB_DEVICE void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
+}
 
 JAB_DEVICE uint32_t warp_id() { return threadIdx.x >> 5; }
 JAB_DEVICE uint32_t lane_id() { return threadIdx.x & 31u; }

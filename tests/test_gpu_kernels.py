@@ -136,6 +136,28 @@ def test_gemm_dequant_is_exact_inside_the_mma():
         assert np.array_equal(_fmt_values(y, 2), want), f"a_fmt={a_fmt}"
 
 
+@pytest.mark.parametrize("gelu_tanh", [0, 1], ids=["erf", "tanh"])
+def test_gemm_gelu_epilogue_accuracy(gelu_tanh):
+    """W8 = identity, scale = 1: Y = GELU(A) on 131,072 f16 values across [-12, 12] plus extremes.
+
+    The accumulator is exact here, so what is left is the epilogue's GELU against the
+    oracle's: fp32 evaluation with an erf (or tanh) approximation good to ~1e-7.
+    """
+    M, K = 512, 256
+    vals = np.linspace(-12.0, 12.0, M * K).astype(np.float16)
+    vals[:6] = np.array([-65504.0, 65504.0, -300.0, 300.0, 0.0, -0.0], dtype=np.float16)
+    a = torch.from_numpy(vals.reshape(M, K)).cuda()
+    eye = np.zeros((K, K), dtype=np.uint8)
+    eye[np.arange(K), np.arange(K)] = 0x38  # e4m3 code of 1.0
+    y = _fmt_empty((M, K), 2)
+    ops.gemm_w8a16(a, dev(eye), dev(np.ones(K, dtype=np.float32)), y, act=1, gelu_tanh=gelu_tanh, a_fmt=1, y_fmt=2)
+    x = vals.astype(np.float64).reshape(M, K)
+    ref = oracle.gelu(x, tanh=bool(gelu_tanh))
+    got = _fmt_values(y, 2)
+    err = np.abs(got - ref) / np.maximum(1.0, np.abs(x))
+    assert np.all(np.isfinite(got)) and err.max() <= 5e-7, f"max scaled error {err.max():.3e}"
+
+
 def _tiny_qkv(shape, seed=3, n_text=None, gh=None, gw=None, batch=1):
     n_text = shape.n_text if n_text is None else n_text
     gh = shape.grid_h if gh is None else gh
