@@ -17,9 +17,9 @@
 //                form) and V read MN-major from shared memory.
 //   warps 2..5   softmax of tile A; warps 6..9 softmax of tile B.  Thread i owns query
 //                row i (TMEM lane i), so the running max and sum are thread-local.
-//                exp2 with the log2(e)/sqrt(hd) scale folded in; a quarter of the
-//                exponentials run as a polynomial on the FMA pipe so the MUFU unit is
-//                not the bottleneck.  P is written back over S in TMEM as 16-bit pairs.
+//                The whole row of S is read from TMEM at once; exp2 with the
+//                log2(e)/sqrt(hd) scale folded in (packed fp32 pair arithmetic for the
+//                scaling and the row sums).  P is written back over S in TMEM as 16-bit pairs.
 //                The running max is only raised (and O rescaled in TMEM) when it grows
 //                by more than 2^8; until then the stale max is used for both P and the
 //                row sum, which leaves O / l unchanged and keeps P <= 256.  At the end
@@ -34,7 +34,7 @@ constexpr int BKV = 128;
 constexpr int THREADS = 320;
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
-constexpr int POLY_FROM = 96;              // keys [96, 128) of a block use the polynomial exp2
+constexpr int POLY_FROM = 128;             // keys [POLY_FROM, 128) of a block use the polynomial exp2
 
 template <int HD>
 struct Layout {
@@ -50,9 +50,9 @@ struct Layout {
 };
 
 // 2^x on the FMA pipe, for x <= 8: x = n + f with n = round(x), f in [-1/2, 1/2];
-// 2^f by a degree-4 polynomial (coefficients fitted to 2^f on [-1/2, 1/2] by
+// 2^f by a degree-3 polynomial (coefficients fitted to 2^f on [-1/2, 1/2] by
 // iteratively reweighted least squares on Chebyshev nodes; max relative error
-// 8.5e-6, below the f16 rounding of P); 2^n by adding n to the exponent field.
+// 7.5e-5, below the f16 rounding of P); 2^n by adding n to the exponent field.
 // Adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits, and
 // (bits(t) << 23) adds exactly n << 23 because the constant's low 9 bits are 0.
 // x is clamped at -125: 2^f can sit just below 1 (exponent field 126), so n must
@@ -64,12 +64,18 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const float t = x + magic;
   const float n = t - magic;
   const float f = x - n;
-  float p = 0.00925496406853199f;
-  p = fmaf(p, f, 0.05585603043437004f);
-  p = fmaf(p, f, 0.24031251668930054f);
-  p = fmaf(p, f, 0.693130612373352f);
-  p = fmaf(p, f, 0.9999977946281433f);
+  float p = 0.05517163500189781f;
+  p = fmaf(p, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// max(a, b, c) in one instruction (three-input form of max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 template <int HD, int F>
@@ -245,26 +251,41 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int valid = seq - j * BKV;  // keys beyond the sequence are masked
       const bool full = valid >= BKV;    // every block but possibly the last
-      // pass 1: row max of the scaled logits (S read from TMEM 64 columns at a time)
-      float mx = -INFINITY;
+      // The whole row of S (128 keys) comes out of TMEM in one round trip; the max and the
+      // exponentials then run from registers with independent partial results.
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32(s_col, s0);
+      tmem_ld32(s_col + 32, s1);
+      tmem_ld32(s_col + 64, s2);
+      tmem_ld32(s_col + 96, s3);
+      tmem_ld_wait_regs(s0);
+      tmem_ld_wait_regs(s1);
+      tmem_ld_wait_regs(s2);
+      tmem_ld_wait_regs(s3);
+      float v[BKV];
 #pragma unroll
-      for (int c = 0; c < BKV / 64; ++c) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(s_col + 64 * c, r0);
-        tmem_ld32(s_col + 64 * c + 32, r1);
-        tmem_ld_wait();
-        if (full) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fmaxf(__uint_as_float(r0[k]), __uint_as_float(r1[k])));
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (64 * c + k < valid) mx = fmaxf(mx, __uint_as_float(r0[k]));
-            if (64 * c + 32 + k < valid) mx = fmaxf(mx, __uint_as_float(r1[k]));
-          }
-        }
+      for (int k = 0; k < 32; ++k) {
+        v[k] = __uint_as_float(s0[k]);
+        v[32 + k] = __uint_as_float(s1[k]);
+        v[64 + k] = __uint_as_float(s2[k]);
+        v[96 + k] = __uint_as_float(s3[k]);
       }
-      mx *= c_log2;
+      if (!full) {
+#pragma unroll
+        for (int k = 0; k < BKV; ++k) v[k] = k < valid ? v[k] : -INFINITY;
+      }
+      // row max: 8 independent chains of three-input maxima, then a short tree
+      float m8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = fmax3(v[k], v[8 + k], v[16 + k]);
+#pragma unroll
+      for (int i = 24; i < BKV - 8; i += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], v[i + k], v[i + 8 + k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], v[BKV - 8 + k]);
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * c_log2;
       float alpha = 1.f;
       bool rescale = false;
       if (mx > m_used + RESCALE_THRESHOLD) {
@@ -272,53 +293,45 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_used = mx;
         rescale = true;
       }
+      // exponentiate, sum, and write P_t(j) as 16-bit pairs over the first 64 columns of S_t
+      // (the A operand of the PV MMA)
+      float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 c2 = make_float2(c_log2, c_log2);
+      const float2 nm2 = make_float2(-m_used, -m_used);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k2 = 0; k2 < 64; k2 += 2) {
+          const int k = 64 * h + k2;
+          const float2 x = fma2(make_float2(v[k], v[k + 1]), c2, nm2);  // packed pair: s c - m
+          float2 e;
+          if (k < POLY_FROM) {
+            e.x = ex2_approx(x.x);
+            e.y = ex2_approx(x.y);
+          } else {
+            e.x = exp2_poly(x.x);
+            e.y = exp2_poly(x.y);
+          }
+          ps[(k2 >> 1) & 3] = add2(ps[(k2 >> 1) & 3], e);
+          pk[k2 >> 1] = pack2<F>(e.x, e.y);
+        }
+        tmem_st32(s_col + 32 * h, pk);
+      }
+      const float2 ps01 = add2(ps[0], ps[1]), ps23 = add2(ps[2], ps[3]);
+      const float2 ps03 = add2(ps01, ps23);
+      const float sum = ps03.x + ps03.y;
       // O_t is up to date here: PV_t(j-1) was issued before S_t(j) and s_full covers it.
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t raw[32];
           tmem_ld32(o_col + 32 * c, raw);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(raw);
 #pragma unroll
           for (int k = 0; k < 32; ++k) raw[k] = __float_as_uint(__uint_as_float(raw[k]) * alpha);
           tmem_st32(o_col + 32 * c, raw);
         }
-      }
-      // pass 2, two halves of 64 keys: exponentiate, sum, and write P_t(j) as 16-bit pairs
-      // over the first 64 columns of S_t (the A operand of the PV MMA).  Half h reads S
-      // columns [64h, 64h + 64) and writes P columns [32h, 32h + 32), which hold S values
-      // already consumed.
-      float sum = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t raw[64];
-        uint32_t* r0 = raw;
-        uint32_t* r1 = raw + 32;
-        tmem_ld32(s_col + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(r0));
-        tmem_ld32(s_col + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(r1));
-        tmem_ld_wait();
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const int key = 64 * h + k;
-          float x0 = fmaf(__uint_as_float(raw[k]), c_log2, -m_used);
-          float x1 = fmaf(__uint_as_float(raw[k + 1]), c_log2, -m_used);
-          if (!full) {
-            x0 = key < valid ? x0 : -INFINITY;
-            x1 = key + 1 < valid ? x1 : -INFINITY;
-          }
-          float e0, e1;
-          if (key < POLY_FROM) {
-            e0 = ex2_approx(x0);
-            e1 = ex2_approx(x1);
-          } else {
-            e0 = exp2_poly(x0);
-            e1 = exp2_poly(x1);
-          }
-          sum += e0 + e1;
-          pk[k / 2] = pack2<F>(e0, e1);
-        }
-        tmem_st32(s_col + 32 * h, pk);
       }
       l = l * alpha + sum;
       tmem_st_wait();

@@ -206,6 +206,40 @@ def test_joint_attention(S, H, hd, batch, fmt):
         assert_close(got[b], ref, max_rel=2e-2, mean_rel=3e-3, what=f"attention S={S} H={H} hd={hd}")
 
 
+@pytest.mark.parametrize("fmt", [0, 1], ids=["bf16", "f16"])
+def test_joint_attention_running_max_rises(fmt):
+    """Rows whose running max rises by ~8.5 log2 units after many keys already carry weight.
+
+    Query row i looks along feature i % 4; along each feature a group of keys has logit 3
+    and four later keys logit 8.9 (natural units): inside key block 0 at chunk 1 (keys
+    32-35) and chunk 3 (keys 100-103), in block 2 (keys 300-303), and in the partial last
+    block (keys 580-583 of 600).  The earlier keys keep ~6-30 % of the mass, so a kernel
+    that skips rescaling O, the row sum or the P values of the block already written is
+    off by a factor of up to 2^8.5 (an emulation without either rescale errs by >3 in
+    max-rel).
+    """
+    S, H, hd = 600, 1, 128
+    r = np.random.default_rng(11)
+    q = 0.3 * r.standard_normal((S, hd))
+    k = 0.3 * r.standard_normal((S, hd))
+    v = r.standard_normal((S, hd))
+    q[:, :4] = 0.0
+    k[:, :4] = 0.0
+    q[np.arange(S), np.arange(S) % 4] = 8.0
+    groups = {0: (range(0, 32), range(32, 36)), 1: (range(0, 96), range(100, 104)),
+              2: (range(0, 128), range(300, 304)), 3: (range(0, 200), range(580, 584))}
+    for g, (base, late) in groups.items():
+        k[list(base), g] = 3.0 * np.sqrt(hd) / 8.0
+        k[list(late), g] = 8.9 * np.sqrt(hd) / 8.0
+    qkv = _fmt_tensor(np.concatenate([q, k, v], axis=1)[None].astype(np.float32), fmt)
+    out = _fmt_empty((1, S, hd), fmt)
+    ops.joint_attention(qkv, out, H, hd, fmt=fmt)
+    x = _fmt_values(qkv, fmt).reshape(S, 3, hd)
+    ref = oracle.attention(x[:, 0][:, None], x[:, 1][:, None], x[:, 2][:, None])[:, 0]
+    got = _fmt_values(out, fmt).reshape(S, hd)
+    assert_close(got, ref, max_rel=2e-2, mean_rel=3e-3, what="attention with rising maxima")
+
+
 def test_bounded_wait_timeout_is_not_hit_in_normal_runs():
     ops.set_wait_timeout_ms(2000)
     assert ops.poll_error() == 0
