@@ -10,6 +10,7 @@ One step = one pass of the whole hot path on the 1024 px workload:
 Metric: DiT block tokens/s (4608 tokens per step per GPU) and TFLOP/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --elementwise [--steps K]    # HBM-bound kernels alone, L2 flushed
 
 With N > 1 (under torchrun) every rank runs its own replica of the workload: the
 block does not shard at batch 1, so the ranks exchange nothing but the timing.
@@ -406,6 +407,95 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ HBM-bound kernels on their own
+
+
+def run_elementwise(args, local_rank):
+    """Achieved HBM bandwidth of the norm, QK-norm + M-RoPE and Euler kernels, each timed alone
+    with L2 flushed before every launch (a 256 MiB buffer is rewritten), on sweeps of several
+    hundred MB and at the sizes of the 1024 px step.  Bytes are algorithmic (each input read
+    once, each output written once); one JSON line."""
+    import torch
+
+    from joint_attention_block_b200 import ops
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+
+    def randn(shape, dtype):
+        return torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(dtype)
+
+    def timed(fn, tag, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        ops.profile_enable(8 * reps + 16)
+        for _ in range(reps):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize(dev)
+        ops.profile_disable()
+        rec = [ms for name, ms in ops.profile_read(8 * reps + 16) if name == tag]
+        if ops.poll_error() != 0:
+            raise RuntimeError(f"device-side error: {ops.last_device_error():#x}")
+        return statistics.median(rec)
+
+    pk, pk_kind = peaks()
+    hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out = {}
+
+    def report(name, ms, nbytes, note):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"us": round(ms * 1e3, 2), "bytes": int(nbytes), "gbs": round(gbs, 1),
+                     "frac": round(gbs / hbm, 3), "what": note}
+
+    s = synth.C1024
+    d = s.d_model
+    g = randn((53248,), torch.bfloat16) * 0.05 + 1.0
+    for rows, xfmt, label in ((65536, ops.FMT_BF16, "rmsnorm_bf16_to_f16"), (32768, ops.FMT_F32, "rmsnorm_f32_to_f16"),
+                              (s.seq, ops.FMT_BF16, "rmsnorm_bf16_to_f16_c1024"),
+                              (s.seq, ops.FMT_F32, "rmsnorm_f32_to_f16_c1024")):
+        x = randn((rows, d), torch.bfloat16 if xfmt == ops.FMT_BF16 else torch.float32)
+        y = torch.empty((rows, d), dtype=torch.float16, device=dev)
+        ms = timed(lambda: ops.rmsnorm_rows(x, g[:d], y, 1e-6, x_fmt=xfmt, y_fmt=ops.FMT_F16, stream=stream),
+                   "rmsnorm", args.steps)
+        report(label, ms, x.numel() * x.element_size() + y.numel() * 2, f"{rows} x {d} rows")
+        del x, y
+    for rows, label in ((4096, "cond_rmsnorm_53248"), (512, "cond_rmsnorm_53248_c1024")):
+        x = randn((rows, 53248), torch.bfloat16)
+        y = torch.empty((rows, 53248), dtype=torch.float16, device=dev)
+        ms = timed(lambda: ops.rmsnorm_rows(x, g, y, 1e-6, x_fmt=ops.FMT_BF16, y_fmt=ops.FMT_F16, stream=stream),
+                   "rmsnorm", args.steps)
+        report(label, ms, x.numel() * 2 + y.numel() * 2, f"{rows} x 53248 conditioning rows")
+        del x, y
+    cfg = ops.make_config(s)
+    gq = randn((s.head_dim,), torch.bfloat16) * 0.05 + 1.0
+    gk = randn((s.head_dim,), torch.bfloat16) * 0.05 + 1.0
+    ws = torch.empty(4 << 20, dtype=torch.uint8, device=dev)
+    for batch, label in ((4, "qknorm_mrope"), (1, "qknorm_mrope_c1024")):
+        qkv = randn((batch, s.seq, 3 * d), torch.float16)
+        ms = timed(lambda: ops.qknorm_mrope(qkv, cfg, s.n_text, s.grid_h, s.grid_w, gq, gk, ws, fmt=ops.FMT_F16,
+                                            stream=stream), "qknorm_mrope", args.steps)
+        report(label, ms, batch * s.seq * 2 * d * 2 * 2, f"q and k of {batch} x {s.seq} tokens, in place")
+        del qkv
+    for n, label in ((1 << 26, "euler_cfg"), (4096 * synth.LATENT_CHANNELS, "euler_cfg_c1024")):
+        lat = randn((n,), torch.float32)
+        vc = randn((n,), torch.bfloat16)
+        vu = randn((n,), torch.bfloat16)
+        ms = timed(lambda: ops.euler_cfg_step(lat, vc, vu, synth.CFG_GUIDANCE, synth.CFG_DT, stream=stream),
+                   "euler_cfg", args.steps)
+        report(label, ms, n * 12, f"{n} latent values")
+        del lat, vc, vu
+    print(json.dumps({"metric": "HBM-bound kernels alone: achieved GB/s, L2 flushed before each launch",
+                      "peak_gbs": hbm, "peak_kind": f"{pk_kind} HBM copy", "reps": args.steps,
+                      "kernels": out}), flush=True)
+
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -413,6 +503,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--elementwise", action="store_true",
+                    help="instead of the step: HBM bandwidth of the norm / QK-norm / Euler kernels alone")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -421,6 +513,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.elementwise:
+        if rank == 0:
+            run_elementwise(args, local_rank)
         return
     if world > 1:
         import datetime

@@ -185,8 +185,9 @@ DIT_API int dit_joint_attention(const void* qkv, void* out, int fmt, int batch, 
 DIT_API int dit_poll_error(void* stream);
 
 /* ---- launch instrumentation (off by default) ----
- * While enabled, each kernel launched by dit_block_forward, cond_proj_forward and
- * euler_cfg_step is bracketed by CUDA events on its stream, so the device time of
+ * While enabled, each kernel launched by dit_block_forward, cond_proj_forward,
+ * euler_cfg_step, dit_rmsnorm_rows and dit_qknorm_mrope is bracketed by CUDA events on
+ * its stream (the standalone GEMM and attention calls are not), so the device time of
  * every launch inside a timed region can be read back.  dit_profile_enable creates
  * max_marks events (host-side handles; the only resources this library creates) and
  * starts recording; dit_profile_read synchronises on the recorded events, writes up to

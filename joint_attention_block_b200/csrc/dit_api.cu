@@ -270,8 +270,11 @@ int dit_rmsnorm_rows(const void* x, int x_fmt, const void* g, void* y, int y_fmt
   if (rows > 0 && (x == nullptr || g == nullptr || y == nullptr)) return DIT_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(g) || !aligned16(y)) return DIT_ERR_INVALID_ARG;
   if (x == y && x_fmt != y_fmt) return DIT_ERR_INVALID_ARG;
-  return from_cuda(launch_rmsnorm(x, x_fmt, static_cast<const uint16_t*>(g), y, y_fmt, rows, cols, eps,
-                                  as_stream(stream)));
+  prof_mark(as_stream(stream), DIT_KERNEL_RMSNORM);
+  const cudaError_t e =
+      launch_rmsnorm(x, x_fmt, static_cast<const uint16_t*>(g), y, y_fmt, rows, cols, eps, as_stream(stream));
+  prof_mark(as_stream(stream), DIT_KERNEL_END);
+  return from_cuda(e);
 }
 
 int euler_cfg_step(float* x, const void* v_cond, const void* v_uncond, int64_t n, float guidance, float dt,
@@ -321,12 +324,15 @@ int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int 
   float* cos_tab = static_cast<float*>(workspace);
   float* sin_tab = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + need / 2);
   cudaStream_t s = as_stream(stream);
+  prof_mark(s, DIT_KERNEL_ROPE_TABLE);
   cudaError_t e = launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections,
                                     cfg->rope_theta, cos_tab, sin_tab, s);
   if (e != cudaSuccess) return DIT_ERR_CUDA;
-  return from_cuda(launch_qknorm_mrope(qkv, fmt, batch, S, cfg->n_heads, cfg->head_dim, cos_tab, sin_tab,
-                                       static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k), cfg->eps,
-                                       s));
+  prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
+  e = launch_qknorm_mrope(qkv, fmt, batch, S, cfg->n_heads, cfg->head_dim, cos_tab, sin_tab,
+                          static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k), cfg->eps, s);
+  prof_mark(s, DIT_KERNEL_END);
+  return from_cuda(e);
 }
 
 int dit_joint_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,

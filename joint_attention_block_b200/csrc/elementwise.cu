@@ -257,59 +257,82 @@ cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, con
 
 // ------------------------------------------------------------------ QK-RMSNorm + M-RoPE (standalone)
 
-// One thread per (batch, token, head, q|k, 8 rotary pairs): it holds elements
-// [8c, 8c+8) and [half+8c, half+8c+8) of the head as two 16-byte vectors, so the
-// hd/16 threads of one head row are consecutive lanes and reduce the sum of
-// squares with xor-shuffles.  F: storage format of the qkv buffer (bf16 or f16).
+// One thread per (batch, token, head, 8 rotary pairs): it holds elements [8c, 8c+8) and
+// [half+8c, half+8c+8) of the head in both q and k as 16-byte vectors (four loads in
+// flight, one cos/sin fetch for both), so the hd/16 threads of one head are consecutive
+// lanes and reduce the two sums of squares with xor-shuffles.  F: storage format of the
+// qkv buffer (bf16 or f16).
 template <int F>
 __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int seq, int n_heads, int head_dim,
                                     const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
                                     const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
   const int half = head_dim / 2;
-  const int group = half / 8;  // threads per head row: 8 (hd 128) or 4 (hd 64)
+  const int group = half / 8;  // threads per head: 8 (hd 128) or 4 (hd 64)
   const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(batch) * seq * n_heads * 2 * group;
+  const int64_t total = static_cast<int64_t>(batch) * seq * n_heads * group;
   const bool live = tid < total;
-  const int64_t t = live ? tid : total - 1;  // dead lanes shadow the last row so the shuffles stay full
+  const int64_t t = live ? tid : total - 1;  // dead lanes shadow the last head so the shuffles stay full
   const int c = static_cast<int>(t % group);
-  const int which = static_cast<int>((t / group) % 2);  // 0 = q, 1 = k
-  const int h = static_cast<int>((t / (2 * group)) % n_heads);
-  const int64_t bs = t / (2 * group * n_heads);
+  const int h = static_cast<int>((t / group) % n_heads);
+  const int64_t bs = t / (group * n_heads);
   const int s = static_cast<int>(bs % seq);
   const int d = n_heads * head_dim;
-  uint16_t* v = qkv + bs * (3 * static_cast<int64_t>(d)) + which * d + h * head_dim;
-  const uint16_t* g = which == 0 ? g_q : g_k;
-  float a[8], b[8], ga[8], gb[8];
-  load8<F>(v + 8 * c, 0, a);
-  load8<F>(v + half + 8 * c, 0, b);
-  load8<FMT_BF16>(g + 8 * c, 0, ga);
-  load8<FMT_BF16>(g + half + 8 * c, 0, gb);
-  float ss = 0.f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) ss = fmaf(a[k], a[k], fmaf(b[k], b[k], ss));
-  for (int o = group / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float rstd = rsqrtf(ss / static_cast<float>(head_dim) + eps);
+  uint16_t* vq = qkv + bs * (3 * static_cast<int64_t>(d)) + h * head_dim;
+  uint16_t* vk = vq + d;
+  float qa[8], qb[8], ka[8], kb[8];
+  load8<F>(vq + 8 * c, 0, qa);
+  load8<F>(vq + half + 8 * c, 0, qb);
+  load8<F>(vk + 8 * c, 0, ka);
+  load8<F>(vk + half + 8 * c, 0, kb);
   float cs[8], sn[8];
   load8<FMT_F32>(cos_tab + static_cast<int64_t>(s) * half + 8 * c, 0, cs);
   load8<FMT_F32>(sin_tab + static_cast<int64_t>(s) * half + 8 * c, 0, sn);
-  float oa[8], ob[8];
+  float sq = 0.f, sk = 0.f;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const float x1 = a[k] * rstd * ga[k];
-    const float x2 = b[k] * rstd * gb[k];
+    sq = fmaf(qa[k], qa[k], fmaf(qb[k], qb[k], sq));
+    sk = fmaf(ka[k], ka[k], fmaf(kb[k], kb[k], sk));
+  }
+  for (int o = group / 2; o > 0; o >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+  }
+  const float rq = rsqrtf(sq / static_cast<float>(head_dim) + eps);
+  const float rk = rsqrtf(sk / static_cast<float>(head_dim) + eps);
+  float ga[8], gb[8];
+  float oa[8], ob[8];
+  load8<FMT_BF16>(g_q + 8 * c, 0, ga);
+  load8<FMT_BF16>(g_q + half + 8 * c, 0, gb);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float x1 = qa[k] * rq * ga[k];
+    const float x2 = qb[k] * rq * gb[k];
     oa[k] = x1 * cs[k] - x2 * sn[k];
     ob[k] = x2 * cs[k] + x1 * sn[k];
   }
   if (live) {
-    store8<F>(v + 8 * c, 0, oa);
-    store8<F>(v + half + 8 * c, 0, ob);
+    store8<F>(vq + 8 * c, 0, oa);
+    store8<F>(vq + half + 8 * c, 0, ob);
+  }
+  load8<FMT_BF16>(g_k + 8 * c, 0, ga);
+  load8<FMT_BF16>(g_k + half + 8 * c, 0, gb);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float x1 = ka[k] * rk * ga[k];
+    const float x2 = kb[k] * rk * gb[k];
+    oa[k] = x1 * cs[k] - x2 * sn[k];
+    ob[k] = x2 * cs[k] + x1 * sn[k];
+  }
+  if (live) {
+    store8<F>(vk + 8 * c, 0, oa);
+    store8<F>(vk + half + 8 * c, 0, ob);
   }
 }
 
 cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
                                 const float* cos_tab, const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k,
                                 float eps, cudaStream_t s) {
-  const int64_t threads = static_cast<int64_t>(batch) * seq * n_heads * 2 * (head_dim / 16);
+  const int64_t threads = static_cast<int64_t>(batch) * seq * n_heads * (head_dim / 16);
   if (threads <= 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
   uint16_t* q = static_cast<uint16_t*>(qkv);
