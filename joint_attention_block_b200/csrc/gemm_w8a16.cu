@@ -24,17 +24,24 @@
 // barrier, and the leader's MMA commits arrive on both CTAs' barriers.  No TMA load
 // is multicast.
 //
-// Per CTA (grid.z = K splits):
+// The kernel is persistent: one pair of CTAs per pair of SMs walks the work units
+// (tile_m, tile_n, K split) pair_id, pair_id + pairs, ...  The rings run on across
+// units, so the producer loads the next unit's first stages while the current
+// unit's epilogue runs, and no CTA is relaunched per tile.
+//
+// Per CTA:
 //   warp 0      TMA producer: 128 x 64 activations (128B swizzle) and 2 x (128 x 64
 //               bytes) e4m3 weights (64B swizzle) per stage, 3-stage ring.
 //   warp 1      TMEM allocation (pair); in the leader, one lane issues 2 x 4 pair
 //               MMAs per stage.
 //   warps 2..9  converters: thread = one weight row; widen 64 e4m3 bytes to f16 (or
-//               bf16) and store them into the 2-stage widened ring.  Then the
-//               epilogue: thread = one token row of TMEM (warp w reads lanes
-//               32*(w%4).., accumulator (w-2)/4), scale, optional GELU; then, through
-//               shared memory, row-major: optional residual, 16-bit or fp32 stores
-//               that fill whole sectors.
+//               bf16) and store them into the 2-stage widened ring.  After a unit's
+//               last stage, the epilogue: thread = one token row of TMEM (warp w reads
+//               lanes 32*(w%4).., accumulator (w-2)/4), scale, optional GELU, optional
+//               residual (TMA-loaded boxes), 32 x 32 output boxes stored by TMA.  The
+//               boxes live in the widened ring (idle until these same warps convert
+//               the next unit) and a small extra region.  The next unit's MMAs wait
+//               for both CTAs' converters, hence for both epilogues to have read TMEM.
 #include <string.h>
 
 #include "common.cuh"
@@ -62,16 +69,19 @@ constexpr int MAX_PAIRS = 74;  // 148 SMs / 2
 constexpr int OFF_X = 0;
 constexpr int OFF_W8 = OFF_X + RAW_STAGES * X_BYTES;
 constexpr int OFF_W16 = OFF_W8 + RAW_STAGES * W8_BYTES;
-constexpr int OFF_SCALE = OFF_W16 + CVT_STAGES * W16_BYTES;
-constexpr int OFF_BAR = OFF_SCALE + BN * 4;
-constexpr int NUM_BARS = 3 * RAW_STAGES + 2 * CVT_STAGES + 2 + 2 * CVT_WARPS;
+// Epilogue boxes of 32 tokens x 32 channels, per epilogue warp two output boxes and two
+// residual boxes (2 KB each in 16-bit, 4 KB in fp32): at most 12 KB per warp (fp32 out
+// with an fp32 residual keeps one output box).  They start at the widened ring and run
+// 32 KB past it.
+constexpr int EPI_WARP_BYTES = 12 * 1024;
+constexpr int OFF_EPI = OFF_W16;
+constexpr int OFF_SCALE = OFF_EPI + CVT_WARPS * EPI_WARP_BYTES;  // per epilogue warp, 256 scales
+static_assert(OFF_SCALE >= OFF_W16 + CVT_STAGES * W16_BYTES, "epilogue region covers the widened ring");
+constexpr int OFF_BAR = OFF_SCALE + CVT_WARPS * BN_MMA * 4;
+constexpr int NUM_BARS = 3 * RAW_STAGES + 2 * CVT_STAGES + 3 + 2 * CVT_WARPS;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
-// Epilogue boxes: per epilogue warp two output boxes and two residual boxes of 32 tokens x 32
-// channels (up to fp32: 4 KB each), placed in the rings, which are free by then.
-constexpr int EPI_BOX = 4096;
-constexpr int EPI_WARP_BYTES = 4 * EPI_BOX;
-static_assert(CVT_WARPS * EPI_WARP_BYTES <= OFF_SCALE, "epilogue boxes must fit the free rings");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
 struct Params {
   const float* scale;
@@ -82,7 +92,8 @@ struct Params {
   int res_fmt;  // -1 none, FMT_BF16 / FMT_F16 / FMT_F32
   int act;      // 0 none, 1 GELU
   int gelu_tanh;
-  int kb_per_split;  // k-blocks per split (grid.z splits, fp32 partial outputs); all of K when not split
+  int kb_per_split;  // k-blocks per split (fp32 partial outputs per split); all of K when not split
+  int tiles_m, tiles_n, units;  // work units: tile_m fastest, then tile_n, then the K split
 };
 
 // GELU, exact form: x * Phi(x), Phi the standard normal CDF.  Phi(-|x|) = erfc(|x| / sqrt 2) / 2
@@ -119,16 +130,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint8_t* sX = smem + OFF_X;
   uint8_t* sW8 = smem + OFF_W8;
   uint8_t* sW16 = smem + OFF_W16;
-  float* sScale = reinterpret_cast<float*>(smem + OFF_SCALE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* x_full = bars;                      // leader: both CTAs' activation halves landed
   uint64_t* w8_full = x_full + RAW_STAGES;      // this CTA's e4m3 rows landed
   uint64_t* raw_empty = w8_full + RAW_STAGES;   // pair MMAs done with the activations + e4m3 rows read
   uint64_t* w16_full = raw_empty + RAW_STAGES;  // leader: both CTAs' widened rows written
   uint64_t* w16_empty = w16_full + CVT_STAGES;  // pair MMAs done with the widened rows
-  uint64_t* acc_full = w16_empty + CVT_STAGES;
+  uint64_t* acc_full = w16_empty + CVT_STAGES;  // one phase per unit
   uint64_t* drain_bar = acc_full + 1;
-  uint64_t* res_full = drain_bar + 1;  // per epilogue warp, two residual boxes
+  uint64_t* epi_done = drain_bar + 1;  // all epilogue warps of this CTA are done with a unit
+  uint64_t* res_full = epi_done + 1;   // per epilogue warp, two residual boxes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
 
@@ -136,14 +147,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int lane = static_cast<int>(lane_id());
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int tile_m = blockIdx.x >> 1;  // pair tile of 256 tokens
-  const int tile_n = blockIdx.y;       // pair tile of 512 channels
-  const int tok_cta = tile_m * BM + static_cast<int>(rank) * BM_CTA;  // this CTA's 128 tokens
+  const int pair = blockIdx.x >> 1;
+  const int pairs = gridDim.x >> 1;
   const int kb_total = (p.K + BK - 1) / BK;
-  const int kb0 = blockIdx.z * p.kb_per_split;
-  const int num_kb = min(kb_total - kb0, p.kb_per_split);
-  // weight rows this CTA widens: block b holds channels tile_n*512 + b*256 + rank*128 + [0, 128)
-  auto w_row0 = [&](int b) { return tile_n * BN + b * BN_MMA + static_cast<int>(rank) * 128; };
+  struct Unit {
+    int tile_m, tile_n, split, tok_cta, kb0, num_kb;
+  };
+  auto unit = [&](int u) {
+    Unit w;
+    w.tile_m = u % p.tiles_m;
+    w.tile_n = (u / p.tiles_m) % p.tiles_n;
+    w.split = u / (p.tiles_m * p.tiles_n);
+    w.tok_cta = w.tile_m * BM + static_cast<int>(rank) * BM_CTA;  // this CTA's 128 tokens
+    w.kb0 = w.split * p.kb_per_split;
+    w.num_kb = min(kb_total - w.kb0, p.kb_per_split);
+    return w;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < RAW_STAGES; ++s) {
@@ -157,6 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(epi_done, CVT_WARPS);
     for (int i = 0; i < 2 * CVT_WARPS; ++i) mbar_init(&res_full[i], 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -168,10 +188,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (p.res_fmt >= 0) tma_prefetch_desc(&tm_r);
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
-  for (int i = threadIdx.x; i < BN; i += THREADS) {
-    const int n = tile_n * BN + i;
-    sScale[i] = n < p.N ? p.scale[n] : 0.f;
-  }
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA
@@ -179,30 +195,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer
-    int issued = 0;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % RAW_STAGES;
-      const uint32_t it = static_cast<uint32_t>(kb / RAW_STAGES);
-      if (!mbar_wait(&raw_empty[s], (it & 1u) ^ 1u, guard, abort_flag,
-                     where_code(ERR_TIMEOUT_GEMM_PRODUCER, rank, kb)))
-        break;
-      if (lane == 0) {
-        const int k = (kb0 + kb) * BK;
-        mbar_arrive_expect_tx(&w8_full[s], W8_BYTES);
-        tma_load_2d(sW8 + s * W8_BYTES, &tm_w, &w8_full[s], k, w_row0(0));
-        tma_load_2d(sW8 + s * W8_BYTES + W8_BLOCK, &tm_w, &w8_full[s], k, w_row0(1));
-        if (leader) mbar_arrive_expect_tx(&x_full[s], 2 * X_BYTES);
-        tma_load_2d_pair(sX + s * X_BYTES, &tm_x, mapa_shared(smem_u32(&x_full[s]), 0), k, tok_cta);
+    // ---------------- TMA producer: runs ahead across units, bounded by the raw ring
+    int g = 0;  // stages issued so far (all units)
+    bool ok = true;
+    for (int u = pair; u < p.units && ok; u += pairs) {
+      const Unit w = unit(u);
+      for (int kb = 0; kb < w.num_kb; ++kb) {
+        const int s = g % RAW_STAGES;
+        const uint32_t it = static_cast<uint32_t>(g / RAW_STAGES);
+        if (!mbar_wait(&raw_empty[s], (it & 1u) ^ 1u, guard, abort_flag,
+                       where_code(ERR_TIMEOUT_GEMM_PRODUCER, rank, g))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const int k = (w.kb0 + kb) * BK;
+          const int wr = w.tile_n * BN + static_cast<int>(rank) * 128;  // block b adds b * 256
+          mbar_arrive_expect_tx(&w8_full[s], W8_BYTES);
+          tma_load_2d(sW8 + s * W8_BYTES, &tm_w, &w8_full[s], k, wr);
+          tma_load_2d(sW8 + s * W8_BYTES + W8_BLOCK, &tm_w, &w8_full[s], k, wr + BN_MMA);
+          if (leader) mbar_arrive_expect_tx(&x_full[s], 2 * X_BYTES);
+          tma_load_2d_pair(sX + s * X_BYTES, &tm_x, mapa_shared(smem_u32(&x_full[s]), 0), k, w.tok_cta);
+        }
+        __syncwarp();
+        ++g;
       }
-      __syncwarp();
-      issued = kb + 1;
     }
     // Never leave with copies in flight: every CTA drains its weight loads; the leader's
     // activation barrier counts both CTAs' activation loads, and the peer is held by the
     // final cluster barrier until the leader has drained.
-    for (int s = 0; s < RAW_STAGES && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / RAW_STAGES) * RAW_STAGES;
+    for (int s = 0; s < RAW_STAGES && s < g; ++s) {
+      const int last = s + ((g - 1 - s) / RAW_STAGES) * RAW_STAGES;
       const uint32_t par = static_cast<uint32_t>(last / RAW_STAGES) & 1u;
       mbar_wait(&w8_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, s), true);
       if (leader) mbar_wait(&x_full[s], par, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, s), true);
@@ -212,100 +235,135 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (leader) {
       constexpr uint32_t idesc = idesc_f16kind(BM, BN_MMA, F16, false, false);
       bool ok = true;
-      for (int kb = 0; kb < num_kb && ok; ++kb) {
-        const int s = kb % RAW_STAGES;
-        const int c = kb % CVT_STAGES;
-        ok = mbar_wait(&x_full[s], static_cast<uint32_t>(kb / RAW_STAGES) & 1u, guard, abort_flag,
-                       where_code(ERR_TIMEOUT_GEMM_MMA_X, rank, kb)) &&
-             mbar_wait(&w16_full[c], static_cast<uint32_t>(kb / CVT_STAGES) & 1u, guard, abort_flag,
-                       where_code(ERR_TIMEOUT_GEMM_MMA, rank, kb));
-        if (!ok) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t x0 = smem_u32(sX + s * X_BYTES);
-          const uint32_t w0 = smem_u32(sW16 + c * W16_BYTES);
+      int g = 0;
+      for (int u = pair; u < p.units && ok; u += pairs) {
+        const Unit w = unit(u);
+        for (int kb = 0; kb < w.num_kb; ++kb) {
+          const int s = g % RAW_STAGES;
+          const int c = g % CVT_STAGES;
+          // the first stage of a unit also waits, through the converters, for both epilogues
+          // of the previous unit to have read the accumulators
+          ok = mbar_wait(&x_full[s], static_cast<uint32_t>(g / RAW_STAGES) & 1u, guard, abort_flag,
+                         where_code(ERR_TIMEOUT_GEMM_MMA_X, rank, g)) &&
+               mbar_wait(&w16_full[c], static_cast<uint32_t>(g / CVT_STAGES) & 1u, guard, abort_flag,
+                         where_code(ERR_TIMEOUT_GEMM_MMA, rank, g));
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t x0 = smem_u32(sX + s * X_BYTES);
+            const uint32_t w0 = smem_u32(sW16 + c * W16_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(x0 + kk * 32, 16, 1024);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(x0 + kk * 32, 16, 1024);
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-              const uint64_t bd = smem_desc_sw128(w0 + b * W16_BLOCK + kk * 32, 16, 1024);
-              mma_f16kind_ss_pair(tmem + b * BN_MMA, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              for (int b = 0; b < 2; ++b) {
+                const uint64_t bd = smem_desc_sw128(w0 + b * W16_BLOCK + kk * 32, 16, 1024);
+                mma_f16kind_ss_pair(tmem + b * BN_MMA, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              }
             }
+            mma_commit_pair(&raw_empty[s], 0x3);
+            mma_commit_pair(&w16_empty[c], 0x3);
+            if (kb + 1 == w.num_kb) mma_commit_pair(acc_full, 0x3);  // this unit's accumulators
           }
-          mma_commit_pair(&raw_empty[s], 0x3);
-          mma_commit_pair(&w16_empty[c], 0x3);
+          __syncwarp();
+          ++g;
         }
-        __syncwarp();
       }
-      if (lane == 0) {
-        if (ok) mma_commit_pair(acc_full, 0x3);
-        mma_commit_pair(drain_bar, 0x3);  // all MMAs retired before either CTA frees TMEM
-      }
+      if (lane == 0) mma_commit_pair(drain_bar, 0x3);  // all MMAs retired before either CTA frees TMEM
       __syncwarp();
     }
     mbar_wait(drain_bar, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_DRAIN_MMA, rank, 0), true);
   } else {
-    // ---------------- converters (warps 2..9): thread = one of this CTA's 256 weight rows
-    const int ct = threadIdx.x - 64;  // 0..255
+    // ---------------- converters + epilogue (warps 2..9)
+    const int ct = threadIdx.x - 64;  // converter: one of this CTA's 256 weight rows
     const int b = ct >> 7;            // which MMA's B half
     const int r = ct & 127;           // row within the 128-row block
+    const int ew = warp - 2;          // epilogue: warp index
+    const int quarter = warp & 3;
+    const int acc = ew >> 2;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN_MMA;
+    float* sScale = reinterpret_cast<float*>(smem + OFF_SCALE) + ew * BN_MMA;
+    const int out_box = 32 * 32 * (p.y_fmt == FMT_F32 ? 4 : 2);
+    const int res_box = p.res_fmt < 0 ? 0 : 32 * 32 * (p.res_fmt == FMT_F32 ? 4 : 2);
+    // two output boxes, except fp32 out with an fp32 residual, which gets one so that the
+    // warp's boxes stay within EPI_WARP_BYTES
+    const int n_out = 2 * (out_box + res_box) <= EPI_WARP_BYTES ? 2 : 1;
+    uint8_t* ebox = smem + OFF_EPI + ew * EPI_WARP_BYTES;  // out boxes, then residual 0, residual 1
+    uint64_t* rbar = res_full + 2 * ew;
+    uint32_t rph = 0u;  // bit b: phase parity of residual box b
     bool ok = true;
-    for (int kb = 0; kb < num_kb && ok; ++kb) {
-      const int s = kb % RAW_STAGES;
-      const int c = kb % CVT_STAGES;
-      ok = mbar_wait(&w8_full[s], static_cast<uint32_t>(kb / RAW_STAGES) & 1u, guard, abort_flag,
-                     where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, kb)) &&
-           mbar_wait(&w16_empty[c], (static_cast<uint32_t>(kb / CVT_STAGES) & 1u) ^ 1u, guard, abort_flag,
-                     where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, kb));
-      if (!ok) break;
-      // e4m3 row: 64 bytes, 64-byte swizzle (16-byte chunk j sits at chunk j ^ ((r >> 1) & 3))
-      const uint8_t* src = sW8 + s * W8_BYTES + b * W8_BLOCK + r * BK;
-      // widened row: 128 bytes, 128-byte swizzle (chunk j sits at chunk j ^ (r & 7))
-      uint8_t* dst = sW16 + c * W16_BYTES + b * W16_BLOCK + r * 128;
+    int g = 0;
+    int ui = 0;
+    for (int u = pair; u < p.units && ok; u += pairs, ++ui) {
+      const Unit w = unit(u);
+      // the epilogue boxes overlap the widened ring: no warp converts for this unit until
+      // every warp has finished the previous unit's epilogue
+      if (ui > 0 && !mbar_wait(epi_done, static_cast<uint32_t>(ui - 1) & 1u, guard, abort_flag,
+                               where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, 0xFFFF))) {
+        ok = false;
+        break;
+      }
+      for (int kb = 0; kb < w.num_kb; ++kb) {
+        const int s = g % RAW_STAGES;
+        const int c = g % CVT_STAGES;
+        ok = mbar_wait(&w8_full[s], static_cast<uint32_t>(g / RAW_STAGES) & 1u, guard, abort_flag,
+                       where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, g)) &&
+             mbar_wait(&w16_empty[c], (static_cast<uint32_t>(g / CVT_STAGES) & 1u) ^ 1u, guard, abort_flag,
+                       where_code(ERR_TIMEOUT_GEMM_CONVERT, rank, g));
+        if (!ok) break;
+        // e4m3 row: 64 bytes, 64-byte swizzle (16-byte chunk j sits at chunk j ^ ((r >> 1) & 3))
+        const uint8_t* src = sW8 + s * W8_BYTES + b * W8_BLOCK + r * BK;
+        // widened row: 128 bytes, 128-byte swizzle (chunk j sits at chunk j ^ (r & 7))
+        uint8_t* dst = sW16 + c * W16_BYTES + b * W16_BLOCK + r * 128;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = *reinterpret_cast<const uint4*>(src + ((q ^ ((r >> 1) & 3)) << 4));
-        uint4 o0, o1;
-        e4m3x4_to_16x4<F16>(v.x, o0.x, o0.y);
-        e4m3x4_to_16x4<F16>(v.y, o0.z, o0.w);
-        e4m3x4_to_16x4<F16>(v.z, o1.x, o1.y);
-        e4m3x4_to_16x4<F16>(v.w, o1.z, o1.w);
-        *reinterpret_cast<uint4*>(dst + (((2 * q) ^ (r & 7)) << 4)) = o0;
-        *reinterpret_cast<uint4*>(dst + (((2 * q + 1) ^ (r & 7)) << 4)) = o1;
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + ((q ^ ((r >> 1) & 3)) << 4));
+          uint4 o0, o1;
+          e4m3x4_to_16x4<F16>(v.x, o0.x, o0.y);
+          e4m3x4_to_16x4<F16>(v.y, o0.z, o0.w);
+          e4m3x4_to_16x4<F16>(v.z, o1.x, o1.y);
+          e4m3x4_to_16x4<F16>(v.w, o1.z, o1.w);
+          *reinterpret_cast<uint4*>(dst + (((2 * q) ^ (r & 7)) << 4)) = o0;
+          *reinterpret_cast<uint4*>(dst + (((2 * q + 1) ^ (r & 7)) << 4)) = o1;
+        }
+        fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+        tc_fence_before();         // and the previous unit's TMEM reads ordered before its MMAs
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_remote(mapa_shared(smem_u32(&w16_full[c]), 0));
+          mbar_arrive(&raw_empty[s]);
+        }
+        ++g;
       }
-      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_remote(mapa_shared(smem_u32(&w16_full[c]), 0));
-        mbar_arrive(&raw_empty[s]);
-      }
-    }
+      if (!ok) break;
 
-    // ---------------- epilogue: TMEM lane = token, column = channel of accumulator `acc`.
-    // Per 32-channel chunk a warp reads its 32 tokens' accumulators, scales (and activates)
-    // them, adds the residual box that TMA brought into shared memory, writes the result row
-    // by row into a swizzled output box and hands the box to a TMA store.  Global traffic is
-    // all asynchronous: the residual boxes of the next two chunks and the stores of the last
-    // two are in flight while a chunk is computed.
-    if (ok && mbar_wait(acc_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_GEMM_EPILOGUE, rank, 0))) {
+      // ---------------- epilogue of unit u: TMEM lane = token, column = channel of `acc`.
+      // Per 32-channel chunk a warp reads its 32 tokens' accumulators, scales (and
+      // activates) them, adds the residual box that TMA brought into shared memory,
+      // writes the result row by row into a swizzled output box and hands the box to a
+      // TMA store.  The residual boxes of the next two chunks and the stores of the last
+      // two are in flight while a chunk is computed.
+      if (!mbar_wait(acc_full, static_cast<uint32_t>(ui) & 1u, guard, abort_flag,
+                     where_code(ERR_TIMEOUT_GEMM_EPILOGUE, rank, ui))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      const int ew = warp - 2;
-      const int quarter = warp & 3;
-      const int acc = ew >> 2;
-      const int tok_warp = tok_cta + quarter * 32;
-      const int ch_warp = tile_n * BN + acc * BN_MMA;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN_MMA;
-      uint8_t* ebox = smem + OFF_X + ew * EPI_WARP_BYTES;  // out box 0, out box 1, residual 0, residual 1
-      uint64_t* rbar = res_full + 2 * ew;
+      const int tok_warp = w.tok_cta + quarter * 32;
+      const int ch_warp = w.tile_n * BN + acc * BN_MMA;
       // valid chunks (N % 32 == 0); none when all 32 of the warp's tokens lie beyond M
       const int nch = tok_warp < p.M ? min(BN_MMA, p.N - ch_warp) / 32 : 0;
+      {  // this warp's 256 channel scales
+        const int n0 = ch_warp + 8 * lane;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) sScale[8 * lane + k] = n0 + k < p.N ? p.scale[n0 + k] : 0.f;
+      }
+      __syncwarp();
       const bool has_res = p.res_fmt >= 0;
-      const uint32_t res_box_bytes = p.res_fmt == FMT_F32 ? 4096u : 2048u;
       auto issue_res = [&](int c) {
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&rbar[c & 1], res_box_bytes);
-        tma_load_2d(ebox + (2 + (c & 1)) * EPI_BOX, &tm_r, &rbar[c & 1], ch_warp + 32 * c, tok_warp);
+        mbar_arrive_expect_tx(&rbar[c & 1], static_cast<uint32_t>(res_box));
+        tma_load_2d(ebox + n_out * out_box + (c & 1) * res_box, &tm_r, &rbar[c & 1], ch_warp + 32 * c, tok_warp);
       };
       int res_issued = 0;
       if (has_res && lane == 0) {
@@ -314,13 +372,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       res_issued = __shfl_sync(0xffffffffu, res_issued, 0);
       int c = 0;
       for (; c < nch; ++c) {
-        uint32_t r[32];
-        tmem_ld32(taddr + 32 * c, r);
+        uint32_t rr[32];
+        tmem_ld32(taddr + 32 * c, rr);
         tmem_ld_wait();
-        const int col = acc * BN_MMA + 32 * c;
         float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * sScale[col + j];
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[j]) * sScale[32 * c + j];
         if (p.act == 1) {
           if (p.gelu_tanh) {
 #pragma unroll
@@ -331,10 +388,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
         if (has_res) {
-          if (!mbar_wait(&rbar[c & 1], static_cast<uint32_t>(c >> 1) & 1u, guard, abort_flag,
-                         where_code(ERR_TIMEOUT_GEMM_EPILOGUE, rank, 1 + c)))
+          const int bx = c & 1;
+          if (!mbar_wait(&rbar[bx], (rph >> bx) & 1u, guard, abort_flag,
+                         where_code(ERR_TIMEOUT_GEMM_EPILOGUE, rank, 0x100 + c))) {
+            ok = false;
             break;
-          const uint8_t* rrow = ebox + (2 + (c & 1)) * EPI_BOX;
+          }
+          rph ^= 1u << bx;
+          const uint8_t* rrow = ebox + n_out * out_box + bx * res_box;
           if (p.res_fmt == FMT_F32) {  // 128-byte rows, 128-byte swizzle
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -345,19 +406,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const uint4 t = *reinterpret_cast<const uint4*>(rrow + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4));
-              const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+              const uint32_t wv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                v[8 * q + 2 * k] += p.res_fmt == FMT_F16 ? f16_lo(w[k]) : bf16_lo(w[k]);
-                v[8 * q + 2 * k + 1] += p.res_fmt == FMT_F16 ? f16_hi(w[k]) : bf16_hi(w[k]);
+                v[8 * q + 2 * k] += p.res_fmt == FMT_F16 ? f16_lo(wv[k]) : bf16_lo(wv[k]);
+                v[8 * q + 2 * k + 1] += p.res_fmt == FMT_F16 ? f16_hi(wv[k]) : bf16_hi(wv[k]);
               }
             }
           }
         }
-        // output box c & 1: the store issued two chunks ago must have read it
-        if (lane == 0) bulk_wait_group_read<1>();
+        // output box c % n_out: the store issued n_out chunks ago must have read it
+        if (lane == 0) {
+          if (n_out == 2) bulk_wait_group_read<1>();
+          else bulk_wait_group_read<0>();
+        }
         __syncwarp();
-        uint8_t* orow = ebox + (c & 1) * EPI_BOX;
+        uint8_t* orow = ebox + (c % n_out) * out_box;
         if (p.y_fmt == FMT_F32) {  // 128-byte rows, 128-byte swizzle
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -378,20 +442,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         fence_proxy_async_smem();  // generic writes -> visible to the TMA store
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tm_y, orow, ch_warp + 32 * c, tok_warp, blockIdx.z);  // rows >= M are clipped
+          tma_store_3d(&tm_y, orow, ch_warp + 32 * c, tok_warp, w.split);  // rows >= M are clipped
           bulk_commit_group();
           if (has_res && res_issued < nch) issue_res(res_issued);  // into the residual box just read
         }
         if (has_res && res_issued < nch) ++res_issued;
       }
-      // nothing in flight when the CTA moves on: residual loads not consumed, stores' reads
+      // Nothing in flight past the unit: residual loads not consumed (after a failed wait),
+      // and the stores' reads of the boxes, which the next unit's conversions overwrite.
       if (lane == 0) {
-        for (int k = c; k < res_issued; ++k)
-          mbar_wait(&rbar[k & 1], static_cast<uint32_t>(k >> 1) & 1u, guard, abort_flag,
-                    where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, 0x100 + k), true);
+        for (int k = c; k < res_issued; ++k) {
+          mbar_wait(&rbar[k & 1], (rph >> (k & 1)) & 1u, guard, abort_flag,
+                    where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, 0x200 + k), true);
+          rph ^= 1u << (k & 1);
+        }
         bulk_wait_group_read<0>();
       }
+      rph = __shfl_sync(0xffffffffu, rph, 0);
       __syncwarp();
+      if (!ok) break;
+      if (lane == 0) mbar_arrive(epi_done);
     }
   }
 
@@ -495,8 +565,15 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
     if (!make_tmap(&tm_r, tdt(a.res_fmt), 2, const_cast<void*>(a.residual), dims, strides, box, tswz(a.res_fmt)))
       return cudaErrorInvalidValue;
   }
-  Params p{a.scale, a.y, a.residual, a.M, a.N, a.K, a.y_fmt, a.residual ? a.res_fmt : -1, a.act, a.gelu_tanh, kb_per};
-  dim3 grid(2 * ((a.M + BM - 1) / BM), (a.N + BN - 1) / BN, splits);
+  const int tiles_m = (a.M + BM - 1) / BM, tiles_n = (a.N + BN - 1) / BN;
+  const int units = tiles_m * tiles_n * splits;
+  Params p{a.scale, a.y,  a.residual, a.M,   a.N,     a.K,     a.y_fmt, a.residual ? a.res_fmt : -1,
+           a.act,   a.gelu_tanh, kb_per, tiles_m, tiles_n, units};
+  int sms = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 2 * MAX_PAIRS;
+  const int pairs = min(units, max(1, sms / 2));
+  dim3 grid(2 * pairs, 1, 1);
   auto kern = f16 ? gemm_w8a16_kernel<true> : gemm_w8a16_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;

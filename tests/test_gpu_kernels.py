@@ -98,7 +98,8 @@ def _fmt_empty(shape, fmt: int) -> torch.Tensor:
     return torch.empty(*shape, dtype=(torch.int16, torch.float16, torch.float32)[fmt], device="cuda")
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 512, 256), (37, 768, 1024), (300, 288, 528)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 512, 256), (37, 768, 1024), (300, 288, 528),
+                                   (4500, 2080, 256)])
 @pytest.mark.parametrize("a_fmt,y_fmt,act,res_fmt", [
     (0, 0, 0, None), (0, 0, 1, None), (0, 0, 0, 0),  # bf16 in / out
     (1, 1, 0, None), (1, 2, 0, 0), (1, 1, 1, None), (1, 0, 0, 2),  # the block's four GEMMs
@@ -121,6 +122,20 @@ def test_gemm_w8a16(M, N, K, a_fmt, y_fmt, act, res_fmt):
     got = _fmt_values(y, y_fmt)
     # fp32 accumulation of exact products, one rounding to the output format
     assert_close(got, ref, max_rel=8e-3, mean_rel=2e-3, what=f"gemm {M}x{N}x{K}")
+
+
+def test_gemm_fp32_out_with_fp32_residual_many_units():
+    """fp32 output plus fp32 residual (one output box per epilogue warp) over more work
+    units than CTA pairs (each pair walks several 256 x 512 tiles, ragged in M and N)."""
+    M, N, K = 4500, 2080, 512
+    r = np.random.default_rng(29)
+    a_t = _fmt_tensor(r.standard_normal((M, K)).astype(np.float32), 1)
+    codes, scale = synth.quantize_rows_e4m3((r.standard_normal((N, K)) * 0.02).astype(np.float32))
+    res_t = _fmt_tensor(r.standard_normal((M, N)).astype(np.float32), 2)
+    y = _fmt_empty((M, N), 2)
+    ops.gemm_w8a16(a_t, dev(codes), dev(scale), y, residual=res_t, a_fmt=1, y_fmt=2, res_fmt=2)
+    ref = _fmt_values(a_t, 1) @ oracle.dequant(codes, scale).T + _fmt_values(res_t, 2)
+    assert_close(_fmt_values(y, 2), ref, max_rel=8e-3, mean_rel=2e-3, what="gemm f32 out + f32 residual")
 
 
 def test_gemm_dequant_is_exact_inside_the_mma():
