@@ -363,7 +363,8 @@ int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, c
   for (const void* p : ptrs)
     if (p == nullptr) return DIT_ERR_INVALID_ARG;
   if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(w->w_qkv) || !aligned16(w->w_o) || !aligned16(w->w_up) ||
-      !aligned16(w->w_down) || !aligned16(w->g_norm1) || !aligned16(w->g_norm2))
+      !aligned16(w->w_down) || !aligned16(w->g_norm1) || !aligned16(w->g_norm2) || !aligned16(w->g_q) ||
+      !aligned16(w->g_k))
     return DIT_ERR_INVALID_ARG;
   const int S = n_text + grid_h * grid_w;
   BlockWorkspace ws = carve_block(cfg, batch, S, nullptr);
