@@ -11,6 +11,7 @@ Metric: DiT block tokens/s (4608 tokens per step per GPU) and TFLOP/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --elementwise [--steps K]    # HBM-bound kernels alone, L2 flushed
+    python bench.py --denoise [--steps K]        # 34 + 34 blocks + Euler/CFG, CUDA graph
 
 With N > 1 (under torchrun) every rank runs its own replica of the workload: the
 block does not shard at batch 1, so the ranks exchange nothing but the timing.
@@ -496,6 +497,97 @@ def run_elementwise(args, local_rank):
 
 
 
+# ------------------------------------------------------------------ one denoising step of the whole DiT
+
+
+def run_denoise(args, local_rank):
+    """One flow-matching denoising step at 1024 px through the full depth of the DiT: the
+    conditional stack (34 blocks over 512 text + 4096 image tokens), the unconditional stack
+    (34 blocks over 32 text + 4096 image tokens, its own weights) and the Euler/CFG update,
+    captured once in a CUDA graph and replayed.  Four distinct weight sets (800 MB, far above
+    L2) are cycled through the 68 blocks; the velocities fed to the update are the synthetic
+    ones of the step benchmark (the projection from block output to latent velocity is not on
+    the path).  One JSON line."""
+    import dataclasses
+
+    import torch
+
+    from joint_attention_block_b200 import ops
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(dev)
+    n_blocks = 34
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    sc, su = synth.C1024, synth.UNCOND1024
+    sets = [synth.block_inputs(dataclasses.replace(sc, index=200 + i)) for i in range(4)]
+    x_c = to_dev(sets[0]["x"])
+    x_u = to_dev(synth.to_bf16_bits(synth.normal(su.index, 0, (1, su.seq, su.d_model))))
+    dev_sets = [{k: to_dev(v) for k, v in st.items() if k != "x"} for st in sets]
+    wts = [ops.make_weights(d) for d in dev_sets]
+    cond_w = [wts[i % 4] for i in range(n_blocks)]
+    uncond_w = [wts[(i + 2) % 4] for i in range(n_blocks)]
+    cfg_c, cfg_u = ops.make_config(sc), ops.make_config(su)
+    out_c, out_u = torch.empty_like(x_c), torch.empty_like(x_u)
+    ws_c = torch.empty(ops.stack_workspace_bytes(cfg_c, 1, sc.n_text, sc.grid_h, sc.grid_w), dtype=torch.uint8,
+                       device=dev)
+    ws_u = torch.empty(ops.stack_workspace_bytes(cfg_u, 1, su.n_text, su.grid_h, su.grid_w), dtype=torch.uint8,
+                       device=dev)
+    eul = synth.euler_inputs(4096 * synth.LATENT_CHANNELS)
+    lat, vc, vu = (to_dev(eul[k]) for k in ("x", "v_cond", "v_uncond"))
+    dt = float(np.float32(synth.CFG_DT))
+
+    def step():
+        ops.dit_stack_forward(cfg_c, cond_w, x_c, out_c, sc.n_text, sc.grid_h, sc.grid_w, ws_c, stream=stream)
+        ops.dit_stack_forward(cfg_u, uncond_w, x_u, out_u, su.n_text, su.grid_h, su.grid_w, ws_u, stream=stream)
+        ops.euler_cfg_step(lat, vc, vu, synth.CFG_GUIDANCE, dt, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 2)):
+            step()
+        stream.synchronize()
+        if ops.poll_error(stream) != 0:
+            raise RuntimeError(f"device-side error: {ops.last_device_error():#x}")
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        graph.replay()
+        stream.synchronize()
+        reps = max(3, min(args.steps, 20))
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        ev1.record(stream)
+        stream.synchronize()
+        ms_graph = ev0.elapsed_time(ev1) / reps
+        ev0.record(stream)
+        for _ in range(reps):
+            step()
+        ev1.record(stream)
+        stream.synchronize()
+        ms_eager = ev0.elapsed_time(ev1) / reps
+        if ops.poll_error(stream) != 0:
+            raise RuntimeError(f"device-side error: {ops.last_device_error():#x}")
+    del graph
+    flops = n_blocks * (sc.flops() + su.flops())
+    pk, pk_kind = peaks()
+    print(json.dumps({
+        "metric": "one 1024 px denoising step: 34 cond blocks (4608 tok) + 34 uncond blocks (4128 tok) + Euler/CFG",
+        "ms_graph": round(ms_graph, 3), "ms_eager": round(ms_eager, 3), "reps": reps,
+        "tflops": round(flops / (ms_graph / 1e3) / 1e12, 1), "flops_per_step": flops,
+        "frac_of_bf16_sustained": round(flops / (ms_graph / 1e3) / 1e12 / pk.get("bf16_tflops_sustained", 1.0), 4),
+        "peak_kind": f"{pk_kind} bf16 dense, sustained",
+        "launches_per_step": 2 * n_blocks * 9 + 1,
+        "data": "synthetic; 4 distinct weight sets cycled over the 68 blocks"}), flush=True)
+
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -505,6 +597,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--elementwise", action="store_true",
                     help="instead of the step: HBM bandwidth of the norm / QK-norm / Euler kernels alone")
+    ap.add_argument("--denoise", action="store_true",
+                    help="instead of the step: one denoising step through 34 + 34 blocks, CUDA-graph captured")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -517,6 +611,10 @@ def main():
     if args.elementwise:
         if rank == 0:
             run_elementwise(args, local_rank)
+        return
+    if args.denoise:
+        if rank == 0:
+            run_denoise(args, local_rank)
         return
     if world > 1:
         import datetime

@@ -101,6 +101,23 @@ DIT_API int dit_block_forward(const dit_block_config* cfg, const dit_block_weigh
                       int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                       void* workspace, size_t ws_bytes, void* stream);
 
+/* Bytes of device workspace dit_stack_forward needs: one block's workspace plus one
+ * activation buffer [batch, S, d_model] bf16 for the ping-pong between blocks. */
+DIT_API size_t dit_stack_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w);
+
+/* n_blocks DiT blocks back to back (the Ideogram 4 DiT stacks 34 of them: Ideogram 4.0
+ * announcement thread, "four key components"; deep dive section 4-2):
+ *   x_out = block[n-1]( ... block[1]( block[0](x_in) ) ... )
+ * w: HOST array of n_blocks weight sets (each as for dit_block_forward; read during the call).
+ * The intermediate activations alternate between x_out and a buffer in the workspace so that
+ * the last block writes x_out; the result equals n_blocks successive dit_block_forward calls
+ * bit for bit.  Other arguments as dit_block_forward; x_out must not alias x_in.
+ * workspace: >= dit_stack_workspace_bytes() bytes, 256-byte aligned.
+ * Errors: as dit_block_forward (INVALID_ARG also for n_blocks < 1 or a null w). */
+DIT_API int dit_stack_forward(const dit_block_config* cfg, const dit_block_weights* w, int n_blocks, const void* x_in,
+                              void* x_out, int batch, int n_text, int grid_h, int grid_w, int t_img,
+                              const int32_t* pos, void* workspace, size_t ws_bytes, void* stream);
+
 /* Size of the fixed device scratch behind dit_block_forward_noalloc (32 MiB).  Every GPU
  * that loads this library holds this much device memory until the process exits. */
 #define DIT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)

@@ -67,6 +67,9 @@ SIGNATURES = {
                                _P, _P, _SZ, _P]),
     "dit_block_forward_noalloc": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I,
                                        _I, _I, _I, _P, _P]),
+    "dit_stack_workspace_bytes": (_SZ, [ctypes.POINTER(BlockConfig), _I, _I, _I, _I]),
+    "dit_stack_forward": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _I, _P, _P, _I, _I, _I, _I,
+                               _I, _P, _P, _SZ, _P]),
     "cond_proj_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "cond_proj_forward": (_I, [_P, _I, _I, _I, _P, _F, _P, _P, _I, _P, _P, _SZ, _P]),
     "euler_cfg_step": (_I, [_P, _P, _P, _I64, _F, _F, _P]),
@@ -154,6 +157,20 @@ def dit_block_forward(cfg: BlockConfig, weights: BlockWeights, x: torch.Tensor, 
                       pos: Optional[torch.Tensor] = None, stream=None) -> None:
     _check("dit_block_forward", lib().dit_block_forward(
         ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
+        _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def stack_workspace_bytes(cfg: BlockConfig, batch: int, n_text: int, grid_h: int, grid_w: int) -> int:
+    return int(lib().dit_stack_workspace_bytes(ctypes.byref(cfg), batch, n_text, grid_h, grid_w))
+
+
+def dit_stack_forward(cfg: BlockConfig, weights, x: torch.Tensor, out: torch.Tensor, n_text: int, grid_h: int,
+                      grid_w: int, workspace: torch.Tensor, t_img: int = -1, pos: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+    """``weights``: sequence of BlockWeights, one per block, applied in order."""
+    arr = (BlockWeights * len(weights))(*weights)
+    _check("dit_stack_forward", lib().dit_stack_forward(
+        ctypes.byref(cfg), arr, len(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
         _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

@@ -413,6 +413,37 @@ int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, c
   return DIT_OK;
 }
 
+size_t dit_stack_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w) {
+  const size_t blk = dit_block_workspace_bytes(cfg, batch, n_text, grid_h, grid_w);
+  if (blk == 0) return 0;
+  const size_t S = static_cast<size_t>(n_text) + static_cast<size_t>(grid_h) * grid_w;
+  return blk + align256(static_cast<size_t>(batch) * S * cfg->d_model * 2);
+}
+
+int dit_stack_forward(const dit_block_config* cfg, const dit_block_weights* w, int n_blocks, const void* x_in,
+                      void* x_out, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
+                      void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_config(cfg);
+  if (st != DIT_OK) return st;
+  if (w == nullptr || n_blocks < 1 || x_in == nullptr || x_out == nullptr || x_in == x_out) return DIT_ERR_INVALID_ARG;
+  if (!shape_ok(batch, n_text, grid_h, grid_w)) return DIT_ERR_INVALID_ARG;
+  const size_t blk = dit_block_workspace_bytes(cfg, batch, n_text, grid_h, grid_w);
+  const size_t need = dit_stack_workspace_bytes(cfg, batch, n_text, grid_h, grid_w);
+  if (blk == 0 || need == 0) return DIT_ERR_UNSUPPORTED;
+  if (workspace == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return DIT_ERR_WORKSPACE;
+  void* buf = static_cast<uint8_t*>(workspace) + blk;  // [batch, S, d] bf16, ping-pong partner of x_out
+  const void* in = x_in;
+  for (int i = 0; i < n_blocks; ++i) {
+    // block i writes x_out when (n_blocks - 1 - i) is even, so the last block lands in x_out
+    void* out = ((n_blocks - 1 - i) & 1) == 0 ? x_out : buf;
+    st = dit_block_forward(cfg, &w[i], in, out, batch, n_text, grid_h, grid_w, t_img, pos, workspace, blk, stream);
+    if (st != DIT_OK) return st;
+    in = out;
+  }
+  return DIT_OK;
+}
+
 size_t cond_proj_workspace_bytes(int n_tok, int n_layers, int hidden, int d_out) {
   if (n_tok <= 0 || n_layers <= 0 || hidden <= 0 || d_out <= 0) return 0;
   const int64_t K = static_cast<int64_t>(n_layers) * hidden;

@@ -10,8 +10,10 @@ from .ideogram4 import (  # noqa: F401
     cond_proj_forward,
     dequant,
     dit_block_forward,
+    dit_stack_forward,
     e4m3_to_f64,
     euler_cfg_step,
+    f64_to_bf16_bits,
     gelu,
     inv_freq,
     mrope,

@@ -82,3 +82,25 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
     rc = lib.dit_block_forward_noalloc(ctypes.byref(cfg), ctypes.byref(w), None, None, 1, s.n_text, s.grid_h,
                                        s.grid_w, -1, None, None)
     assert rc == 2  # DIT_ERR_UNSUPPORTED
+
+
+def test_stack_workspace_and_validation_without_gpu(lib):
+    """The stack's workspace is one block's plus one [B, S, d] bf16 ping-pong buffer; bad calls
+    are rejected on the host."""
+    from joint_attention_block_b200 import synth
+    s = synth.C1024
+    cfg = _abi.make_config(s)
+    blk = lib.dit_block_workspace_bytes(ctypes.byref(cfg), 1, s.n_text, s.grid_h, s.grid_w)
+    assert lib.dit_stack_workspace_bytes(ctypes.byref(cfg), 1, s.n_text, s.grid_h, s.grid_w) == \
+        blk + s.seq * s.d_model * 2
+    w = (_abi.BlockWeights * 2)()
+    # no blocks, null weights, aliasing input and output: INVALID_ARG before any device work
+    assert lib.dit_stack_forward(ctypes.byref(cfg), w, 0, 16, 32, 1, s.n_text, s.grid_h, s.grid_w, -1, None,
+                                 None, 0, None) == 1
+    assert lib.dit_stack_forward(ctypes.byref(cfg), None, 2, 16, 32, 1, s.n_text, s.grid_h, s.grid_w, -1, None,
+                                 None, 0, None) == 1
+    assert lib.dit_stack_forward(ctypes.byref(cfg), w, 2, 16, 16, 1, s.n_text, s.grid_h, s.grid_w, -1, None,
+                                 None, 0, None) == 1
+    # no workspace
+    assert lib.dit_stack_forward(ctypes.byref(cfg), w, 2, 16, 32, 1, s.n_text, s.grid_h, s.grid_w, -1, None,
+                                 None, 0, None) == 3

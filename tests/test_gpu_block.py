@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from joint_attention_block_b200 import ops, synth
-from gpu_util import as_f64, assert_close, dev, empty_bf16, workspace
+from gpu_util import as_f64, assert_close, bits, dev, empty_bf16, workspace
 
 pytestmark = pytest.mark.gpu
 
@@ -113,3 +113,66 @@ def test_cond_proj(n_tok):
     rows = np.arange(n_tok) if n_tok <= 64 else np.sort(np.random.default_rng(4).choice(n_tok, 48, replace=False))
     ref = oracle.cond_proj_forward(inp["feats"][rows], inp["g"], c.eps, inp["w"], inp["scale"])
     assert_close(as_f64(out)[rows], ref, what=f"cond_proj {n_tok}")
+
+
+def _stack_inputs(shape, n_blocks):
+    """n_blocks weight sets with their own seed streams; x from the first."""
+    sets = [synth.block_inputs(dataclasses.replace(shape, index=100 + i)) for i in range(n_blocks)]
+    return sets[0]["x"], [{k: v for k, v in inp.items() if k != "x"} for inp in sets]
+
+
+def _run_stack(shape, x_bits, wsets):
+    cfg = ops.make_config(shape)
+    dev_sets = [{k: dev(v) for k, v in w.items()} for w in wsets]  # kept alive for the call
+    weights = [ops.make_weights(d) for d in dev_sets]
+    x = dev(x_bits)
+    out = torch.empty_like(x)
+    ws = workspace(ops.stack_workspace_bytes(cfg, x.shape[0], shape.n_text, shape.grid_h, shape.grid_w))
+    ops.dit_stack_forward(cfg, weights, x, out, shape.n_text, shape.grid_h, shape.grid_w, ws)
+    torch.cuda.synchronize()
+    return out, dev_sets
+
+
+def test_stack_equals_successive_block_calls_bitwise():
+    """Five distinct blocks through dit_stack_forward equal five dit_block_forward calls, bit for bit
+    (odd count: the ping-pong ends in x_out)."""
+    s = synth.TINY
+    x_bits, wsets = _stack_inputs(s, 5)
+    got, dev_sets = _run_stack(s, x_bits, wsets)
+    cfg = ops.make_config(s)
+    cur = dev(x_bits)
+    ws = workspace(ops.block_workspace_bytes(cfg, 1, s.n_text, s.grid_h, s.grid_w))
+    for d in dev_sets:
+        nxt = torch.empty_like(cur)
+        ops.dit_block_forward(cfg, ops.make_weights(d), cur, nxt, s.n_text, s.grid_h, s.grid_w, ws)
+        cur = nxt
+    torch.cuda.synchronize()
+    assert torch.equal(got, cur)
+
+
+def test_stack_of_34_tiny_blocks_against_oracle():
+    """The DiT's depth (34 blocks) on the tiny shape with 34 distinct weight sets.
+
+    Per block: each GPU block's output against the oracle block fed the same bf16 input (the
+    GPU's previous output), within the single-block tolerances.  End to end: the stack against
+    the oracle's own stack (bf16 between blocks, as the API defines a block's input and output);
+    independent per-block errors add in quadrature, so the budget there is sqrt(34) times the
+    single-block one (measured: max-rel 1.4e-2, mean-rel 5.9e-3)."""
+    s = synth.TINY
+    n = 34
+    x_bits, wsets = _stack_inputs(s, n)
+    got, dev_sets = _run_stack(s, x_bits, wsets)
+    cfg = ops.make_config(s)
+    ws = workspace(ops.block_workspace_bytes(cfg, 1, s.n_text, s.grid_h, s.grid_w))
+    cur = dev(x_bits)
+    for i, d in enumerate(dev_sets):
+        nxt = torch.empty_like(cur)
+        ops.dit_block_forward(cfg, ops.make_weights(d), cur, nxt, s.n_text, s.grid_h, s.grid_w, ws)
+        torch.cuda.synchronize()
+        ref_i = oracle.dit_block_forward(s, wsets[i], bits(cur), s.n_text, s.grid_h, s.grid_w)
+        assert_close(as_f64(nxt), ref_i, what=f"block {i} of the stack")
+        cur = nxt
+    assert torch.equal(got, cur)
+    ref = oracle.dit_stack_forward(s, wsets, x_bits, s.n_text, s.grid_h, s.grid_w)
+    k = float(np.sqrt(n))
+    assert_close(as_f64(got), ref, max_rel=2e-2 * k, mean_rel=3e-3 * k, what="34-block stack")

@@ -406,3 +406,37 @@ def test_block_flop_count():
     assert s.seq == 4608
     assert abs(s.flops() - 2.203e12) / 2.203e12 < 1e-3
     assert abs(synth.UNCOND1024.flops() - 1.941e12) / 1.941e12 < 1e-3
+
+
+# ---------------------------------------------------------------- stacks of blocks
+
+
+def test_bf16_rounding_matches_torch():
+    """The oracle's fp64 -> bf16 rounding against torch's own bf16 cast (a library routine),
+    on random values, exact ties, huge and tiny magnitudes."""
+    r = np.random.default_rng(21)
+    x = np.concatenate([r.standard_normal(4096) * 10.0 ** r.integers(-30, 30, 4096),
+                        np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -1.0 - 2.0 ** -8, 3.0e38, -3.0e38, 0.0, -0.0,
+                                  1e-40, 2.0 ** -133])])
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.f64_to_bf16_bits(x), want)
+
+
+def test_stack_of_blocks_with_zero_outputs_is_identity():
+    """Blocks whose output projections are zero pass x through exactly, so a stack of them
+    returns x; a single-block stack is the block itself."""
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg)
+    r = np.random.default_rng(22)
+    x_bits = synth.to_bf16_bits(r.standard_normal((1, 6, cfg.d_model)))
+    z = dict(w)
+    z["w_o"] = np.zeros_like(w["w_o"])
+    z["w_down"] = np.zeros_like(w["w_down"])
+    assert np.array_equal(oracle.dit_stack_forward(cfg, [z, z, z], x_bits, 2, 2, 2), oracle.bf16_to_f64(x_bits))
+    assert np.array_equal(oracle.dit_stack_forward(cfg, [w], x_bits, 2, 2, 2),
+                          oracle.dit_block_forward(cfg, w, x_bits, 2, 2, 2))
+    # a zero block after a real one returns the real block's output rounded to bf16
+    two = oracle.dit_stack_forward(cfg, [w, z], x_bits, 2, 2, 2)
+    one = oracle.dit_block_forward(cfg, w, x_bits, 2, 2, 2)
+    assert np.array_equal(two, oracle.bf16_to_f64(oracle.f64_to_bf16_bits(one)))
+    assert not np.array_equal(two, one)
