@@ -115,6 +115,32 @@ def test_cond_proj(n_tok):
     assert_close(as_f64(out)[rows], ref, what=f"cond_proj {n_tok}")
 
 
+@pytest.mark.slow
+def test_block_d4608_variant():
+    """The 4608-wide model the quickstart's "~4.5 MiB per 512 projected tokens" implies (36 heads
+    x 128, MLP 18,432): a 16 + 6x6 token block, every row against the oracle."""
+    s = dataclasses.replace(synth.C1024, name="d4608", index=7, n_text=16, grid_h=6, grid_w=6, d_model=4608,
+                            n_heads=36, d_mlp=18432)
+    inp = synth.block_inputs(s)
+    got = run_block(s, inp)
+    ref = oracle.dit_block_forward(s, inp, inp["x"], s.n_text, s.grid_h, s.grid_w)
+    assert_close(got, ref, what="d4608 block")
+
+
+def test_cond_proj_to_4608():
+    """llm_cond_proj onto a 4608-wide model: 512 x 4608 bf16 = 4.5 MiB, the quickstart's figure."""
+    c = dataclasses.replace(synth.COND, index=8, d_out=4608)
+    n_tok = 24
+    inp = synth.cond_inputs(c, n_tok=n_tok)
+    out = empty_bf16(n_tok, c.d_out)
+    ws = workspace(ops.cond_proj_workspace_bytes(n_tok, c.n_layers, c.hidden, c.d_out))
+    ops.cond_proj_forward(dev(inp["feats"]), c.n_layers, c.hidden, dev(inp["g"]), c.eps, dev(inp["w"]),
+                          dev(inp["scale"]), out, ws)
+    ref = oracle.cond_proj_forward(inp["feats"], inp["g"], c.eps, inp["w"], inp["scale"])
+    assert_close(as_f64(out), ref, what="cond_proj to 4608")
+    assert 512 * c.d_out * 2 == 4.5 * 2 ** 20
+
+
 def _stack_inputs(shape, n_blocks):
     """n_blocks weight sets with their own seed streams; x from the first."""
     sets = [synth.block_inputs(dataclasses.replace(shape, index=100 + i)) for i in range(n_blocks)]
