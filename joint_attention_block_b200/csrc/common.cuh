@@ -351,6 +351,22 @@ JAB_DEVICE void tma_store_3d(const CUtensorMap* m, const void* src, int32_t x, i
                "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
+// The same store with an L2 cache-policy hint (see l2_evict_first_policy).
+JAB_DEVICE void tma_store_3d_hint(const CUtensorMap* m, const void* src, int32_t x, int32_t y, int32_t z,
+                                  uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+// L2 policy marking lines as the first to evict: for output streams larger than L2 that
+// would otherwise push out operands the same kernel still re-reads.
+JAB_DEVICE uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
 JAB_DEVICE void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N of this thread's committed bulk groups still read shared memory.
 template <int N>

@@ -94,6 +94,7 @@ struct Params {
   int gelu_tanh;
   int kb_per_split;  // k-blocks per split (fp32 partial outputs per split); all of K when not split
   int tiles_m, tiles_n, units;  // work units: tile_m fastest, then tile_n, then the K split
+  int y_evict_first;            // output stream larger than L2: store it with an evict-first hint
 };
 
 // GELU, exact form: x * Phi(x), Phi the standard normal CDF.  Phi(-|x|) = erfc(|x| / sqrt 2) / 2
@@ -442,7 +443,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         fence_proxy_async_smem();  // generic writes -> visible to the TMA store
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tm_y, orow, ch_warp + 32 * c, tok_warp, w.split);  // rows >= M are clipped
+          if (p.y_evict_first)  // keep the re-read activation tiles in L2, not the output
+            tma_store_3d_hint(&tm_y, orow, ch_warp + 32 * c, tok_warp, w.split, l2_evict_first_policy());
+          else
+            tma_store_3d(&tm_y, orow, ch_warp + 32 * c, tok_warp, w.split);  // rows >= M are clipped
           bulk_commit_group();
           if (has_res && res_issued < nch) issue_res(res_issued);  // into the residual box just read
         }
@@ -567,8 +571,11 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
   }
   const int tiles_m = (a.M + BM - 1) / BM, tiles_n = (a.N + BN - 1) / BN;
   const int units = tiles_m * tiles_n * splits;
+  // outputs of more than ~100 MB (the QKV and MLP-up projections at 1024 px) cannot stay in the
+  // 126 MB L2 anyway; smaller ones (O's fp32 residual stream) are read back from L2 by the next kernel
+  const int64_t y_bytes = static_cast<int64_t>(a.M) * a.N * (a.y_fmt == FMT_F32 ? 4 : 2) * splits;
   Params p{a.scale, a.y,  a.residual, a.M,   a.N,     a.K,     a.y_fmt, a.residual ? a.res_fmt : -1,
-           a.act,   a.gelu_tanh, kb_per, tiles_m, tiles_n, units};
+           a.act,   a.gelu_tanh, kb_per, tiles_m, tiles_n, units, y_bytes > (100ll << 20) ? 1 : 0};
   int sms = 0, dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     sms = 2 * MAX_PAIRS;
