@@ -281,11 +281,10 @@ def run_ours(args, rank, world, local_rank):
     if ops.poll_error() != 0:
         raise RuntimeError(f"device-side error during warm-up: {ops.last_device_error():#x}")
 
-    # ---- timed region: device-resident inputs; per-launch events inside the library
+    # ---- timed region: device-resident inputs, nothing but the step's own launches on the stream
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(1.0)
-    ops.profile_enable(args.steps * 24 + 64)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
@@ -297,12 +296,23 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     w1 = time.time()
     barrier()
-    ops.profile_disable()
     clocks.stop()
     ms = max_over_ranks(ev0.elapsed_time(ev1))
-    records = ops.profile_read(args.steps * 24 + 64)
     if ops.poll_error() != 0:
         raise RuntimeError(f"device-side error in the timed region: {ops.last_device_error():#x}")
+
+    # ---- per-kernel device times: the same steps again with the library's launch events, which
+    # sit between the kernels and so also stop each kernel from starting during its predecessor's
+    # tail (the un-instrumented run above lets them)
+    prof_steps = max(3, min(args.steps, 20))
+    ops.profile_enable(prof_steps * 24 + 64)
+    for _ in range(prof_steps):
+        step()
+    torch.cuda.synchronize(dev)
+    ops.profile_disable()
+    records = ops.profile_read(prof_steps * 24 + 64)
+    if ops.poll_error() != 0:
+        raise RuntimeError(f"device-side error in the profiled steps: {ops.last_device_error():#x}")
 
     # ---- end to end through the public calls: pinned host inputs in, results out, every step
     h_feats = torch.from_numpy(cond["feats"].view(np.int16)).pin_memory()
@@ -398,7 +408,8 @@ def run_ours(args, rank, world, local_rank):
                      "all_gemms_tflops": round(gemm_all, 1) if gemm_all else None,
                      "all_gemms_frac": round(gemm_all / peak_tc, 4) if gemm_all else None},
         "kernels": kernels,
-        "gpu_launches": len(records),
+        "kernels_from": f"{prof_steps} instrumented steps after the timed ones",
+        "gpu_launches": len(records) // prof_steps * args.steps,
         "clocks": clk,
         "e2e": {"value": round(s.seq * e2e_steps * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait_then_release();  // the setup above overlaps the previous kernel's tail
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -378,7 +379,9 @@ cudaError_t launch_hd(const CUtensorMap& tm, void* out, int batch, int seq, int 
       cudaFuncSetAttribute(attention_kernel<HD, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((seq + 2 * BQ - 1) / (2 * BQ), n_heads, batch);
-  attention_kernel<HD, F><<<grid, THREADS, L::SMEM, s>>>(tm, static_cast<uint16_t*>(out), seq, n_heads, g);
+  e = launch_pdl(attention_kernel<HD, F>, grid, dim3(THREADS), L::SMEM, s, tm, static_cast<uint16_t*>(out), seq,
+                 n_heads, g);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -21,6 +21,13 @@ namespace jab {
 
 // ------------------------------------------------------------------ misc
 
+// Programmatic dependent launch (see launch_pdl): wait for the previous kernel on the stream,
+// then let the next one launch.
+JAB_DEVICE void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 JAB_DEVICE uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -65,6 +65,7 @@ __device__ float block_sum(float v, float* red) {
 template <int kThreads, int kVec, int XF, int YF>
 __global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const void* x, const uint16_t* __restrict__ g, void* y,
                                                            int64_t cols, float eps) {
+  pdl_wait_then_release();
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const int64_t nv = cols / 8;
@@ -119,13 +120,13 @@ static void rmsnorm_dispatch(const void* x, const uint16_t* g, void* y, int64_t 
                              cudaStream_t s) {
   const unsigned r = static_cast<unsigned>(rows);
   if (cols <= 256 * 8 * 1) {
-    rmsnorm_kernel<256, 1, XF, YF><<<r, 256, 0, s>>>(x, g, y, cols, eps);
+    launch_pdl(rmsnorm_kernel<256, 1, XF, YF>, dim3(r), dim3(256), 0, s, x, g, y, cols, eps);
   } else if (cols <= 256 * 8 * 2) {
-    rmsnorm_kernel<256, 2, XF, YF><<<r, 256, 0, s>>>(x, g, y, cols, eps);
+    launch_pdl(rmsnorm_kernel<256, 2, XF, YF>, dim3(r), dim3(256), 0, s, x, g, y, cols, eps);
   } else if (cols <= 256 * 8 * 4) {
-    rmsnorm_kernel<256, 4, XF, YF><<<r, 256, 0, s>>>(x, g, y, cols, eps);
+    launch_pdl(rmsnorm_kernel<256, 4, XF, YF>, dim3(r), dim3(256), 0, s, x, g, y, cols, eps);
   } else {
-    rmsnorm_kernel<512, 0, XF, YF><<<r, 512, 0, s>>>(x, g, y, cols, eps);
+    launch_pdl(rmsnorm_kernel<512, 0, XF, YF>, dim3(r), dim3(512), 0, s, x, g, y, cols, eps);
   }
 }
 
@@ -145,6 +146,7 @@ cudaError_t launch_rmsnorm(const void* x, int x_fmt, const uint16_t* g, void* y,
 // x <- x + dt * (v_u + g * (v_c - v_u)); 8 elements per thread per iteration.
 __global__ void euler_cfg_kernel(float* __restrict__ x, const uint16_t* __restrict__ vc,
                                  const uint16_t* __restrict__ vu, int64_t n, float guidance, float dt) {
+  pdl_wait_then_release();
   const int64_t nvec = n / 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec; i += stride) {
@@ -182,7 +184,7 @@ cudaError_t launch_euler_cfg(float* x, const uint16_t* vc, const uint16_t* vu, i
   int64_t blocks = (nvec + 255) / 256;
   if (blocks < 1) blocks = 1;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  euler_cfg_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, vc, vu, n, g, dt);
+  launch_pdl(euler_cfg_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, vc, vu, n, g, dt);
   return cudaGetLastError();
 }
 
@@ -228,6 +230,7 @@ cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int3
 // fp64 and rounded once to fp32.
 __global__ void rope_table_kernel(int S, int n_text, int grid_w, int t_img, const int32_t* pos, int half,
                                   int sec_t, int sec_h, double theta, float* cos_tab, float* sin_tab) {
+  pdl_wait_then_release();
   const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (idx >= static_cast<int64_t>(S) * half) return;
   const int s = static_cast<int>(idx / half);
@@ -250,8 +253,8 @@ cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, con
   const int64_t n = static_cast<int64_t>(S) * half;
   if (n <= 0) return cudaSuccess;
   if (t_img < 0) t_img = n_text;
-  rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
-      S, n_text, grid_w, t_img, pos, half, sections[0], sections[1], static_cast<double>(theta), cos_tab, sin_tab);
+  launch_pdl(rope_table_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, S, n_text, grid_w, t_img,
+             pos, half, sections[0], sections[1], static_cast<double>(theta), cos_tab, sin_tab);
   return cudaGetLastError();
 }
 
@@ -266,6 +269,7 @@ template <int F>
 __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int seq, int n_heads, int head_dim,
                                     const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
                                     const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
+  pdl_wait_then_release();
   const int half = head_dim / 2;
   const int group = half / 8;  // threads per head: 8 (hd 128) or 4 (hd 64)
   const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
@@ -337,11 +341,11 @@ cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_he
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
   uint16_t* q = static_cast<uint16_t*>(qkv);
   if (fmt == FMT_F16)
-    qknorm_mrope_kernel<FMT_F16><<<blocks, 256, 0, s>>>(q, batch, seq, n_heads, head_dim, cos_tab, sin_tab, g_q, g_k,
-                                                        eps);
+    launch_pdl(qknorm_mrope_kernel<FMT_F16>, dim3(blocks), dim3(256), 0, s, q, batch, seq, n_heads, head_dim, cos_tab,
+               sin_tab, g_q, g_k, eps);
   else if (fmt == FMT_BF16)
-    qknorm_mrope_kernel<FMT_BF16><<<blocks, 256, 0, s>>>(q, batch, seq, n_heads, head_dim, cos_tab, sin_tab, g_q, g_k,
-                                                         eps);
+    launch_pdl(qknorm_mrope_kernel<FMT_BF16>, dim3(blocks), dim3(256), 0, s, q, batch, seq, n_heads, head_dim, cos_tab,
+               sin_tab, g_q, g_k, eps);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

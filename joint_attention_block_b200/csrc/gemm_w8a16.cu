@@ -194,6 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait_then_release();  // the setup above overlaps the previous kernel's tail
 
   if (warp == 0) {
     // ---------------- TMA producer: runs ahead across units, bounded by the raw ring
@@ -481,6 +482,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 // out[i] = sum over splits of part[z][i], as bf16; 8 elements per thread.
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, uint16_t* __restrict__ out, int64_t n,
                                      int splits) {
+  pdl_wait_then_release();
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (i >= n / 8) return;
   float v[8];
@@ -516,7 +518,8 @@ int gemm_pick_splits(int M, int N, int K) {
 
 cudaError_t launch_splitk_reduce(const float* part, uint16_t* out, int64_t n, int splits, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  gemm::splitk_reduce_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s>>>(part, out, n, splits);
+  launch_pdl(gemm::splitk_reduce_kernel, dim3(static_cast<unsigned>((n / 8 + 255) / 256)), dim3(256), 0, s, part, out, n,
+             splits);
   return cudaGetLastError();
 }
 
@@ -584,7 +587,8 @@ cudaError_t launch_gemm_w8a16(const GemmArgs& a, const KernelGuard& g, cudaStrea
   auto kern = f16 ? gemm_w8a16_kernel<true> : gemm_w8a16_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, THREADS, SMEM_BYTES, s>>>(tm_x, tm_w, tm_y, tm_r, p, g);
+  e = launch_pdl(kern, grid, dim3(THREADS), SMEM_BYTES, s, tm_x, tm_w, tm_y, tm_r, p, g);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

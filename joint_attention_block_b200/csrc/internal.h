@@ -8,6 +8,27 @@
 
 namespace jab {
 
+// Launch with programmatic stream serialisation: the kernel may start while the previous
+// kernel on the stream is finishing.  Every kernel launched this way executes
+// griddepcontrol.wait (pdl_wait) before its first global-memory access, which returns once
+// the previous kernel has completed and its writes are visible, and then
+// griddepcontrol.launch_dependents, so the next kernel's CTAs can take the SMs its own tail
+// leaves idle.  Outside such a chain the two instructions do nothing.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Passed by value to every kernel that waits: where to record errors and how long to wait.
 struct KernelGuard {
   uint32_t* err;        // device error word of the current device
