@@ -133,12 +133,17 @@ def mrope(x: np.ndarray, pos: np.ndarray, sections: Sequence[int], theta: float)
     return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
 
 
-def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
-    """Bidirectional softmax attention per head; q [Sq, H, hd], k/v [S, H, hd] -> [Sq, H, hd]."""
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, key_valid: Optional[np.ndarray] = None) -> np.ndarray:
+    """Bidirectional softmax attention per head; q [Sq, H, hd], k/v [S, H, hd] -> [Sq, H, hd].
+
+    ``key_valid`` (bool [S]), when given, removes the other keys (padding) from every row's
+    softmax: their logits are -inf, so they get weight exactly 0."""
     hd = q.shape[-1]
     out = np.empty((q.shape[0], q.shape[1], v.shape[-1]), dtype=np.float64)
     for h in range(q.shape[1]):
         s = q[:, h, :] @ k[:, h, :].T / math.sqrt(hd)
+        if key_valid is not None:
+            s = np.where(np.asarray(key_valid, dtype=bool)[None, :], s, -np.inf)
         s = s - s.max(axis=1, keepdims=True)
         p = np.exp(s)
         p /= p.sum(axis=1, keepdims=True)
@@ -159,6 +164,7 @@ def dit_block_forward(
     t_img: Optional[int] = None,
     rows: Optional[np.ndarray] = None,
     pos: Optional[np.ndarray] = None,
+    text_lens: Optional[Sequence[int]] = None,
 ) -> np.ndarray:
     """One single-stream DiT block forward, fp64, for x [B, S, d] (bf16 bits) -> [B, S, d].
 
@@ -167,6 +173,12 @@ def dit_block_forward(
     w_down [d, F], fp32 scales s_qkv, s_o, s_up, s_down and bf16 gains g_norm1,
     g_norm2 [d], g_q, g_k [hd].  With ``rows`` given only those query rows are
     computed (K and V still cover every token) and the result is [B, len(rows), d].
+
+    ``text_lens`` (one per batch element, each <= n_text) makes a padded batch of prompts of
+    different lengths: element b's text occupies rows [0, text_lens[b]) and rows
+    [text_lens[b], n_text) are padding.  Each element is positioned as if unpadded (text j at
+    (j, j, j), image cell (r, c) at (text_lens[b], r, c) unless t_img is given), padding rows
+    are excluded as keys, and their own outputs are not defined (returned as computed).
     """
     d, nh, hd = cfg.d_model, cfg.n_heads, cfg.head_dim
     eps = cfg.eps
@@ -185,6 +197,17 @@ def dit_block_forward(
     outs = []
     for b in range(x_all.shape[0]):
         x = x_all[b]
+        key_valid = None
+        pos_b = pos
+        if text_lens is not None:
+            L = int(text_lens[b])
+            assert 0 <= L <= n_text
+            key_valid = np.ones(S, dtype=bool)
+            key_valid[L:n_text] = False
+            own = mrope_positions(L, grid_h, grid_w, L if t_img is None else t_img)
+            pos_b = np.zeros((S, 3), dtype=np.int64)
+            pos_b[:L] = own[:L]
+            pos_b[n_text:] = own[L:]
         h = rmsnorm(x, g1, eps)
         # K and V for every token, Q only for the requested rows.
         k = (h @ W_qkv[d : 2 * d].T).reshape(S, nh, hd)
@@ -192,9 +215,9 @@ def dit_block_forward(
         q = (h[sel] @ W_qkv[:d].T).reshape(len(sel), nh, hd)
         q = rmsnorm(q, gq, eps)
         k = rmsnorm(k, gk, eps)
-        q = mrope(q, pos[sel], cfg.rope_sections, cfg.rope_theta)
-        k = mrope(k, pos, cfg.rope_sections, cfg.rope_theta)
-        o = attention(q, k, v).reshape(len(sel), d)
+        q = mrope(q, pos_b[sel], cfg.rope_sections, cfg.rope_theta)
+        k = mrope(k, pos_b, cfg.rope_sections, cfg.rope_theta)
+        o = attention(q, k, v, key_valid).reshape(len(sel), d)
         x1 = x[sel] + o @ W_o.T
         h2 = rmsnorm(x1, g2, eps)
         u = gelu(h2 @ W_up.T, tanh=bool(cfg.gelu_tanh))

@@ -440,3 +440,44 @@ def test_stack_of_blocks_with_zero_outputs_is_identity():
     one = oracle.dit_block_forward(cfg, w, x_bits, 2, 2, 2)
     assert np.array_equal(two, oracle.bf16_to_f64(oracle.f64_to_bf16_bits(one)))
     assert not np.array_equal(two, one)
+
+
+# ---------------------------------------------------------------- padded batches of prompts
+
+
+def test_padded_text_with_full_lengths_is_the_plain_block():
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg)
+    x_bits = synth.to_bf16_bits(np.random.default_rng(31).standard_normal((2, 5 + 4, cfg.d_model)))
+    plain = oracle.dit_block_forward(cfg, w, x_bits, 5, 2, 2)
+    assert np.array_equal(oracle.dit_block_forward(cfg, w, x_bits, 5, 2, 2, text_lens=[5, 5]), plain)
+
+
+def test_padded_text_rows_equal_each_prompt_alone():
+    """A batch of prompts with 3 and 5 text tokens padded to 5: every real row equals the block
+    run on that prompt alone (its own positions, no padding); padding is invisible as a key."""
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg)
+    r = np.random.default_rng(32)
+    n_text, gh, gw = 5, 2, 3
+    x_bits = synth.to_bf16_bits(r.standard_normal((2, n_text + gh * gw, cfg.d_model)))
+    lens = [3, 5]
+    got = oracle.dit_block_forward(cfg, w, x_bits, n_text, gh, gw, text_lens=lens)
+    for b, L in enumerate(lens):
+        keep = np.r_[0:L, n_text:n_text + gh * gw]
+        alone = oracle.dit_block_forward(cfg, w, x_bits[b:b + 1, keep], L, gh, gw)[0]
+        assert np.allclose(got[b, keep], alone, rtol=1e-12, atol=1e-12)
+    # the padding rows' contents change nothing else
+    x2 = x_bits.copy()
+    x2[0, 3:5] = synth.to_bf16_bits(r.standard_normal((2, cfg.d_model)) * 7.0)
+    got2 = oracle.dit_block_forward(cfg, w, x2, n_text, gh, gw, text_lens=lens)
+    keep0 = np.r_[0:3, n_text:n_text + gh * gw]
+    assert np.array_equal(got2[0, keep0], got[0, keep0])
+    assert np.array_equal(got2[1], got[1])
+
+
+def test_masked_attention_equals_attention_over_the_kept_keys():
+    r = np.random.default_rng(33)
+    q, k, v = (r.standard_normal((4, 2, 8)), r.standard_normal((7, 2, 8)), r.standard_normal((7, 2, 8)))
+    keep = np.array([1, 0, 1, 1, 0, 0, 1], dtype=bool)
+    assert np.allclose(oracle.attention(q, k, v, keep), oracle.attention(q, k[keep], v[keep]), rtol=1e-13, atol=1e-13)
