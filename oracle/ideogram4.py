@@ -175,10 +175,11 @@ def dit_block_forward(
     computed (K and V still cover every token) and the result is [B, len(rows), d].
 
     ``text_lens`` (one per batch element, each <= n_text) makes a padded batch of prompts of
-    different lengths: element b's text occupies rows [0, text_lens[b]) and rows
-    [text_lens[b], n_text) are padding.  Each element is positioned as if unpadded (text j at
-    (j, j, j), image cell (r, c) at (text_lens[b], r, c) unless t_img is given), padding rows
-    are excluded as keys, and their own outputs are not defined (returned as computed).
+    different lengths: element b holds its text_lens[b] text rows, then its grid_h*grid_w image
+    rows, then n_text - text_lens[b] rows of padding at the end.  Each element is positioned as
+    if alone (text j at (j, j, j), image cell (r, c) at (text_lens[b], r, c) unless t_img is
+    given), padding rows are excluded as keys, and their own outputs are not defined (returned
+    as computed).
     """
     d, nh, hd = cfg.d_model, cfg.n_heads, cfg.head_dim
     eps = cfg.eps
@@ -202,12 +203,10 @@ def dit_block_forward(
         if text_lens is not None:
             L = int(text_lens[b])
             assert 0 <= L <= n_text
-            key_valid = np.ones(S, dtype=bool)
-            key_valid[L:n_text] = False
-            own = mrope_positions(L, grid_h, grid_w, L if t_img is None else t_img)
+            n_valid = L + grid_h * grid_w
+            key_valid = np.arange(S) < n_valid
             pos_b = np.zeros((S, 3), dtype=np.int64)
-            pos_b[:L] = own[:L]
-            pos_b[n_text:] = own[L:]
+            pos_b[:n_valid] = mrope_positions(L, grid_h, grid_w, L if t_img is None else t_img)
         h = rmsnorm(x, g1, eps)
         # K and V for every token, Q only for the requested rows.
         k = (h @ W_qkv[d : 2 * d].T).reshape(S, nh, hd)

@@ -454,8 +454,9 @@ def test_padded_text_with_full_lengths_is_the_plain_block():
 
 
 def test_padded_text_rows_equal_each_prompt_alone():
-    """A batch of prompts with 3 and 5 text tokens padded to 5: every real row equals the block
-    run on that prompt alone (its own positions, no padding); padding is invisible as a key."""
+    """A batch of prompts with 3 and 5 text tokens, each followed by its 2x3 image tokens and padded
+    at the end to 5 + 6 rows: every real row equals the block run on that prompt alone (its own
+    positions, no padding); padding is invisible as a key."""
     cfg = _tiny_cfg()
     w = _tiny_weights(cfg)
     r = np.random.default_rng(32)
@@ -464,15 +465,14 @@ def test_padded_text_rows_equal_each_prompt_alone():
     lens = [3, 5]
     got = oracle.dit_block_forward(cfg, w, x_bits, n_text, gh, gw, text_lens=lens)
     for b, L in enumerate(lens):
-        keep = np.r_[0:L, n_text:n_text + gh * gw]
-        alone = oracle.dit_block_forward(cfg, w, x_bits[b:b + 1, keep], L, gh, gw)[0]
-        assert np.allclose(got[b, keep], alone, rtol=1e-12, atol=1e-12)
+        n = L + gh * gw
+        alone = oracle.dit_block_forward(cfg, w, x_bits[b:b + 1, :n], L, gh, gw)[0]
+        assert np.allclose(got[b, :n], alone, rtol=1e-12, atol=1e-12)
     # the padding rows' contents change nothing else
     x2 = x_bits.copy()
-    x2[0, 3:5] = synth.to_bf16_bits(r.standard_normal((2, cfg.d_model)) * 7.0)
+    x2[0, 3 + gh * gw:] = synth.to_bf16_bits(r.standard_normal((2, cfg.d_model)) * 7.0)
     got2 = oracle.dit_block_forward(cfg, w, x2, n_text, gh, gw, text_lens=lens)
-    keep0 = np.r_[0:3, n_text:n_text + gh * gw]
-    assert np.array_equal(got2[0, keep0], got[0, keep0])
+    assert np.array_equal(got2[0, :3 + gh * gw], got[0, :3 + gh * gw])
     assert np.array_equal(got2[1], got[1])
 
 
