@@ -138,10 +138,20 @@ def make_config(shape) -> BlockConfig:
 
 
 def make_weights(w) -> BlockWeights:
-    """``w``: dict of device tensors named like the struct fields."""
+    """``w``: dict of device tensors named like the struct fields.
+
+    The struct holds raw device addresses, so it also keeps a reference to every tensor it
+    points into: the weights stay allocated for as long as the returned struct is alive, even
+    when the caller's dict was a temporary.  Keep the struct alive until the kernels that read
+    the weights have been queued (torch's caching allocator reuses freed memory in stream
+    order, so work on the tensors' own stream is safe once the call has returned)."""
     bw = BlockWeights()
+    keep = {}
     for name, _ in BlockWeights._fields_:
-        setattr(bw, name, _ptr(w[name]))
+        t = w[name]
+        setattr(bw, name, _ptr(t))
+        keep[name] = t
+    bw._keep = keep
     return bw
 
 

@@ -45,4 +45,13 @@ def empty_bf16(*shape) -> torch.Tensor:
 
 
 def workspace(nbytes: int) -> torch.Tensor:
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device="cuda")
+    """Device scratch filled with 0xFF bytes (NaN in every 16- and 32-bit float format), so that a
+    kernel reading scratch it has not written shows up as a non-finite output."""
+    return torch.full((max(int(nbytes), 256),), 0xFF, dtype=torch.uint8, device="cuda")
+
+
+def poisoned_like(t: torch.Tensor) -> torch.Tensor:
+    """An output buffer of t's shape filled with 0xFF bytes (NaN as bf16, f16 and fp32)."""
+    out = torch.empty_like(t)
+    out.view(torch.uint8).fill_(0xFF)
+    return out

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from joint_attention_block_b200 import ops, synth
-from gpu_util import as_f64, assert_close, bits, dev, empty_bf16, workspace
+from gpu_util import as_f64, assert_close, bits, dev, empty_bf16, poisoned_like, workspace
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +32,7 @@ def run_block(shape, inp, n_text=None, gh=None, gw=None, t_img=-1, pos=None):
     wd = {k: dev(v) for k, v in inp.items() if k != "x"}
     weights = ops.make_weights(wd)
     x = dev(inp["x"])
-    out = torch.empty_like(x)
+    out = poisoned_like(x)
     ws = workspace(ops.block_workspace_bytes(cfg, x.shape[0], n_text, gh, gw))
     ops.dit_block_forward(cfg, weights, x, out, n_text, gh, gw, ws, t_img=t_img,
                           pos=None if pos is None else dev(pos.astype(np.int32)))
@@ -152,7 +152,7 @@ def _run_stack(shape, x_bits, wsets):
     dev_sets = [{k: dev(v) for k, v in w.items()} for w in wsets]  # kept alive for the call
     weights = [ops.make_weights(d) for d in dev_sets]
     x = dev(x_bits)
-    out = torch.empty_like(x)
+    out = poisoned_like(x)
     ws = workspace(ops.stack_workspace_bytes(cfg, x.shape[0], shape.n_text, shape.grid_h, shape.grid_w))
     ops.dit_stack_forward(cfg, weights, x, out, shape.n_text, shape.grid_h, shape.grid_w, ws)
     torch.cuda.synchronize()

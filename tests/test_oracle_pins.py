@@ -411,6 +411,22 @@ def test_block_flop_count():
 # ---------------------------------------------------------------- stacks of blocks
 
 
+def test_bf16_decode_all_patterns_match_torch():
+    """Every one of the 65,536 bf16 bit patterns decoded by the oracle against torch's own
+    bfloat16 -> float64 cast (a library routine): normals, subnormals, both zeros (sign kept),
+    both infinities and every NaN pattern (NaN in, NaN out)."""
+    pats = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = oracle.bf16_to_f64(pats)
+    want = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    fin = ~np.isnan(want)
+    assert np.array_equal(got[fin], want[fin])
+    assert np.array_equal(np.signbit(got[fin]), np.signbit(want[fin]))
+    # spot values fixed by the format: 0x3F80 = 1, 0xC000 = -2, 0x0001 = 2^-133, 0x7F80 = +inf
+    assert oracle.bf16_to_f64(np.array([0x3F80, 0xC000, 0x0001, 0x7F80], dtype=np.uint16)).tolist() == \
+        [1.0, -2.0, 2.0 ** -133, math.inf]
+
+
 def test_bf16_rounding_matches_torch():
     """The oracle's fp64 -> bf16 rounding against torch's own bf16 cast (a library routine),
     on random values, exact ties, huge and tiny magnitudes."""
