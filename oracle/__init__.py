@@ -8,6 +8,7 @@ from .ideogram4 import (  # noqa: F401
     attention,
     bf16_to_f64,
     cond_proj_forward,
+    denoise_steps,
     dequant,
     dit_block_forward,
     dit_stack_forward,

@@ -497,3 +497,61 @@ def test_masked_attention_equals_attention_over_the_kept_keys():
     q, k, v = (r.standard_normal((4, 2, 8)), r.standard_normal((7, 2, 8)), r.standard_normal((7, 2, 8)))
     keep = np.array([1, 0, 1, 1, 0, 0, 1], dtype=bool)
     assert np.allclose(oracle.attention(q, k, v, keep), oracle.attention(q, k[keep], v[keep]), rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- denoising steps and the guidance schedule
+
+
+def test_guidance_schedule_and_depth_follow_the_pages():
+    """V4_QUALITY_48 and the DiT depth as the pages print them (tests/golden/page_facts.json)."""
+    from joint_attention_block_b200 import schedule
+
+    f = facts()
+    q = f["v4_quality_48"]["value"]
+    gw = schedule.guidance("V4_QUALITY_48")
+    assert len(gw) == q["steps"] == q["n_first"] + q["n_last"]
+    assert gw[: q["n_first"]] == [float(q["gw_first"])] * q["n_first"]
+    assert gw[q["n_first"]:] == [float(q["gw_last"])] * q["n_last"]
+    assert schedule.DIT_LAYERS == f["dit_layers"]["value"]
+    dts = schedule.uniform_dts(q["steps"])
+    assert len(dts) == q["steps"] and abs(sum(dts) + 1.0) < 1e-6  # t runs from 1 to 0
+    assert all(d == np.float32(-1.0 / q["steps"]) for d in dts)
+
+
+def _zero_out(w):
+    z = dict(w)
+    z["w_o"] = np.zeros_like(w["w_o"])
+    z["w_down"] = np.zeros_like(w["w_down"])
+    return z
+
+
+def test_denoise_with_identity_stacks_is_a_closed_form():
+    """Stacks whose output projections are zero return their input, so each branch's velocity is
+    bf16(z) and every step is z + dt * bf16(z), whatever the guidance."""
+    cfg = _tiny_cfg()
+    w = _zero_out(_tiny_weights(cfg))
+    r = np.random.default_rng(40)
+    z0 = r.standard_normal((1, 4, cfg.d_model))
+    tc = synth.to_bf16_bits(r.standard_normal((1, 3, cfg.d_model)))
+    tu = synth.to_bf16_bits(np.zeros((1, 2, cfg.d_model)))
+    got = oracle.denoise_steps(cfg, [w, w], [w], tc, tu, z0, 2, 2, [7.0, 3.0], [-0.25, -0.5])
+    want = z0.copy()
+    for dt in (-0.25, -0.5):
+        want = want + dt * oracle.bf16_to_f64(oracle.f64_to_bf16_bits(want))
+    assert np.array_equal(got, want)
+
+
+def test_denoise_guidance_one_and_zero_drop_a_branch():
+    """gw = 1 uses only the conditional branch and gw = 0 only the unconditional one: changing the
+    other branch's weights changes nothing."""
+    cfg = _tiny_cfg()
+    wa, wb, wc = _tiny_weights(cfg, 41), _tiny_weights(cfg, 42), _tiny_weights(cfg, 43)
+    r = np.random.default_rng(44)
+    z0 = r.standard_normal((1, 4, cfg.d_model))
+    tc = synth.to_bf16_bits(r.standard_normal((1, 3, cfg.d_model)))
+    tu = synth.to_bf16_bits(np.zeros((1, 1, cfg.d_model)))
+    one = [oracle.denoise_steps(cfg, [wa], [u], tc, tu, z0, 2, 2, [1.0], [-0.1]) for u in (wb, wc)]
+    assert np.array_equal(one[0], one[1])
+    zero = [oracle.denoise_steps(cfg, [c], [wb], tc, tu, z0, 2, 2, [0.0], [-0.1]) for c in (wa, wc)]
+    assert np.array_equal(zero[0], zero[1])
+    assert not np.array_equal(one[0], zero[0])
