@@ -12,6 +12,7 @@ from .ideogram4 import (  # noqa: F401
     dequant,
     dit_block_forward,
     dit_stack_forward,
+    e4m3_round,
     e4m3_to_f64,
     euler_cfg_step,
     f64_to_bf16_bits,
@@ -20,5 +21,6 @@ from .ideogram4 import (  # noqa: F401
     mrope,
     mrope_angles,
     mrope_positions,
+    quantize_rows_act,
     rmsnorm,
 )

@@ -69,6 +69,29 @@ def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
     return np.where((e == 0xF) & ((c & 0x7) == 0x7), np.nan, val)
 
 
+def e4m3_round(v: np.ndarray) -> np.ndarray:
+    """Nearest e4m3 value (ties to even), saturating at +-448, written from the format: a finite
+    magnitude in [2^e, 2^(e+1)) with e >= -6 has 3 fraction bits, so the spacing there is
+    2^(e-3); below 2^-6 the subnormal spacing is 2^-9; 448 = 1.75 * 2^8 is the largest value."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)  # a = m * 2^ex with m in [0.5, 1), so the binary exponent is ex - 1
+    e = np.maximum(ex - 1, -6)
+    step = np.exp2(e.astype(np.float64) - 3.0)
+    q = np.round(a / step) * step  # numpy rounds halves to even; a / step is exact in fp64
+    return np.sign(v) * np.minimum(q, 448.0)
+
+
+def quantize_rows_act(h: np.ndarray):
+    """Per-token e4m3 quantisation of activations [rows, cols]: scale_row = fp32(amax_row / 448)
+    (1 for an all-zero row), values e4m3_round(h / scale_row).  Returns (dequantised values, scales);
+    the product of a code and its scale is exact in fp64."""
+    h = np.asarray(h, dtype=np.float64)
+    amax = np.abs(h).max(axis=-1, keepdims=True)
+    scale = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32).astype(np.float64)
+    return e4m3_round(h / scale) * scale, scale[..., 0]
+
+
 def dequant(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     """Real weight = fp8 value * weight_scale[:, None] (scale indexed by output row)."""
     return e4m3_to_f64(codes) * np.asarray(scale, dtype=np.float32).astype(np.float64)[:, None]
@@ -165,8 +188,13 @@ def dit_block_forward(
     rows: Optional[np.ndarray] = None,
     pos: Optional[np.ndarray] = None,
     text_lens: Optional[Sequence[int]] = None,
+    w8a8: bool = False,
 ) -> np.ndarray:
     """One single-stream DiT block forward, fp64, for x [B, S, d] (bf16 bits) -> [B, S, d].
+
+    ``w8a8`` quantises the inputs of the QKV and MLP-up projections (the two pre-norm outputs)
+    to e4m3 per token (quantize_rows_act) before the FP8-weight products, as an FP8-activation
+    pipeline would; the other products keep 16-bit activations.
 
     ``cfg`` carries d_model, n_heads, head_dim, d_mlp, rope_sections, rope_theta,
     eps, gelu_tanh.  ``w`` holds e4m3 codes w_qkv [3d, d], w_o [d, d], w_up [F, d],
@@ -208,6 +236,8 @@ def dit_block_forward(
             pos_b = np.zeros((S, 3), dtype=np.int64)
             pos_b[:n_valid] = mrope_positions(L, grid_h, grid_w, L if t_img is None else t_img)
         h = rmsnorm(x, g1, eps)
+        if w8a8:
+            h = quantize_rows_act(h)[0]
         # K and V for every token, Q only for the requested rows.
         k = (h @ W_qkv[d : 2 * d].T).reshape(S, nh, hd)
         v = (h @ W_qkv[2 * d :].T).reshape(S, nh, hd)
@@ -219,6 +249,8 @@ def dit_block_forward(
         o = attention(q, k, v, key_valid).reshape(len(sel), d)
         x1 = x[sel] + o @ W_o.T
         h2 = rmsnorm(x1, g2, eps)
+        if w8a8:
+            h2 = quantize_rows_act(h2)[0]
         u = gelu(h2 @ W_up.T, tanh=bool(cfg.gelu_tanh))
         outs.append(x1 + u @ W_dn.T)
     return np.stack(outs)

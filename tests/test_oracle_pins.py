@@ -555,3 +555,59 @@ def test_denoise_guidance_one_and_zero_drop_a_branch():
     zero = [oracle.denoise_steps(cfg, [c], [wb], tc, tu, z0, 2, 2, [0.0], [-0.1]) for c in (wa, wc)]
     assert np.array_equal(zero[0], zero[1])
     assert not np.array_equal(one[0], zero[0])
+
+
+# ---------------------------------------------------------------- FP8 activations (W8A8 variant)
+
+
+def test_e4m3_round_matches_torch_float8_cast():
+    """The oracle's e4m3 rounding against torch's float32 -> float8_e4m3fn cast (a library routine)
+    on random in-range values, every exact tie between neighbouring codes, subnormals and zeros;
+    values beyond 448 saturate."""
+    r = np.random.default_rng(80)
+    x = np.concatenate([r.standard_normal(20000) * 10.0 ** r.uniform(-3, 2.6, 20000),
+                        r.uniform(-448, 448, 5000), [0.0, -0.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -10, 448.0, -448.0]])
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle.e4m3_to_f64(codes)
+    fin = np.sort(np.unique(vals[np.isfinite(vals)]))
+    ties = (fin[:-1] + fin[1:]) / 2.0  # halfway points: ties to even
+    x = np.concatenate([x, ties]).astype(np.float32)
+    x = x[np.abs(x) <= 448.0]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_round(x.astype(np.float64)), want)
+    assert oracle.e4m3_round(np.array([500.0, -1e6, 449.0]))[:].tolist() == [448.0, -448.0, 448.0]
+    assert np.array_equal(oracle.e4m3_round(fin), fin)  # every code is a fixed point
+
+
+def test_activation_quantiser_scale_and_range():
+    r = np.random.default_rng(81)
+    h = r.standard_normal((5, 64)) * np.array([[1.0], [0.01], [100.0], [3.0], [0.5]])
+    h[3] = 0.0
+    q, s = oracle.quantize_rows_act(h)
+    amax = np.abs(h).max(axis=1)
+    assert np.array_equal(s, np.where(amax > 0, (amax / 448.0).astype(np.float32), 1.0))
+    assert np.all(np.abs(q).max(axis=1)[amax > 0] <= 448.0 * s[amax > 0] * (1 + 1e-12))
+    assert np.array_equal(q[3], np.zeros(64))
+    # relative error of each element at most half an e4m3 step (2^-4 of its binade), or the subnormal step
+    err = np.abs(q - h) / s[:, None]
+    mag = np.abs(h) / s[:, None]
+    bound = np.maximum(np.exp2(np.floor(np.log2(np.maximum(mag, 2.0 ** -6))) - 4.0), 2.0 ** -10)
+    assert np.all(err <= bound * (1 + 1e-12))
+    q2, s2 = oracle.quantize_rows_act(q)
+    assert np.allclose(q2, q, rtol=0, atol=1e-12 * np.abs(q).max())  # quantised rows stay put
+
+
+def test_w8a8_block_is_the_block_with_quantised_norm_outputs():
+    """The W8A8 block differs from the W8A16 block only through the two quantised inputs: with the
+    attention and MLP output projections zeroed both reduce to the residual path exactly, and with
+    real weights the difference is the few per cent that e4m3 activations cost."""
+    cfg = _tiny_cfg()
+    w = _zero_out(_tiny_weights(cfg))
+    x_bits = synth.to_bf16_bits(np.random.default_rng(82).standard_normal((1, 6, cfg.d_model)))
+    a = oracle.dit_block_forward(cfg, w, x_bits, 2, 2, 2, w8a8=True)
+    assert np.array_equal(a, oracle.bf16_to_f64(x_bits))
+    w2 = _tiny_weights(cfg)
+    b16 = oracle.dit_block_forward(cfg, w2, x_bits, 2, 2, 2)
+    b8 = oracle.dit_block_forward(cfg, w2, x_bits, 2, 2, 2, w8a8=True)
+    assert not np.array_equal(b8, b16)
+    assert np.abs(b8 - b16).max() / np.abs(b16).max() < 0.1  # a few per cent from e4m3 activations
