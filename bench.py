@@ -76,24 +76,31 @@ def attention_flops_per_step():
 # ------------------------------------------------------------------ DRAM traffic from the committed ncu summary
 
 
-def traffic_per_launch(kernel: str):
-    """DRAM bytes (read + write) per launch from profiles/ncu_traffic.json, or None when the
-    kernel source changed since those counters were taken."""
+def sources_sha256(paths):
+    """sha256 over the bytes of the given repo files, in order (a kernel and the headers it includes)."""
     import hashlib
 
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_per_launch(kernel: str):
+    """DRAM bytes (read + write) per launch from profiles/ncu_traffic.json, or None when the
+    kernel's sources changed since those counters were taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec:
+    if not rec or "sources" not in rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src):
+    if not all(os.path.exists(os.path.join(ROOT, p)) for p in rec["sources"]):
         return None
-    with open(src, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-            return None
+    if sources_sha256(rec["sources"]) != rec["sources_sha256"]:
+        return None
     return rec["dram_bytes_per_launch"]
 
 
@@ -153,19 +160,20 @@ class ClockSampler:
 
 
 def oracle_sample_step(state):
-    """One bounded sample of the step on the host: 1 query row of the block (K/V over all
-    4608 tokens), 1 conditioning token, and the whole Euler/CFG update."""
+    """One bounded sample of the step on the host: 2 query rows of the block (one text, one image;
+    K/V over all 4608 tokens), 1 conditioning token, and the whole Euler/CFG update."""
     import oracle
 
     s = synth.C1024
-    row = np.array([state["row"] % s.seq])
+    r = state["row"] % s.n_text
+    rows = np.array([r, s.n_text + (state["row"] * 7) % s.n_img])
     state["row"] += 997
     oracle.cond_proj_forward(state["cond"]["feats"][:1], state["cond"]["g"], synth.COND.eps, state["cond"]["w"],
                              state["cond"]["scale"])
-    oracle.dit_block_forward(s, state["blk"], state["blk"]["x"], s.n_text, s.grid_h, s.grid_w, rows=row)
+    oracle.dit_block_forward(s, state["blk"], state["blk"]["x"], s.n_text, s.grid_h, s.grid_w, rows=rows)
     e = state["eul"]
     oracle.euler_cfg_step(e["x"], e["v_cond"], e["v_uncond"], synth.CFG_GUIDANCE, synth.CFG_DT)
-    return 1  # block tokens processed
+    return len(rows)  # block tokens processed
 
 
 def oracle_state():
@@ -182,17 +190,8 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-SAMPLE_DESC = ("per step: 1 of 4608 query rows of the c1024 block (K/V projections over all 4608 tokens), "
+SAMPLE_DESC = ("per step: 2 of 4608 query rows of the c1024 block (K/V projections over all 4608 tokens), "
                "cond_proj of 1 of 512 tokens, full Euler/CFG on 4096x128; fp64 numpy oracle")
-
-
-def cpu_baseline():
-    st = oracle_state()
-    t0 = time.perf_counter()
-    n = oracle_sample_step(st)
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": SAMPLE_DESC,
-            "seconds": dt}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -229,10 +228,19 @@ def run_reference(args, rank, world):
 # ------------------------------------------------------------------ our arm
 
 
+def _kernel_table(records, prof_steps):
+    per = {}
+    for name, t in records:
+        d = per.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += t
+    return per
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
-    from joint_attention_block_b200 import ops
+    from joint_attention_block_b200 import ops, schedule
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -249,22 +257,30 @@ def run_ours(args, rank, world, local_rank):
     cfg = ops.make_config(s)
     wd = {k: to_dev(v) for k, v in blk.items() if k != "x"}
     weights = ops.make_weights(wd)
-    x_in = to_dev(blk["x"])  # [1, 4608, 4096]; rows 0..511 are overwritten by the projection
-    x_out = torch.empty_like(x_in)
-    text_rows = x_in.view(s.seq, s.d_model)[: s.n_text]
-    img_rows = x_in.view(s.seq, s.d_model)[s.n_text:]
-    feats, g_c, w_c, sc_c = (to_dev(cond[k]) for k in ("feats", "g", "w", "scale"))
-    lat, vc, vu = (to_dev(eul[k]) for k in ("x", "v_cond", "v_uncond"))
+    g_c, w_c, sc_c = (to_dev(cond[k]) for k in ("g", "w", "scale"))
     ws_blk = torch.empty(ops.block_workspace_bytes(cfg, 1, s.n_text, s.grid_h, s.grid_w), dtype=torch.uint8, device=dev)
     ws_c = torch.empty(ops.cond_proj_workspace_bytes(c.n_tok, c.n_layers, c.hidden, c.d_out), dtype=torch.uint8,
                        device=dev)
     dt = float(np.float32(synth.CFG_DT))
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        ops.cond_proj_forward(feats, c.n_layers, c.hidden, g_c, c.eps, w_c, sc_c, text_rows, ws_c, stream=stream)
-        ops.dit_block_forward(cfg, weights, x_in, x_out, s.n_text, s.grid_h, s.grid_w, ws_blk, stream=stream)
-        ops.euler_cfg_step(lat, vc, vu, synth.CFG_GUIDANCE, dt, stream=stream)
+    class Buffers:
+        """One set of the step's per-step inputs and outputs."""
+
+        def __init__(self):
+            self.feats = to_dev(cond["feats"])
+            self.x_in = to_dev(blk["x"])  # [1, 4608, 4096]; rows 0..511 are overwritten by the projection
+            self.x_out = torch.empty_like(self.x_in)
+            self.text_rows = self.x_in.view(s.seq, s.d_model)[: s.n_text]
+            self.img_rows = self.x_in.view(s.seq, s.d_model)[s.n_text:]
+            self.lat, self.vc, self.vu = (to_dev(eul[k]) for k in ("x", "v_cond", "v_uncond"))
+
+    B0 = Buffers()
+
+    def step(b=B0):
+        ops.cond_proj_forward(b.feats, c.n_layers, c.hidden, g_c, c.eps, w_c, sc_c, b.text_rows, ws_c, stream=stream)
+        ops.dit_block_forward(cfg, weights, b.x_in, b.x_out, s.n_text, s.grid_h, s.grid_w, ws_blk, stream=stream)
+        ops.euler_cfg_step(b.lat, b.vc, b.vu, synth.CFG_GUIDANCE, dt, stream=stream)
 
     from joint_attention_block_b200 import replicas
 
@@ -273,13 +289,16 @@ def run_ours(args, rank, world, local_rank):
     def max_over_ranks(v: float) -> float:
         return replicas.max_over_ranks(v, dev)
 
+    def check_errors(where):
+        if ops.poll_error() != 0:
+            raise RuntimeError(f"device-side error {where}: {ops.last_device_error():#x}")
+
     for i in range(args.warmup):
         step()
-        if i == 0 and ops.poll_error() != 0:  # fail fast: a broken step must not be repeated
-            raise RuntimeError(f"device-side error in the first step: {ops.last_device_error():#x}")
+        if i == 0:
+            check_errors("in the first step")  # fail fast: a broken step must not be repeated
     torch.cuda.synchronize(dev)
-    if ops.poll_error() != 0:
-        raise RuntimeError(f"device-side error during warm-up: {ops.last_device_error():#x}")
+    check_errors("during warm-up")
 
     # ---- timed region: device-resident inputs, nothing but the step's own launches on the stream
     clocks = ClockSampler(local_rank)
@@ -298,8 +317,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clocks.stop()
     ms = max_over_ranks(ev0.elapsed_time(ev1))
-    if ops.poll_error() != 0:
-        raise RuntimeError(f"device-side error in the timed region: {ops.last_device_error():#x}")
+    check_errors("in the timed region")
 
     # ---- per-kernel device times: the same steps again with the library's launch events, which
     # sit between the kernels and so also stop each kernel from starting during its predecessor's
@@ -311,58 +329,96 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     ops.profile_disable()
     records = ops.profile_read(prof_steps * 24 + 64)
-    if ops.poll_error() != 0:
-        raise RuntimeError(f"device-side error in the profiled steps: {ops.last_device_error():#x}")
+    check_errors("in the profiled steps")
 
-    # ---- end to end through the public calls: pinned host inputs in, results out, every step
+    # ---- end to end through the public calls: pinned host inputs in, results out, every step.
+    # Two buffer sets: while the compute stream runs step i on one set, a copy stream fills the
+    # other set with step i+1's inputs and a second copy stream reads step i-1's results back.
     h_feats = torch.from_numpy(cond["feats"].view(np.int16)).pin_memory()
     h_img = torch.from_numpy(np.ascontiguousarray(blk["x"].reshape(s.seq, s.d_model)[s.n_text:]).view(np.int16)).pin_memory()
     h_lat = torch.from_numpy(eul["x"]).pin_memory()
     h_vc = torch.from_numpy(eul["v_cond"].view(np.int16)).pin_memory()
     h_vu = torch.from_numpy(eul["v_uncond"].view(np.int16)).pin_memory()
-    h_out = torch.empty(x_out.shape, dtype=x_out.dtype).pin_memory()
+    h_out = torch.empty(B0.x_out.shape, dtype=B0.x_out.dtype).pin_memory()
     h_lat_out = torch.empty_like(h_lat).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_feats, h_img, h_lat, h_vc, h_vu))
     d2h = h_out.numel() * h_out.element_size() + h_lat_out.numel() * h_lat_out.element_size()
+    sets = [B0, Buffers()]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in sets]
+    out_ready = [torch.cuda.Event() for _ in sets]
+    out_done = [torch.cuda.Event() for _ in sets]
 
-    def e2e_step():
-        feats.copy_(h_feats, non_blocking=True)
-        img_rows.copy_(h_img, non_blocking=True)
-        lat.copy_(h_lat, non_blocking=True)
-        vc.copy_(h_vc, non_blocking=True)
-        vu.copy_(h_vu, non_blocking=True)
-        step()
-        h_out.copy_(x_out, non_blocking=True)
-        h_lat_out.copy_(lat, non_blocking=True)
+    def e2e_step(i):
+        k = i % 2
+        b = sets[k]
+        s_in.wait_event(out_done[k])  # step i-2 on this set is computed and copied out
+        with torch.cuda.stream(s_in):
+            b.feats.copy_(h_feats, non_blocking=True)
+            b.img_rows.copy_(h_img, non_blocking=True)
+            b.lat.copy_(h_lat, non_blocking=True)
+            b.vc.copy_(h_vc, non_blocking=True)
+            b.vu.copy_(h_vu, non_blocking=True)
+            in_ready[k].record(s_in)
+        stream.wait_event(in_ready[k])
+        step(b)
+        out_ready[k].record(stream)
+        s_out.wait_event(out_ready[k])
+        with torch.cuda.stream(s_out):
+            h_out.copy_(b.x_out, non_blocking=True)
+            h_lat_out.copy_(b.lat, non_blocking=True)
+            out_done[k].record(s_out)
 
     e2e_steps = max(3, min(args.steps, 20))
-    e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier()
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    ev1.record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    s_out.synchronize()
+    e1.record(s_out)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    check_errors("in the end-to-end steps")
+
+    c2048 = measure_c2048(ops, weights, dev, stream) if not args.no_extras else None
+    w8a8 = measure_w8a8(ops, cfg, weights, B0.x_in, ws_blk, dev, stream) if not args.no_extras else None
+    denoise = measure_denoise(ops, schedule, dev, stream) if not args.no_extras else None
+    check_errors("in the extra measurements")
 
     if rank != 0:
         return
+
+    # ---- correctness of what was timed: a plain step on the first buffer set, then sampled rows
+    # of its outputs against the oracle (the oracle's time is the CPU baseline)
+    step()
+    torch.cuda.synchronize(dev)
+    x_bits = B0.x_in.cpu().numpy().view(np.uint16)
+    y_bits = B0.x_out.cpu().numpy().view(np.uint16)
+    lat_before = B0.lat.cpu().numpy().copy()
+    ops.euler_cfg_step(B0.lat, B0.vc, B0.vu, synth.CFG_GUIDANCE, dt, stream=stream)
+    lat_after = B0.lat.cpu().numpy()
+    check_errors("in the checked step")
+    check, base = oracle_check(x_bits, y_bits, lat_before, lat_after, blk, cond, eul, dt)
 
     # ---- numbers
     toks = s.seq * args.steps * world
     value = toks / (ms / 1e3)
     tflops = step_flops() * args.steps * world / (ms / 1e3) / 1e12
     pk, pk_kind = peaks()
-    per = {}
-    for name, t in records:
-        d = per.setdefault(name, [0, 0.0])
-        d[0] += 1
-        d[1] += t
+    per = _kernel_table(records, prof_steps)
     total_kernel_ms = sum(v[1] for v in per.values())
     gf = gemm_flops_per_step()
-    peak_tc = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    # The per-kernel times come from a region well under a second (the GPU does not reach its
+    # power-capped steady state there), so the burst peak is the denominator; the sustained one
+    # applies only to regions of seconds.
+    prof_region_ms = total_kernel_ms
+    sustained = prof_region_ms >= 1000.0
+    peak_tc = pk.get("bf16_tflops_sustained" if sustained else "bf16_tflops", pk.get("bf16_tflops"))
     kernels = {}
     for n, (cnt, t) in sorted(per.items(), key=lambda kv: -kv[1][1]):
         k = {"launches": cnt, "ms_total": round(t, 4), "ms_avg": round(t / cnt, 5),
@@ -371,6 +427,8 @@ def run_ours(args, rank, world, local_rank):
             k["tflops"] = round(gf[n] * cnt / (t / 1e3) / 1e12, 1)
         if n == "attention":
             k["tflops"] = round(attention_flops_per_step() * cnt / (t / 1e3) / 1e12, 1)
+        if "tflops" in k:
+            k["frac"] = round(k["tflops"] / peak_tc, 4)
         kernels[n] = k
     # dominant kernel: the MLP up-projection GEMM (largest share of the step)
     dom = "gemm_up"
@@ -403,7 +461,9 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": round(achieved, 1) if achieved else None, "peak": peak_tc, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_tc, 4) if achieved else None,
                      "traffic": traffic_per_launch(dom),
-                     "peak_kind": f"{pk_kind} bf16 dense, sustained (kernel timed inside the step)",
+                     "peak_kind": f"{pk_kind} bf16 dense, " + (
+                         "sustained (kernels timed over >= 1 s)" if sustained else
+                         f"burst (kernels timed over {prof_region_ms:.0f} ms, under the power cap's time scale)"),
                      "flops_per_launch": gf[dom], "launches": cnt, "ms_avg": round(t / cnt, 5) if cnt else None,
                      "all_gemms_tflops": round(gemm_all, 1) if gemm_all else None,
                      "all_gemms_frac": round(gemm_all / peak_tc, 4) if gemm_all else None},
@@ -412,11 +472,190 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": len(records) // prof_steps * args.steps,
         "clocks": clk,
         "e2e": {"value": round(s.seq * e2e_steps * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "pipeline": "two buffer sets; host-to-device and device-to-host copies on their own streams"},
+        "check": check,
     }
+    if c2048 is not None:
+        c2048["frac"] = round(c2048["tflops"] / peak_tc, 4)
+        if c2048.get("attention_tflops"):
+            c2048["attention_frac"] = round(c2048["attention_tflops"] / peak_tc, 4)
+        line["c2048"] = c2048
+    if w8a8 is not None:
+        line["w8a8"] = w8a8
+    if denoise is not None:
+        denoise["frac"] = round(denoise["tflops"] / pk.get("bf16_tflops_sustained", peak_tc), 4)
+        denoise["peak_kind"] = f"{pk_kind} bf16 dense, sustained (a {denoise['ms_per_step']:.0f} ms step)"
+        line["denoise"] = denoise
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
+        line["cpu_baseline"] = base
     print(json.dumps(line), flush=True)
+
+
+def measure_c2048(ops, weights, dev, stream):
+    """The 2048 px block (512 text + 128x128 image tokens, S = 16,896) with the 1024 px block's
+    weights (same widths): time per block and its attention's share, from CUDA events."""
+    import torch
+
+    s2 = synth.C2048
+    cfg2 = ops.make_config(s2)
+    x2 = synth.bf16_normal_device((1, s2.seq, s2.d_model), 4000, dev)
+    y2 = torch.empty_like(x2)
+    ws2 = torch.empty(ops.block_workspace_bytes(cfg2, 1, s2.n_text, s2.grid_h, s2.grid_w), dtype=torch.uint8,
+                      device=dev)
+
+    def run():
+        ops.dit_block_forward(cfg2, weights, x2, y2, s2.n_text, s2.grid_h, s2.grid_w, ws2, stream=stream)
+
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize(dev)
+    reps = 5
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(reps):
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / reps
+    ops.profile_enable(64)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize(dev)
+    ops.profile_disable()
+    per = _kernel_table(ops.profile_read(64), 3)
+    att = per.get("attention")
+    att_fl = 4.0 * s2.seq * s2.seq * s2.d_model
+    out = {"workload": "2048 px block: 512 text + 128x128 image tokens (S=16896), d=4096, 32x128 heads, MLP 16384",
+           "ms_per_block": round(ms, 4), "tokens_per_s": round(s2.seq / (ms / 1e3), 1),
+           "tflops": round(s2.flops() / (ms / 1e3) / 1e12, 1), "reps": reps}
+    if att:
+        out["attention_ms"] = round(att[1] / att[0], 4)
+        out["attention_tflops"] = round(att_fl / (att[1] / att[0] / 1e3) / 1e12, 1)
+        out["attention_share"] = round(att[1] / sum(v[1] for v in per.values()), 4)
+    del x2, y2, ws2
+    return out
+
+
+def measure_w8a8(ops, cfg, weights, x_in, ws, dev, stream):
+    """The 1024 px block through the W8A8 variant (e4m3 activations into the QKV and MLP-up
+    projections on the FP8 tensor path), same inputs and weights as the timed step."""
+    import torch
+
+    s = synth.C1024
+    y = torch.empty_like(x_in)
+
+    def run():
+        ops.dit_block_forward_w8a8(cfg, weights, x_in, y, s.n_text, s.grid_h, s.grid_w, ws, stream=stream)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize(dev)
+    reps = 10
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(reps):
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / reps
+    ops.profile_enable(64)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize(dev)
+    ops.profile_disable()
+    per = _kernel_table(ops.profile_read(64), 3)
+    S, d, F = s.seq, s.d_model, s.d_mlp
+    out = {"workload": "1024 px block, W8A8 variant (e4m3 per-token activations into QKV and MLP-up)",
+           "ms_per_block": round(ms, 4), "tokens_per_s": round(S / (ms / 1e3), 1),
+           "tflops": round(s.flops() / (ms / 1e3) / 1e12, 1), "reps": reps}
+    for name, fl in (("gemm_qkv", 2.0 * S * d * 3 * d), ("gemm_up", 2.0 * S * d * F)):
+        if name in per:
+            cnt, t = per[name]
+            out[name + "_fp8_tflops"] = round(fl * cnt / (t / 1e3) / 1e12, 1)
+    return out
+
+
+def measure_denoise(ops, schedule, dev, stream):
+    """One 1024 px denoising step through the whole depth (dit_denoise_steps): the conditional
+    stack (34 blocks, 512 text + 4096 image tokens), the unconditional stack (34 blocks, 32 zero
+    text + 4096 image tokens) and the CFG/Euler update, with V4_QUALITY_48's guidance.  Four
+    distinct weight sets (drawn on the device, 800 MB, far above L2) are cycled over the 68 blocks."""
+    import torch
+
+    sc, su = synth.C1024, synth.UNCOND1024
+    n_blocks = schedule.DIT_LAYERS
+    sets = [synth.block_weights_device(sc, 7000 + i, dev) for i in range(4)]
+    wts = [ops.make_weights(d) for d in sets]
+    w_cond = [wts[i % 4] for i in range(n_blocks)]
+    w_uncond = [wts[(i + 2) % 4] for i in range(n_blocks)]
+    cfg = ops.make_config(sc)
+    text_c = synth.bf16_normal_device((1, sc.n_text, sc.d_model), 4100, dev)
+    text_u = torch.zeros((1, su.n_text, su.d_model), dtype=torch.int16, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4200)
+    z = torch.randn((1, sc.n_img, sc.d_model), generator=gen, device=dev, dtype=torch.float32)
+    ws = torch.empty(ops.denoise_workspace_bytes(cfg, 1, sc.n_text, su.n_text, sc.grid_h, sc.grid_w),
+                     dtype=torch.uint8, device=dev)
+    gws = schedule.guidance("V4_QUALITY_48")
+    dts = schedule.uniform_dts(len(gws))
+
+    def run(i0, n):
+        ops.dit_denoise_steps(cfg, w_cond, w_uncond, text_c, text_u, z, sc.grid_h, sc.grid_w, gws[i0:i0 + n],
+                              dts[i0:i0 + n], ws, stream=stream)
+
+    run(0, 1)
+    torch.cuda.synchronize(dev)
+    reps = 3
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    run(44, reps)  # steps 45..47 of the preset: gw 7, then 3, 3
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / reps
+    flops = n_blocks * (sc.flops() + su.flops())
+    finite = bool(torch.isfinite(z).all().item())
+    del sets, wts, ws
+    return {"workload": "one 1024 px denoising step: 34 cond blocks (512 + 4096 tokens) + 34 uncond blocks "
+                        "(32 + 4096 tokens) + CFG/Euler, V4_QUALITY_48 guidance",
+            "ms_per_step": round(ms, 3), "tflops": round(flops / (ms / 1e3) / 1e12, 1), "steps_timed": reps,
+            "flops_per_step": flops, "latent_finite": finite, "launches_per_step": 2 * n_blocks * 9 + 2}
+
+
+def oracle_check(x_bits, y_bits, lat_before, lat_after, blk, cond, eul, dt):
+    """Sampled outputs of the timed step against the oracle: two block rows (one text, one image;
+    K and V over all 4608 tokens), one conditioning token and the whole Euler/CFG update.  Raises
+    if any is outside the tolerances; returns the check record and the CPU baseline (the oracle's
+    own time for this sample)."""
+    import oracle
+
+    s, c = synth.C1024, synth.COND
+    rows = np.array([7, s.n_text + 2345])
+    tok = 7
+    t0 = time.perf_counter()
+    ref_c = oracle.cond_proj_forward(cond["feats"][tok:tok + 1], cond["g"], c.eps, cond["w"], cond["scale"])
+    ref_b = oracle.dit_block_forward(s, blk, x_bits, s.n_text, s.grid_h, s.grid_w, rows=rows)
+    ref_e = oracle.euler_cfg_step(lat_before, eul["v_cond"], eul["v_uncond"], synth.CFG_GUIDANCE, dt)
+    secs = time.perf_counter() - t0
+
+    def rel(got, ref):
+        d = np.abs(got - ref)
+        return float(d.max() / np.abs(ref).max()), float(d.mean() / np.abs(ref).mean())
+
+    got_c = oracle.bf16_to_f64(x_bits[0, tok:tok + 1])
+    got_b = oracle.bf16_to_f64(y_bits[:, rows])
+    cmx, cmn = rel(got_c, ref_c)
+    bmx, bmn = rel(got_b, ref_b)
+    emx = float(np.abs(lat_after - ref_e).max())
+    ok = cmx <= 2e-2 and cmn <= 3e-3 and bmx <= 2e-2 and bmn <= 3e-3 and emx < 1e-5
+    check = {"ok": ok, "block_rows": rows.tolist(), "block_max_rel": round(bmx, 6), "block_mean_rel": round(bmn, 6),
+             "cond_token": tok, "cond_max_rel": round(cmx, 6), "cond_mean_rel": round(cmn, 6),
+             "euler_max_abs": emx, "tolerance": "max-rel 2e-2, mean-rel 3e-3; Euler 1e-5 abs"}
+    if not ok:
+        raise RuntimeError(f"bench output does not match the oracle: {check}")
+    base = {"value": len(rows) / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": SAMPLE_DESC, "seconds": secs}
+    return check, base
 
 
 # ------------------------------------------------------------------ HBM-bound kernels on their own
@@ -512,91 +751,22 @@ def run_elementwise(args, local_rank):
 
 
 def run_denoise(args, local_rank):
-    """One flow-matching denoising step at 1024 px through the full depth of the DiT: the
-    conditional stack (34 blocks over 512 text + 4096 image tokens), the unconditional stack
-    (34 blocks over 32 text + 4096 image tokens, its own weights) and the Euler/CFG update,
-    captured once in a CUDA graph and replayed.  Four distinct weight sets (800 MB, far above
-    L2) are cycled through the 68 blocks; the velocities fed to the update are the synthetic
-    ones of the step benchmark (the projection from block output to latent velocity is not on
-    the path).  One JSON line."""
-    import dataclasses
-
+    """One denoising step through the whole depth alone (see measure_denoise); one JSON line."""
     import torch
 
-    from joint_attention_block_b200 import ops
+    from joint_attention_block_b200 import ops, schedule
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    stream = torch.cuda.Stream(dev)
-    n_blocks = 34
-
-    def to_dev(a):
-        a = np.ascontiguousarray(a)
-        t = torch.from_numpy(a.view(np.int16)) if a.dtype == np.uint16 else torch.from_numpy(a)
-        return t.to(dev)
-
-    sc, su = synth.C1024, synth.UNCOND1024
-    sets = [synth.block_inputs(dataclasses.replace(sc, index=200 + i)) for i in range(4)]
-    x_c = to_dev(sets[0]["x"])
-    x_u = to_dev(synth.to_bf16_bits(synth.normal(su.index, 0, (1, su.seq, su.d_model))))
-    dev_sets = [{k: to_dev(v) for k, v in st.items() if k != "x"} for st in sets]
-    wts = [ops.make_weights(d) for d in dev_sets]
-    cond_w = [wts[i % 4] for i in range(n_blocks)]
-    uncond_w = [wts[(i + 2) % 4] for i in range(n_blocks)]
-    cfg_c, cfg_u = ops.make_config(sc), ops.make_config(su)
-    out_c, out_u = torch.empty_like(x_c), torch.empty_like(x_u)
-    ws_c = torch.empty(ops.stack_workspace_bytes(cfg_c, 1, sc.n_text, sc.grid_h, sc.grid_w), dtype=torch.uint8,
-                       device=dev)
-    ws_u = torch.empty(ops.stack_workspace_bytes(cfg_u, 1, su.n_text, su.grid_h, su.grid_w), dtype=torch.uint8,
-                       device=dev)
-    eul = synth.euler_inputs(4096 * synth.LATENT_CHANNELS)
-    lat, vc, vu = (to_dev(eul[k]) for k in ("x", "v_cond", "v_uncond"))
-    dt = float(np.float32(synth.CFG_DT))
-
-    def step():
-        ops.dit_stack_forward(cfg_c, cond_w, x_c, out_c, sc.n_text, sc.grid_h, sc.grid_w, ws_c, stream=stream)
-        ops.dit_stack_forward(cfg_u, uncond_w, x_u, out_u, su.n_text, su.grid_h, su.grid_w, ws_u, stream=stream)
-        ops.euler_cfg_step(lat, vc, vu, synth.CFG_GUIDANCE, dt, stream=stream)
-
-    with torch.cuda.stream(stream):
-        for _ in range(max(args.warmup, 2)):
-            step()
-        stream.synchronize()
-        if ops.poll_error(stream) != 0:
-            raise RuntimeError(f"device-side error: {ops.last_device_error():#x}")
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            step()
-        graph.replay()
-        stream.synchronize()
-        reps = max(3, min(args.steps, 20))
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ev0.record(stream)
-        for _ in range(reps):
-            graph.replay()
-        ev1.record(stream)
-        stream.synchronize()
-        ms_graph = ev0.elapsed_time(ev1) / reps
-        ev0.record(stream)
-        for _ in range(reps):
-            step()
-        ev1.record(stream)
-        stream.synchronize()
-        ms_eager = ev0.elapsed_time(ev1) / reps
-        if ops.poll_error(stream) != 0:
-            raise RuntimeError(f"device-side error: {ops.last_device_error():#x}")
-    del graph
-    flops = n_blocks * (sc.flops() + su.flops())
+    stream = torch.cuda.current_stream(dev)
+    out = measure_denoise(ops, schedule, dev, stream)
+    if ops.poll_error() != 0:
+        raise RuntimeError(f"device-side error: {ops.last_device_error():#x}")
     pk, pk_kind = peaks()
-    print(json.dumps({
-        "metric": "one 1024 px denoising step: 34 cond blocks (4608 tok) + 34 uncond blocks (4128 tok) + Euler/CFG",
-        "ms_graph": round(ms_graph, 3), "ms_eager": round(ms_eager, 3), "reps": reps,
-        "tflops": round(flops / (ms_graph / 1e3) / 1e12, 1), "flops_per_step": flops,
-        "frac_of_bf16_sustained": round(flops / (ms_graph / 1e3) / 1e12 / pk.get("bf16_tflops_sustained", 1.0), 4),
-        "peak_kind": f"{pk_kind} bf16 dense, sustained",
-        "launches_per_step": 2 * n_blocks * 9 + 1,
-        "data": "synthetic; 4 distinct weight sets cycled over the 68 blocks"}), flush=True)
-
+    out["frac"] = round(out["tflops"] / pk.get("bf16_tflops_sustained", 1.0), 4)
+    out["peak_kind"] = f"{pk_kind} bf16 dense, sustained"
+    out["metric"] = "one 1024 px denoising step (34 + 34 blocks + CFG/Euler)"
+    print(json.dumps(out), flush=True)
 
 
 def main():
@@ -606,6 +776,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--no-extras", action="store_true", help="skip the 2048 px block and the denoising step")
     ap.add_argument("--elementwise", action="store_true",
                     help="instead of the step: HBM bandwidth of the norm / QK-norm / Euler kernels alone")
     ap.add_argument("--denoise", action="store_true",

@@ -101,6 +101,34 @@ DIT_API int dit_block_forward(const dit_block_config* cfg, const dit_block_weigh
                       int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                       void* workspace, size_t ws_bytes, void* stream);
 
+/* dit_block_forward over a padded batch of prompts of different text lengths (SimpleTuner
+ * Ideogram 4 quickstart, "Text Embed Cache": text embeddings are kept at each prompt's own token
+ * length and only padded when a batch is formed).  Element b of x_in [batch, n_text +
+ * grid_h*grid_w, d_model] holds, in this order, its L_b text rows, its grid_h*grid_w image rows
+ * (raster order) and n_text - L_b rows of padding.  Every element is computed as if it were run
+ * alone: text token j at (j, j, j), image cell (r, c) at (t, r, c) with t = L_b (or t_img when
+ * t_img >= 0), and its attention takes only its first L_b + grid_h*grid_w tokens as keys.  The
+ * outputs of padding rows are unspecified (they are computed like any row, at position (0,0,0)).
+ * text_lens: DEVICE int32 [batch], 16-byte aligned; each value is clamped to [0, n_text]; an
+ *   element must have at least one token (L_b + grid_h*grid_w >= 1).
+ * workspace: >= dit_block_workspace_bytes() bytes (the same size as dit_block_forward).
+ * Errors: as dit_block_forward; INVALID_ARG for a null or misaligned text_lens. */
+DIT_API int dit_block_forward_padded(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in,
+                                     void* x_out, int batch, int n_text, int grid_h, int grid_w, int t_img,
+                                     const int32_t* text_lens, void* workspace, size_t ws_bytes, void* stream);
+
+/* The W8A8 variant of dit_block_forward: the inputs of the QKV and MLP-up projections (the two
+ * pre-norm outputs) are quantised to e4m3 per token (scale = amax of the row / 448, codes rounded
+ * to nearest even, saturating) and multiplied with the e4m3 weights on the FP8 tensor-core path
+ * (tcgen05 kind::f8f6f4, twice the 16-bit rate).  The attention, output and MLP-down products keep
+ * 16-bit activations.  The pages run the dequantised model with 16-bit activations; this variant
+ * trades accuracy for speed (FP8 training through fp8-torchao is what SimpleTuner's quickstart,
+ * "ハードウェアと精度", uses); its error against the 16-bit pipeline is a few per cent per element.
+ * Arguments, workspace and errors as dit_block_forward; UNSUPPORTED for d_model > 8192. */
+DIT_API int dit_block_forward_w8a8(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in,
+                                   void* x_out, int batch, int n_text, int grid_h, int grid_w, int t_img,
+                                   const int32_t* pos, void* workspace, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace dit_stack_forward needs: one block's workspace plus one
  * activation buffer [batch, S, d_model] bf16 for the ping-pong between blocks. */
 DIT_API size_t dit_stack_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w);
@@ -117,6 +145,45 @@ DIT_API size_t dit_stack_workspace_bytes(const dit_block_config* cfg, int batch,
 DIT_API int dit_stack_forward(const dit_block_config* cfg, const dit_block_weights* w, int n_blocks, const void* x_in,
                               void* x_out, int batch, int n_text, int grid_h, int grid_w, int t_img,
                               const int32_t* pos, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace dit_denoise_steps needs: the block inputs and outputs of both
+ * branches ([batch, n_text + grid_h*grid_w, d_model] bf16, four buffers) plus the larger of the
+ * two stacks' workspaces. */
+DIT_API size_t dit_denoise_workspace_bytes(const dit_block_config* cfg, int batch, int n_text_c, int n_text_u,
+                                           int grid_h, int grid_w);
+
+/* n_steps flow-matching denoising steps with dual-branch classifier-free guidance (Ideogram 4
+ * deep dive, section 4-6 pseudocode; section 4-4: asymmetric CFG with a separate unconditional
+ * DiT, and a guidance weight that may change per step, e.g. V4_QUALITY_48 = 45 steps at 7 then
+ * 3 steps at 3).  Per step i:
+ *   v_c = stack_cond  ([text_cond;   z])   (n_blocks blocks, weights w_cond)
+ *   v_u = stack_uncond([text_uncond; z])   (n_blocks blocks, weights w_uncond)
+ *   z   = z + dt[i] * (v_u + guidance[i] * (v_c - v_u))    (= gw v_c + (1 - gw) v_u)
+ * The pages describe neither the map from the latent to the DiT's image tokens nor the final
+ * projection back to a velocity; both are taken as the identity here: z holds the image tokens
+ * themselves (d_model channels), enters each branch as bf16 rows after its text rows, and the
+ * velocity of a branch is the image rows of its stack's bf16 output.  The update is fp32 as in
+ * euler_cfg_step.
+ * text_cond: bf16 [batch, n_text_c, d_model]; text_uncond: bf16 [batch, n_text_u, d_model]
+ *   (the unconditional branch's text, zeros on the pages; n_text_u may be 0).
+ * z: fp32 [batch, grid_h*grid_w, d_model], updated in place.
+ * w_cond, w_uncond: HOST arrays of n_blocks weight sets each.
+ * guidance, dt: HOST arrays of n_steps values (dt = s - t < 0 when integrating from t=1 to 0).
+ * workspace: >= dit_denoise_workspace_bytes() bytes, 256-byte aligned.
+ * Errors: as dit_stack_forward; INVALID_ARG for null arrays or n_steps < 0. */
+DIT_API int dit_denoise_steps(const dit_block_config* cfg, const dit_block_weights* w_cond,
+                              const dit_block_weights* w_uncond, int n_blocks, const void* text_cond, int n_text_c,
+                              const void* text_uncond, int n_text_u, float* z, int batch, int grid_h, int grid_w,
+                              int n_steps, const float* guidance, const float* dt, void* workspace, size_t ws_bytes,
+                              void* stream);
+
+/* One branch's block input of a denoising step, the first part of each step of dit_denoise_steps
+ * (for callers that run the two branches themselves, e.g. on two GPUs):
+ *   x[b] = [text[b]; bf16(z[b])]
+ * z: fp32 [batch, n_img, d_model]; text: bf16 [batch, n_text, d_model] (NULL when n_text = 0);
+ * x: bf16 [batch, n_text + n_img, d_model].  d_model % 8 == 0. */
+DIT_API int dit_tokens_from_latent(const float* z, const void* text, void* x, int batch, int n_text, int n_img,
+                                   int d_model, void* stream);
 
 /* Size of the fixed device scratch behind dit_block_forward_noalloc (32 MiB).  Every GPU
  * that loads this library holds this much device memory until the process exits. */
@@ -184,6 +251,20 @@ DIT_API int dit_gemm_w8a16(const void* a, int a_fmt, const uint8_t* w8, const fl
                            const void* residual, int res_fmt, int M, int N, int K, int act, int gelu_tanh,
                            void* stream);
 
+/* Y[M, N] = act( A8[M, K] (W8[N, K])^T * sa[m] * sw[n] ): e4m3 activations with a per-row fp32
+ * scale sa [M] and e4m3 weights with their per-row weight_scale sw [N], both row-major; Y in y_fmt
+ * (BF16/F16/F32); act 0 = none, 1 = GELU (gelu_tanh selects the form).  fp32 accumulation.
+ * N % 32 == 0, K % 16 == 0. */
+DIT_API int dit_gemm_w8a8(const uint8_t* a8, const float* sa, const uint8_t* w8, const float* sw, void* y, int y_fmt,
+                          int M, int N, int K, int act, int gelu_tanh, void* stream);
+
+/* Row RMSNorm to per-token e4m3: o = x / sqrt(mean(x^2) + eps) * g (fp32), s = amax|o| / 448
+ * (1 for a zero row), y8 = e4m3(o / s) rounded to nearest even; y_scale[row] = s.
+ * x: [rows, cols] in x_fmt (BF16 or F32); g: bf16 [cols]; y8: bytes [rows, cols]; y_scale: fp32
+ * [rows].  cols % 8 == 0, cols <= 8192. */
+DIT_API int dit_rmsnorm_rows_e4m3(const void* x, int x_fmt, const void* g, uint8_t* y8, float* y_scale, int64_t rows,
+                                  int64_t cols, float eps, void* stream);
+
 /* Per-head QK-RMSNorm + 3D M-RoPE, in place on a fused qkv buffer [batch, S, 3d] in fmt
  * (BF16 or F16; Q columns [0, d), K columns [d, 2d); V untouched).  pos: int32 [S, 3] or
  * NULL (derived from n_text/grid/t_img as in dit_block_forward).  workspace holds the
@@ -244,6 +325,9 @@ DIT_API int dit_wait_selftest(void* stream);
 DIT_API int dit_set_wait_timeout_ms(uint32_t ms);
 
 DIT_API const char* dit_status_str(int status);
+
+/* The cudaError_t code behind the last DIT_ERR_CUDA status returned on any thread (0 if none). */
+DIT_API int dit_last_cuda_error(void);
 
 /* ABI version of this header (bumped on any signature change). */
 DIT_API int dit_abi_version(void);

@@ -32,7 +32,10 @@ STATUS_NAMES = {
 class DitError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} ({lib().dit_status_str(status).decode()})")
+        msg = f"{fn} failed: {STATUS_NAMES.get(status, status)} ({lib().dit_status_str(status).decode()})"
+        if status == 4:
+            msg += f", cudaError {lib().dit_last_cuda_error()}"
+        super().__init__(msg)
 
 
 class BlockConfig(ctypes.Structure):
@@ -65,11 +68,22 @@ SIGNATURES = {
     "dit_block_workspace_bytes": (_SZ, [ctypes.POINTER(BlockConfig), _I, _I, _I, _I]),
     "dit_block_forward": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I, _I, _I, _I,
                                _P, _P, _SZ, _P]),
+    "dit_block_forward_padded": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I, _I,
+                                      _I, _I, _P, _P, _SZ, _P]),
+    "dit_block_forward_w8a8": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I, _I, _I,
+                                    _I, _P, _P, _SZ, _P]),
+    "dit_gemm_w8a8": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "dit_rmsnorm_rows_e4m3": (_I, [_P, _I, _P, _P, _P, _I64, _I64, _F, _P]),
     "dit_block_forward_noalloc": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _P, _P, _I, _I,
                                        _I, _I, _I, _P, _P]),
     "dit_stack_workspace_bytes": (_SZ, [ctypes.POINTER(BlockConfig), _I, _I, _I, _I]),
     "dit_stack_forward": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), _I, _P, _P, _I, _I, _I, _I,
                                _I, _P, _P, _SZ, _P]),
+    "dit_denoise_workspace_bytes": (_SZ, [ctypes.POINTER(BlockConfig), _I, _I, _I, _I, _I]),
+    "dit_denoise_steps": (_I, [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockWeights),
+                               _I, _P, _I, _P, _I, _P, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float),
+                               ctypes.POINTER(ctypes.c_float), _P, _SZ, _P]),
+    "dit_tokens_from_latent": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "cond_proj_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "cond_proj_forward": (_I, [_P, _I, _I, _I, _P, _F, _P, _P, _I, _P, _P, _SZ, _P]),
     "euler_cfg_step": (_I, [_P, _P, _P, _I64, _F, _F, _P]),
@@ -87,6 +101,7 @@ SIGNATURES = {
     "dit_last_device_error": (ctypes.c_uint32, []),
     "dit_wait_selftest": (_I, [_P]),
     "dit_status_str": (ctypes.c_char_p, [_I]),
+    "dit_last_cuda_error": (_I, []),
     "dit_abi_version": (_I, []),
 }
 
@@ -170,6 +185,42 @@ def dit_block_forward(cfg: BlockConfig, weights: BlockWeights, x: torch.Tensor, 
         _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def dit_block_forward_padded(cfg: BlockConfig, weights: BlockWeights, x: torch.Tensor, out: torch.Tensor,
+                             n_text: int, grid_h: int, grid_w: int, text_lens: torch.Tensor, workspace: torch.Tensor,
+                             t_img: int = -1, stream=None) -> None:
+    """Padded batch of prompts: element b has text_lens[b] text rows, then its image rows, then
+    padding (``text_lens``: int32 device tensor [batch])."""
+    if text_lens.dtype != torch.int32 or text_lens.numel() != x.shape[0]:
+        raise ValueError("text_lens must be an int32 tensor with one entry per batch element")
+    _check("dit_block_forward_padded", lib().dit_block_forward_padded(
+        ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
+        _ptr(text_lens), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dit_block_forward_w8a8(cfg: BlockConfig, weights: BlockWeights, x: torch.Tensor, out: torch.Tensor, n_text: int,
+                           grid_h: int, grid_w: int, workspace: torch.Tensor, t_img: int = -1,
+                           pos: Optional[torch.Tensor] = None, stream=None) -> None:
+    """The W8A8 variant: e4m3 per-token activations into the QKV and MLP-up projections."""
+    _check("dit_block_forward_w8a8", lib().dit_block_forward_w8a8(
+        ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
+        _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gemm_w8a8(a8: torch.Tensor, sa: torch.Tensor, w8: torch.Tensor, sw: torch.Tensor, y: torch.Tensor, act: int = 0,
+              gelu_tanh: int = 0, y_fmt: int = FMT_BF16, stream=None) -> None:
+    M, K = a8.shape
+    N = w8.shape[0]
+    _check("dit_gemm_w8a8", lib().dit_gemm_w8a8(_ptr(a8), _ptr(sa), _ptr(w8), _ptr(sw), _ptr(y), y_fmt, M, N, K, act,
+                                                gelu_tanh, _stream(stream)))
+
+
+def rmsnorm_rows_e4m3(x: torch.Tensor, g: torch.Tensor, y8: torch.Tensor, y_scale: torch.Tensor, eps: float,
+                      x_fmt: int = FMT_BF16, stream=None) -> None:
+    cols = x.shape[-1]
+    _check("dit_rmsnorm_rows_e4m3", lib().dit_rmsnorm_rows_e4m3(_ptr(x), x_fmt, _ptr(g), _ptr(y8), _ptr(y_scale),
+                                                                x.numel() // cols, cols, eps, _stream(stream)))
+
+
 def stack_workspace_bytes(cfg: BlockConfig, batch: int, n_text: int, grid_h: int, grid_w: int) -> int:
     return int(lib().dit_stack_workspace_bytes(ctypes.byref(cfg), batch, n_text, grid_h, grid_w))
 
@@ -182,6 +233,38 @@ def dit_stack_forward(cfg: BlockConfig, weights, x: torch.Tensor, out: torch.Ten
     _check("dit_stack_forward", lib().dit_stack_forward(
         ctypes.byref(cfg), arr, len(weights), _ptr(x), _ptr(out), x.shape[0], n_text, grid_h, grid_w, t_img,
         _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def denoise_workspace_bytes(cfg: BlockConfig, batch: int, n_text_c: int, n_text_u: int, grid_h: int,
+                            grid_w: int) -> int:
+    return int(lib().dit_denoise_workspace_bytes(ctypes.byref(cfg), batch, n_text_c, n_text_u, grid_h, grid_w))
+
+
+def dit_denoise_steps(cfg: BlockConfig, w_cond, w_uncond, text_cond: Optional[torch.Tensor],
+                      text_uncond: Optional[torch.Tensor], z: torch.Tensor, grid_h: int, grid_w: int, guidance,
+                      dt, workspace: torch.Tensor, stream=None) -> None:
+    """len(guidance) denoising steps: ``w_cond``/``w_uncond`` are equal-length sequences of
+    BlockWeights; text tensors are bf16 [batch, L, d] (or None for L = 0); z fp32 [batch, gh*gw, d]
+    is updated in place; ``guidance`` and ``dt`` hold one value per step."""
+    if len(w_cond) != len(w_uncond) or len(guidance) != len(dt):
+        raise ValueError("w_cond/w_uncond and guidance/dt must have equal lengths")
+    n = len(w_cond)
+    wc = (BlockWeights * n)(*w_cond)
+    wu = (BlockWeights * n)(*w_uncond)
+    g = (ctypes.c_float * max(1, len(guidance)))(*[float(v) for v in guidance])
+    t = (ctypes.c_float * max(1, len(dt)))(*[float(v) for v in dt])
+    lc = 0 if text_cond is None else text_cond.shape[1]
+    lu = 0 if text_uncond is None else text_uncond.shape[1]
+    _check("dit_denoise_steps", lib().dit_denoise_steps(
+        ctypes.byref(cfg), wc, wu, n, _ptr(text_cond), lc, _ptr(text_uncond), lu, _ptr(z), z.shape[0], grid_h,
+        grid_w, len(guidance), g, t, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def tokens_from_latent(z: torch.Tensor, text: Optional[torch.Tensor], x: torch.Tensor, stream=None) -> None:
+    """x[b] = [text[b]; bf16(z[b])]: z fp32 [B, n_img, d], text bf16 [B, L, d] or None, x bf16 [B, L + n_img, d]."""
+    n_text = 0 if text is None else text.shape[1]
+    _check("dit_tokens_from_latent", lib().dit_tokens_from_latent(
+        _ptr(z), _ptr(text), _ptr(x), z.shape[0], n_text, z.shape[1], z.shape[2], _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # DIT_NOALLOC_SCRATCH_BYTES

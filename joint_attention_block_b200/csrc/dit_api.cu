@@ -106,7 +106,17 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA; }
+std::atomic<int> g_last_cuda_error{0};
+
+int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return DIT_OK;
+  g_last_cuda_error.store(static_cast<int>(e));
+  return DIT_ERR_CUDA;
+}
+
+// A launch error is reported once by the next cudaGetLastError() of the thread; clear any that an
+// earlier, unrelated call left behind so that it is not reported as this call's failure.
+void clear_stale_error() { (void)cudaGetLastError(); }
 
 int check_config(const dit_block_config* c) {
   if (c == nullptr) return DIT_ERR_INVALID_ARG;
@@ -121,14 +131,18 @@ int check_config(const dit_block_config* c) {
 
 // Internal activations: h, qkv, o, u in f16 (every one is bounded: post-norm,
 // softmax-weighted or a GEMM of bounded inputs); the residual x1 in fp32.
+// The rotary tables hold one [S, hd/2] pair per batch element (padded batches position each
+// element on its own; otherwise only the first is used) and kv_len the per-element key counts.
 struct BlockWorkspace {
   float* cos_tab;
   float* sin_tab;
+  int32_t* kv_len;
   uint16_t* h;
   uint16_t* qkv;
   uint16_t* o;
   float* x1;
   uint16_t* u;
+  float* sa;  // per-token e4m3 scales of the W8A8 variant (its e4m3 codes reuse h)
   size_t bytes;
 };
 
@@ -142,19 +156,21 @@ BlockWorkspace carve_block(const dit_block_config* c, int batch, int seq, void* 
     off += align256(bytes);
     return o;
   };
-  const size_t o_cos = take(seq * half * 4), o_sin = take(seq * half * 4);
+  const size_t o_cos = take(M * half * 4), o_sin = take(M * half * 4), o_kv = take(static_cast<size_t>(batch) * 4);
   const size_t o_h = take(M * d * 2), o_qkv = take(M * 3 * d * 2), o_o = take(M * d * 2), o_x1 = take(M * d * 4);
-  const size_t o_u = take(M * F * 2);
+  const size_t o_u = take(M * F * 2), o_sa = take(M * 4);
   w.bytes = off;
   if (base != nullptr) {
     uint8_t* b = static_cast<uint8_t*>(base);
     w.cos_tab = reinterpret_cast<float*>(b + o_cos);
     w.sin_tab = reinterpret_cast<float*>(b + o_sin);
+    w.kv_len = reinterpret_cast<int32_t*>(b + o_kv);
     w.h = reinterpret_cast<uint16_t*>(b + o_h);
     w.qkv = reinterpret_cast<uint16_t*>(b + o_qkv);
     w.o = reinterpret_cast<uint16_t*>(b + o_o);
     w.x1 = reinterpret_cast<float*>(b + o_x1);
     w.u = reinterpret_cast<uint16_t*>(b + o_u);
+    w.sa = reinterpret_cast<float*>(b + o_sa);
   }
   return w;
 }
@@ -169,7 +185,9 @@ bool shape_ok(int batch, int n_text, int grid_h, int grid_w) {
 
 extern "C" {
 
-int dit_abi_version(void) { return 1; }
+int dit_abi_version(void) { return 2; }
+
+int dit_last_cuda_error(void) { return g_last_cuda_error.load(); }
 
 int dit_profile_enable(int max_marks) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -252,12 +270,14 @@ int dit_poll_error(void* stream) {
 }
 
 int dit_wait_selftest(void* stream) {
+  clear_stale_error();
   KernelGuard g;
   if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
   return from_cuda(launch_wait_selftest(g, as_stream(stream)));
 }
 
 int dit_e4m3_to_bf16(const uint8_t* codes, void* out, int64_t n, void* stream) {
+  clear_stale_error();
   if (n < 0 || (n > 0 && (codes == nullptr || out == nullptr))) return DIT_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(out)) return DIT_ERR_INVALID_ARG;
   return from_cuda(launch_e4m3_to_bf16(codes, static_cast<uint16_t*>(out), n, as_stream(stream)));
@@ -265,6 +285,7 @@ int dit_e4m3_to_bf16(const uint8_t* codes, void* out, int64_t n, void* stream) {
 
 int dit_rmsnorm_rows(const void* x, int x_fmt, const void* g, void* y, int y_fmt, int64_t rows, int64_t cols,
                      float eps, void* stream) {
+  clear_stale_error();
   if (rows < 0 || cols <= 0 || cols % 8 != 0 || rows > (1ll << 31) - 1) return DIT_ERR_INVALID_ARG;
   if ((x_fmt != FMT_BF16 && x_fmt != FMT_F32) || (y_fmt != FMT_BF16 && y_fmt != FMT_F16)) return DIT_ERR_INVALID_ARG;
   if (rows > 0 && (x == nullptr || g == nullptr || y == nullptr)) return DIT_ERR_INVALID_ARG;
@@ -279,6 +300,7 @@ int dit_rmsnorm_rows(const void* x, int x_fmt, const void* g, void* y, int y_fmt
 
 int euler_cfg_step(float* x, const void* v_cond, const void* v_uncond, int64_t n, float guidance, float dt,
                    void* stream) {
+  clear_stale_error();
   if (n < 0 || (n > 0 && (x == nullptr || v_cond == nullptr || v_uncond == nullptr))) return DIT_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(v_cond) || !aligned16(v_uncond)) return DIT_ERR_INVALID_ARG;
   prof_mark(as_stream(stream), DIT_KERNEL_EULER_CFG);
@@ -289,6 +311,7 @@ int euler_cfg_step(float* x, const void* v_cond, const void* v_uncond, int64_t n
 }
 
 int dit_mrope_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos_out, void* stream) {
+  clear_stale_error();
   if (!shape_ok(1, n_text, grid_h, grid_w) || pos_out == nullptr) return DIT_ERR_INVALID_ARG;
   if (t_img < 0) t_img = n_text;
   return from_cuda(launch_positions(n_text, grid_h, grid_w, t_img, pos_out, as_stream(stream)));
@@ -296,6 +319,7 @@ int dit_mrope_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* 
 
 int dit_gemm_w8a16(const void* a, int a_fmt, const uint8_t* w8, const float* scale, void* y, int y_fmt,
                    const void* residual, int res_fmt, int M, int N, int K, int act, int gelu_tanh, void* stream) {
+  clear_stale_error();
   if (M < 0 || N <= 0 || K <= 0) return DIT_ERR_INVALID_ARG;
   if (N % 32 != 0 || K % 16 != 0) return DIT_ERR_UNSUPPORTED;
   if ((a_fmt != FMT_BF16 && a_fmt != FMT_F16) || y_fmt < FMT_BF16 || y_fmt > FMT_F32) return DIT_ERR_INVALID_ARG;
@@ -313,6 +337,7 @@ int dit_gemm_w8a16(const void* a, int a_fmt, const uint8_t* w8, const float* sca
 int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                      const dit_block_config* cfg, const void* g_q, const void* g_k, void* workspace, size_t ws_bytes,
                      void* stream) {
+  clear_stale_error();
   int st = check_config(cfg);
   if (st != DIT_OK) return st;
   if (!shape_ok(batch, n_text, grid_h, grid_w) || qkv == nullptr || g_q == nullptr || g_k == nullptr)
@@ -330,20 +355,21 @@ int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int 
   if (e != cudaSuccess) return DIT_ERR_CUDA;
   prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
   e = launch_qknorm_mrope(qkv, fmt, batch, S, cfg->n_heads, cfg->head_dim, cos_tab, sin_tab,
-                          static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k), cfg->eps, s);
+                          static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k), cfg->eps, false, s);
   prof_mark(s, DIT_KERNEL_END);
   return from_cuda(e);
 }
 
 int dit_joint_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
                         void* stream) {
+  clear_stale_error();
   if (batch <= 0 || seq <= 0 || n_heads <= 0 || qkv == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
   if (fmt != FMT_BF16 && fmt != FMT_F16) return DIT_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return DIT_ERR_UNSUPPORTED;
   if (!aligned16(qkv) || !aligned16(out)) return DIT_ERR_INVALID_ARG;
   KernelGuard g;
   if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
-  return from_cuda(launch_attention(qkv, out, fmt, batch, seq, n_heads, head_dim, g, as_stream(stream)));
+  return from_cuda(launch_attention(qkv, out, fmt, batch, seq, n_heads, head_dim, nullptr, g, as_stream(stream)));
 }
 
 size_t dit_block_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w) {
@@ -351,9 +377,15 @@ size_t dit_block_workspace_bytes(const dit_block_config* cfg, int batch, int n_t
   return carve_block(cfg, batch, n_text + grid_h * grid_w, nullptr).bytes;
 }
 
-int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in, void* x_out,
-                      int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, void* workspace,
-                      size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The block forward behind dit_block_forward (text_lens == nullptr) and dit_block_forward_padded.
+int block_forward(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in, void* x_out, int batch,
+                  int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, const int32_t* text_lens,
+                  void* workspace, size_t ws_bytes, void* stream, bool w8a8 = false) {
+  clear_stale_error();
   int st = check_config(cfg);
   if (st != DIT_OK) return st;
   if (w == nullptr || x_in == nullptr || x_out == nullptr || x_in == x_out) return DIT_ERR_INVALID_ARG;
@@ -378,39 +410,113 @@ int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, c
   const uint16_t* x = static_cast<const uint16_t*>(x_in);
   uint16_t* y = static_cast<uint16_t*>(x_out);
 
-#define JAB_TRY(expr)                               \
-  do {                                              \
-    if ((expr) != cudaSuccess) return DIT_ERR_CUDA; \
+#define JAB_TRY(expr)                         \
+  do {                                        \
+    const cudaError_t jab_e = (expr);         \
+    if (jab_e != cudaSuccess) return from_cuda(jab_e); \
   } while (0)
+  const bool padded = text_lens != nullptr;
   prof_mark(s, DIT_KERNEL_ROPE_TABLE);
-  JAB_TRY(launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections, cfg->rope_theta,
-                            ws.cos_tab, ws.sin_tab, s));
+  if (padded)
+    JAB_TRY(launch_rope_table_padded(batch, n_text, grid_h, grid_w, t_img, text_lens, cfg->head_dim,
+                                     cfg->rope_sections, cfg->rope_theta, ws.cos_tab, ws.sin_tab, ws.kv_len, s));
+  else
+    JAB_TRY(launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections,
+                              cfg->rope_theta, ws.cos_tab, ws.sin_tab, s));
   const uint16_t* g1 = static_cast<const uint16_t*>(w->g_norm1);
   const uint16_t* g2 = static_cast<const uint16_t*>(w->g_norm2);
+  uint8_t* h8 = reinterpret_cast<uint8_t*>(ws.h);  // e4m3 codes of the W8A8 variant
   prof_mark(s, DIT_KERNEL_RMSNORM);
-  JAB_TRY(launch_rmsnorm(x, FMT_BF16, g1, ws.h, FMT_F16, M, d, cfg->eps, s));
+  if (w8a8)
+    JAB_TRY(launch_rmsnorm_e4m3(x, FMT_BF16, g1, h8, ws.sa, M, d, cfg->eps, s));
+  else
+    JAB_TRY(launch_rmsnorm(x, FMT_BF16, g1, ws.h, FMT_F16, M, d, cfg->eps, s));
   prof_mark(s, DIT_KERNEL_GEMM_QKV);
-  JAB_TRY(launch_gemm_w8a16(
-      GemmArgs{ws.h, FMT_F16, w->w_qkv, w->s_qkv, ws.qkv, FMT_F16, nullptr, -1, M, 3 * d, d, 0, 0}, g, s));
+  if (w8a8)
+    JAB_TRY(launch_gemm_w8a8(GemmArgs8{h8, ws.sa, w->w_qkv, w->s_qkv, ws.qkv, FMT_F16, M, 3 * d, d, 0, 0}, g, s));
+  else
+    JAB_TRY(launch_gemm_w8a16(
+        GemmArgs{ws.h, FMT_F16, w->w_qkv, w->s_qkv, ws.qkv, FMT_F16, nullptr, -1, M, 3 * d, d, 0, 0}, g, s));
   prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
   JAB_TRY(launch_qknorm_mrope(ws.qkv, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, ws.cos_tab, ws.sin_tab,
                               static_cast<const uint16_t*>(w->g_q), static_cast<const uint16_t*>(w->g_k), cfg->eps,
-                              s));
+                              padded, s));
   prof_mark(s, DIT_KERNEL_ATTENTION);
-  JAB_TRY(launch_attention(ws.qkv, ws.o, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, g, s));
+  JAB_TRY(launch_attention(ws.qkv, ws.o, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, padded ? ws.kv_len : nullptr,
+                           g, s));
   prof_mark(s, DIT_KERNEL_GEMM_O);
   JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.o, FMT_F16, w->w_o, w->s_o, ws.x1, FMT_F32, x, FMT_BF16, M, d, d, 0, 0}, g, s));
   prof_mark(s, DIT_KERNEL_RMSNORM);
-  JAB_TRY(launch_rmsnorm(ws.x1, FMT_F32, g2, ws.h, FMT_F16, M, d, cfg->eps, s));
+  if (w8a8)
+    JAB_TRY(launch_rmsnorm_e4m3(ws.x1, FMT_F32, g2, h8, ws.sa, M, d, cfg->eps, s));
+  else
+    JAB_TRY(launch_rmsnorm(ws.x1, FMT_F32, g2, ws.h, FMT_F16, M, d, cfg->eps, s));
   prof_mark(s, DIT_KERNEL_GEMM_UP);
-  JAB_TRY(launch_gemm_w8a16(
-      GemmArgs{ws.h, FMT_F16, w->w_up, w->s_up, ws.u, FMT_F16, nullptr, -1, M, F, d, 1, cfg->gelu_tanh}, g, s));
+  if (w8a8)
+    JAB_TRY(launch_gemm_w8a8(GemmArgs8{h8, ws.sa, w->w_up, w->s_up, ws.u, FMT_F16, M, F, d, 1, cfg->gelu_tanh}, g, s));
+  else
+    JAB_TRY(launch_gemm_w8a16(
+        GemmArgs{ws.h, FMT_F16, w->w_up, w->s_up, ws.u, FMT_F16, nullptr, -1, M, F, d, 1, cfg->gelu_tanh}, g, s));
   prof_mark(s, DIT_KERNEL_GEMM_DOWN);
   JAB_TRY(launch_gemm_w8a16(
       GemmArgs{ws.u, FMT_F16, w->w_down, w->s_down, y, FMT_BF16, ws.x1, FMT_F32, M, d, F, 0, 0}, g, s));
   prof_mark(s, DIT_KERNEL_END);
 #undef JAB_TRY
   return DIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dit_block_forward(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in, void* x_out,
+                      int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  return block_forward(cfg, w, x_in, x_out, batch, n_text, grid_h, grid_w, t_img, pos, nullptr, workspace, ws_bytes,
+                       stream);
+}
+
+int dit_block_forward_w8a8(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in, void* x_out,
+                           int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  if (cfg != nullptr && cfg->d_model > 8192) return DIT_ERR_UNSUPPORTED;  // the e4m3 norm holds a row in registers
+  return block_forward(cfg, w, x_in, x_out, batch, n_text, grid_h, grid_w, t_img, pos, nullptr, workspace, ws_bytes,
+                       stream, true);
+}
+
+int dit_gemm_w8a8(const uint8_t* a8, const float* sa, const uint8_t* w8, const float* sw, void* y, int y_fmt, int M,
+                  int N, int K, int act, int gelu_tanh, void* stream) {
+  clear_stale_error();
+  if (M < 0 || N <= 0 || K <= 0) return DIT_ERR_INVALID_ARG;
+  if (N % 32 != 0 || K % 16 != 0) return DIT_ERR_UNSUPPORTED;
+  if (y_fmt < FMT_BF16 || y_fmt > FMT_F32 || act < 0 || act > 1) return DIT_ERR_INVALID_ARG;
+  if (M == 0) return DIT_OK;
+  if (a8 == nullptr || sa == nullptr || w8 == nullptr || sw == nullptr || y == nullptr) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(a8) || !aligned16(w8) || !aligned16(y)) return DIT_ERR_INVALID_ARG;
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  return from_cuda(launch_gemm_w8a8(GemmArgs8{a8, sa, w8, sw, y, y_fmt, M, N, K, act, gelu_tanh}, g,
+                                    as_stream(stream)));
+}
+
+int dit_rmsnorm_rows_e4m3(const void* x, int x_fmt, const void* g, uint8_t* y8, float* y_scale, int64_t rows,
+                          int64_t cols, float eps, void* stream) {
+  clear_stale_error();
+  if (rows < 0 || cols <= 0 || cols % 8 != 0 || rows > (1ll << 31) - 1) return DIT_ERR_INVALID_ARG;
+  if (cols > 8192) return DIT_ERR_UNSUPPORTED;
+  if (x_fmt != FMT_BF16 && x_fmt != FMT_F32) return DIT_ERR_INVALID_ARG;
+  if (rows > 0 && (x == nullptr || g == nullptr || y8 == nullptr || y_scale == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(g) || !aligned16(y8)) return DIT_ERR_INVALID_ARG;
+  return from_cuda(launch_rmsnorm_e4m3(x, x_fmt, static_cast<const uint16_t*>(g), y8, y_scale, rows, cols, eps,
+                                       as_stream(stream)));
+}
+
+int dit_block_forward_padded(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in, void* x_out,
+                             int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* text_lens,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  if (text_lens == nullptr || !aligned16(text_lens)) return DIT_ERR_INVALID_ARG;
+  return block_forward(cfg, w, x_in, x_out, batch, n_text, grid_h, grid_w, t_img, nullptr, text_lens, workspace,
+                       ws_bytes, stream);
 }
 
 size_t dit_stack_workspace_bytes(const dit_block_config* cfg, int batch, int n_text, int grid_h, int grid_w) {
@@ -457,6 +563,7 @@ size_t cond_proj_workspace_bytes(int n_tok, int n_layers, int hidden, int d_out)
 int cond_proj_forward(const void* feats, int n_tok, int n_layers, int hidden, const void* g_norm, float eps,
                       const uint8_t* w, const float* scale, int d_out, void* out, void* workspace, size_t ws_bytes,
                       void* stream) {
+  clear_stale_error();
   if (n_tok <= 0 || n_layers <= 0 || hidden <= 0 || d_out <= 0) return DIT_ERR_INVALID_ARG;
   const int64_t K = static_cast<int64_t>(n_layers) * hidden;
   if (K % 256 != 0 || d_out % 256 != 0 || K > (1 << 30)) return DIT_ERR_UNSUPPORTED;
@@ -494,6 +601,75 @@ int cond_proj_forward(const void* feats, int n_tok, int n_layers, int hidden, co
   }
   prof_mark(s, DIT_KERNEL_END);
   return from_cuda(e);
+}
+
+
+size_t dit_denoise_workspace_bytes(const dit_block_config* cfg, int batch, int n_text_c, int n_text_u, int grid_h,
+                                   int grid_w) {
+  const size_t sc = dit_stack_workspace_bytes(cfg, batch, n_text_c, grid_h, grid_w);
+  const size_t su = dit_stack_workspace_bytes(cfg, batch, n_text_u, grid_h, grid_w);
+  if (sc == 0 || su == 0 || grid_h * grid_w <= 0) return 0;
+  const size_t n_img = static_cast<size_t>(grid_h) * grid_w;
+  const size_t xc = align256(static_cast<size_t>(batch) * (n_text_c + n_img) * cfg->d_model * 2);
+  const size_t xu = align256(static_cast<size_t>(batch) * (n_text_u + n_img) * cfg->d_model * 2);
+  return 2 * xc + 2 * xu + (sc > su ? sc : su);
+}
+
+int dit_denoise_steps(const dit_block_config* cfg, const dit_block_weights* w_cond, const dit_block_weights* w_uncond,
+                      int n_blocks, const void* text_cond, int n_text_c, const void* text_uncond, int n_text_u,
+                      float* z, int batch, int grid_h, int grid_w, int n_steps, const float* guidance, const float* dt,
+                      void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_config(cfg);
+  if (st != DIT_OK) return st;
+  if (w_cond == nullptr || w_uncond == nullptr || n_blocks < 1 || z == nullptr || n_steps < 0) return DIT_ERR_INVALID_ARG;
+  if (n_steps > 0 && (guidance == nullptr || dt == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (grid_h <= 0 || grid_w <= 0 || n_text_c < 0 || n_text_u < 0) return DIT_ERR_INVALID_ARG;
+  if ((n_text_c > 0 && text_cond == nullptr) || (n_text_u > 0 && text_uncond == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (!shape_ok(batch, n_text_c, grid_h, grid_w) || !shape_ok(batch, n_text_u, grid_h, grid_w))
+    return DIT_ERR_INVALID_ARG;
+  if (!aligned16(z) || !aligned16(text_cond) || !aligned16(text_uncond)) return DIT_ERR_INVALID_ARG;
+  const size_t need = dit_denoise_workspace_bytes(cfg, batch, n_text_c, n_text_u, grid_h, grid_w);
+  if (need == 0) return DIT_ERR_UNSUPPORTED;
+  if (workspace == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return DIT_ERR_WORKSPACE;
+  const int d = cfg->d_model, n_img = grid_h * grid_w;
+  const size_t xc = align256(static_cast<size_t>(batch) * (n_text_c + n_img) * d * 2);
+  const size_t xu = align256(static_cast<size_t>(batch) * (n_text_u + n_img) * d * 2);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint16_t* x_c = reinterpret_cast<uint16_t*>(base);
+  uint16_t* out_c = reinterpret_cast<uint16_t*>(base + xc);
+  uint16_t* x_u = reinterpret_cast<uint16_t*>(base + 2 * xc);
+  uint16_t* out_u = reinterpret_cast<uint16_t*>(base + 2 * xc + xu);
+  void* stack_ws = base + 2 * xc + 2 * xu;
+  const size_t stack_bytes = ws_bytes - (2 * xc + 2 * xu);
+  cudaStream_t s = as_stream(stream);
+  for (int i = 0; i < n_steps; ++i) {
+    if (launch_denoise_pack(z, static_cast<const uint16_t*>(text_cond), static_cast<const uint16_t*>(text_uncond), x_c,
+                            x_u, batch, n_img, d, n_text_c, n_text_u, s) != cudaSuccess)
+      return DIT_ERR_CUDA;
+    st = dit_stack_forward(cfg, w_cond, n_blocks, x_c, out_c, batch, n_text_c, grid_h, grid_w, -1, nullptr, stack_ws,
+                           stack_bytes, stream);
+    if (st != DIT_OK) return st;
+    st = dit_stack_forward(cfg, w_uncond, n_blocks, x_u, out_u, batch, n_text_u, grid_h, grid_w, -1, nullptr, stack_ws,
+                           stack_bytes, stream);
+    if (st != DIT_OK) return st;
+    prof_mark(s, DIT_KERNEL_EULER_CFG);
+    const cudaError_t e = launch_denoise_update(z, out_c, out_u, batch, n_img, d, n_text_c, n_text_u, guidance[i],
+                                                dt[i], s);
+    prof_mark(s, DIT_KERNEL_END);
+    if (e != cudaSuccess) return DIT_ERR_CUDA;
+  }
+  return DIT_OK;
+}
+
+int dit_tokens_from_latent(const float* z, const void* text, void* x, int batch, int n_text, int n_img, int d_model,
+                           void* stream) {
+  clear_stale_error();
+  if (batch <= 0 || n_text < 0 || n_img <= 0 || d_model <= 0 || d_model % 8 != 0) return DIT_ERR_INVALID_ARG;
+  if (z == nullptr || x == nullptr || (n_text > 0 && text == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(z) || !aligned16(text) || !aligned16(x)) return DIT_ERR_INVALID_ARG;
+  return from_cuda(launch_denoise_pack(z, static_cast<const uint16_t*>(text), nullptr, static_cast<uint16_t*>(x),
+                                       nullptr, batch, n_img, d_model, n_text, 0, as_stream(stream)));
 }
 
 }  // extern "C"

@@ -141,6 +141,113 @@ cudaError_t launch_rmsnorm(const void* x, int x_fmt, const uint16_t* g, void* y,
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ RMSNorm to per-token e4m3
+
+template <int kThreads>
+__device__ float block_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (threadIdx.x < 32) {
+    t = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, o));
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+// Two fp32 -> packed e4m3x2 (round to nearest even, saturating at +-448), lo in the low byte.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// One CTA per row, the row held in registers: o = x / sqrt(mean(x^2) + eps) * g in fp32, then
+// the row's scale s = amax(|o|) / 448 and codes e4m3(o / s) (IEEE division, then round to nearest
+// even).  The scale goes to ys[row].
+template <int kThreads, int kVec, int XF>
+__global__ void __launch_bounds__(kThreads) rmsnorm_e4m3_kernel(const void* x, const uint16_t* __restrict__ g,
+                                                                uint8_t* __restrict__ y8, float* __restrict__ ys,
+                                                                int64_t cols, float eps) {
+  pdl_wait_then_release();
+  __shared__ float red[32];
+  __shared__ float red2[32];
+  const int64_t row = blockIdx.x;
+  const int64_t nv = cols / 8;
+  float v[kVec][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    const int64_t i = threadIdx.x + static_cast<int64_t>(j) * kThreads;
+    if (i < nv) {
+      load8<XF>(x, row * nv + i, v[j]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ss = fmaf(v[j][k], v[j][k], ss);
+  }
+  const float rstd = rsqrtf(block_sum<kThreads>(ss, red) / static_cast<float>(cols) + eps);
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    const int64_t i = threadIdx.x + static_cast<int64_t>(j) * kThreads;
+    float gv[8];
+    if (i < nv) {
+      load8<FMT_BF16>(g, i, gv);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) gv[k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v[j][k] = v[j][k] * rstd * gv[k];
+      amax = fmaxf(amax, fabsf(v[j][k]));
+    }
+  }
+  amax = block_max<kThreads>(amax, red2);
+  const float scale = amax > 0.f ? amax / 448.f : 1.f;
+  if (threadIdx.x == 0) ys[row] = scale;
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    const int64_t i = threadIdx.x + static_cast<int64_t>(j) * kThreads;
+    if (i >= nv) break;
+    uint2 o;
+    o.x = static_cast<uint32_t>(pack_e4m3x2(v[j][0] / scale, v[j][1] / scale)) |
+          (static_cast<uint32_t>(pack_e4m3x2(v[j][2] / scale, v[j][3] / scale)) << 16);
+    o.y = static_cast<uint32_t>(pack_e4m3x2(v[j][4] / scale, v[j][5] / scale)) |
+          (static_cast<uint32_t>(pack_e4m3x2(v[j][6] / scale, v[j][7] / scale)) << 16);
+    reinterpret_cast<uint2*>(y8)[row * nv + i] = o;
+  }
+}
+
+template <int XF>
+static void rmsnorm_e4m3_dispatch(const void* x, const uint16_t* g, uint8_t* y8, float* ys, int64_t rows,
+                                  int64_t cols, float eps, cudaStream_t s) {
+  const unsigned r = static_cast<unsigned>(rows);
+  if (cols <= 256 * 8 * 1)
+    launch_pdl(rmsnorm_e4m3_kernel<256, 1, XF>, dim3(r), dim3(256), 0, s, x, g, y8, ys, cols, eps);
+  else if (cols <= 256 * 8 * 2)
+    launch_pdl(rmsnorm_e4m3_kernel<256, 2, XF>, dim3(r), dim3(256), 0, s, x, g, y8, ys, cols, eps);
+  else
+    launch_pdl(rmsnorm_e4m3_kernel<256, 4, XF>, dim3(r), dim3(256), 0, s, x, g, y8, ys, cols, eps);
+}
+
+cudaError_t launch_rmsnorm_e4m3(const void* x, int x_fmt, const uint16_t* g, uint8_t* y8, float* ys, int64_t rows,
+                                int64_t cols, float eps, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (cols % 8 != 0 || cols > 256 * 8 * 4) return cudaErrorInvalidValue;
+  if (x_fmt == FMT_BF16) rmsnorm_e4m3_dispatch<FMT_BF16>(x, g, y8, ys, rows, cols, eps, s);
+  else if (x_fmt == FMT_F32) rmsnorm_e4m3_dispatch<FMT_F32>(x, g, y8, ys, rows, cols, eps, s);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ CFG + Euler
 
 // x <- x + dt * (v_u + g * (v_c - v_u)); 8 elements per thread per iteration.
@@ -185,6 +292,83 @@ cudaError_t launch_euler_cfg(float* x, const uint16_t* vc, const uint16_t* vu, i
   if (blocks < 1) blocks = 1;
   if (blocks > 148 * 8) blocks = 148 * 8;
   launch_pdl(euler_cfg_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, vc, vu, n, g, dt);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ denoising step: latent <-> tokens
+
+// Block inputs of one denoising step: for every batch element, x_c = [text_c; bf16(z)] and
+// x_u = [text_u; bf16(z)] (the latent's rows are the image tokens).  One thread per 8 values
+// of one row of x_c (the uncond rows are written by the same thread when they exist); x_u may
+// be null (one branch only).
+__global__ void denoise_pack_kernel(const float* __restrict__ z, const uint16_t* __restrict__ text_c,
+                                    const uint16_t* __restrict__ text_u, uint16_t* __restrict__ x_c,
+                                    uint16_t* __restrict__ x_u, int batch, int n_img, int d, int lc, int lu) {
+  pdl_wait_then_release();
+  const int v8 = d / 8;
+  const int rows = max(lc, lu) + n_img;
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= static_cast<int64_t>(batch) * rows * v8) return;
+  const int c = static_cast<int>(idx % v8);
+  const int64_t br = idx / v8;
+  const int b = static_cast<int>(br / rows);
+  const int r = static_cast<int>(br % rows);  // r < n_img: image row r; otherwise text row r - n_img
+  if (r < n_img) {
+    float v[8];
+    load8<FMT_F32>(z, (static_cast<int64_t>(b) * n_img + r) * v8 + c, v);
+    store8<FMT_BF16>(x_c, (static_cast<int64_t>(b) * (lc + n_img) + lc + r) * v8 + c, v);
+    if (x_u != nullptr) store8<FMT_BF16>(x_u, (static_cast<int64_t>(b) * (lu + n_img) + lu + r) * v8 + c, v);
+  } else {
+    const int t = r - n_img;
+    const uint4* src;
+    if (t < lc) {
+      src = reinterpret_cast<const uint4*>(text_c) + (static_cast<int64_t>(b) * lc + t) * v8 + c;
+      reinterpret_cast<uint4*>(x_c)[(static_cast<int64_t>(b) * (lc + n_img) + t) * v8 + c] = *src;
+    }
+    if (t < lu && x_u != nullptr) {
+      src = reinterpret_cast<const uint4*>(text_u) + (static_cast<int64_t>(b) * lu + t) * v8 + c;
+      reinterpret_cast<uint4*>(x_u)[(static_cast<int64_t>(b) * (lu + n_img) + t) * v8 + c] = *src;
+    }
+  }
+}
+
+cudaError_t launch_denoise_pack(const float* z, const uint16_t* text_c, const uint16_t* text_u, uint16_t* x_c,
+                                uint16_t* x_u, int batch, int n_img, int d, int lc, int lu, cudaStream_t s) {
+  const int64_t n = static_cast<int64_t>(batch) * (max(lc, lu) + n_img) * (d / 8);
+  if (n <= 0) return cudaSuccess;
+  launch_pdl(denoise_pack_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, z, text_c, text_u,
+             x_c, x_u, batch, n_img, d, lc, lu);
+  return cudaGetLastError();
+}
+
+// z[b, i] += dt * (v_u + g (v_c - v_u)) with v_c = out_c[b, lc + i] and v_u = out_u[b, lu + i]
+// (the image rows of the two stacks' outputs), the fp32 arithmetic of euler_cfg_kernel.
+__global__ void denoise_update_kernel(float* __restrict__ z, const uint16_t* __restrict__ out_c,
+                                      const uint16_t* __restrict__ out_u, int batch, int n_img, int d, int lc, int lu,
+                                      float guidance, float dt) {
+  pdl_wait_then_release();
+  const int v8 = d / 8;
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= static_cast<int64_t>(batch) * n_img * v8) return;
+  const int c = static_cast<int>(idx % v8);
+  const int64_t bi = idx / v8;
+  const int b = static_cast<int>(bi / n_img);
+  const int i = static_cast<int>(bi % n_img);
+  float x[8], vc[8], vu[8];
+  load8<FMT_F32>(z, idx, x);
+  load8<FMT_BF16>(out_c, (static_cast<int64_t>(b) * (lc + n_img) + lc + i) * v8 + c, vc);
+  load8<FMT_BF16>(out_u, (static_cast<int64_t>(b) * (lu + n_img) + lu + i) * v8 + c, vu);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x[k] = fmaf(dt, fmaf(guidance, vc[k] - vu[k], vu[k]), x[k]);
+  store8<FMT_F32>(z, idx, x);
+}
+
+cudaError_t launch_denoise_update(float* z, const uint16_t* out_c, const uint16_t* out_u, int batch, int n_img, int d,
+                                  int lc, int lu, float guidance, float dt, cudaStream_t s) {
+  const int64_t n = static_cast<int64_t>(batch) * n_img * (d / 8);
+  if (n <= 0) return cudaSuccess;
+  launch_pdl(denoise_update_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, z, out_c, out_u,
+             batch, n_img, d, lc, lu, guidance, dt);
   return cudaGetLastError();
 }
 
@@ -245,6 +429,53 @@ __global__ void rope_table_kernel(int S, int n_text, int grid_w, int t_img, cons
   sin_tab[idx] = static_cast<float>(sn);
 }
 
+// Padded batches of prompts: element b holds L_b = clamp(text_lens[b], 0, n_text) text rows,
+// then its grid_h*grid_w image rows, then padding up to S.  Each element is positioned as if
+// alone: text j at (j, j, j), image cell (r, c) at (t_b, r, c) with t_b = L_b (or t_img when
+// t_img >= 0), padding rows at (0, 0, 0).  The tables are [batch, S, hd/2]; the (b, 0, 0) thread
+// also writes the element's key count L_b + grid_h*grid_w to kv_len[b].
+__global__ void rope_table_padded_kernel(int batch, int S, int n_text, int grid_w, int n_img, int t_img,
+                                         const int32_t* __restrict__ text_lens, int half, int sec_t, int sec_h,
+                                         double theta, float* cos_tab, float* sin_tab, int32_t* kv_len) {
+  pdl_wait_then_release();
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= static_cast<int64_t>(batch) * S * half) return;
+  const int64_t bs = idx / half;
+  const int i = static_cast<int>(idx - bs * half);
+  const int b = static_cast<int>(bs / S);
+  const int s = static_cast<int>(bs - static_cast<int64_t>(b) * S);
+  const int L = min(max(text_lens[b], 0), n_text);
+  if (s == 0 && i == 0) kv_len[b] = L + n_img;
+  int pt = 0, ph = 0, pw = 0;
+  if (s < L) {
+    pt = ph = pw = s;
+  } else if (s < L + n_img) {
+    const int k = s - L;
+    pt = t_img < 0 ? L : t_img;
+    ph = k / grid_w;
+    pw = k - ph * grid_w;
+  }
+  const int p = i < sec_t ? pt : (i < sec_t + sec_h ? ph : pw);
+  const float inv = static_cast<float>(pow(theta, -2.0 * i / (2.0 * half)));
+  double sn, cs;
+  sincos(static_cast<double>(p) * static_cast<double>(inv), &sn, &cs);
+  cos_tab[idx] = static_cast<float>(cs);
+  sin_tab[idx] = static_cast<float>(sn);
+}
+
+cudaError_t launch_rope_table_padded(int batch, int n_text, int grid_h, int grid_w, int t_img,
+                                     const int32_t* text_lens, int head_dim, const int32_t sections[3], float theta,
+                                     float* cos_tab, float* sin_tab, int32_t* kv_len, cudaStream_t s) {
+  const int S = n_text + grid_h * grid_w;
+  const int half = head_dim / 2;
+  const int64_t n = static_cast<int64_t>(batch) * S * half;
+  if (n <= 0) return cudaSuccess;
+  launch_pdl(rope_table_padded_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, batch, S, n_text,
+             grid_w, grid_h * grid_w, t_img, text_lens, half, sections[0], sections[1], static_cast<double>(theta),
+             cos_tab, sin_tab, kv_len);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, int head_dim,
                               const int32_t sections[3], float theta, float* cos_tab, float* sin_tab,
                               cudaStream_t s) {
@@ -265,10 +496,12 @@ cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, con
 // flight, one cos/sin fetch for both), so the hd/16 threads of one head are consecutive
 // lanes and reduce the two sums of squares with xor-shuffles.  F: storage format of the
 // qkv buffer (bf16 or f16).
+// tab_per_batch: the tables are [batch, seq, hd/2] (padded batches) rather than [seq, hd/2].
 template <int F>
 __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int seq, int n_heads, int head_dim,
                                     const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
-                                    const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
+                                    const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps,
+                                    int tab_per_batch) {
   pdl_wait_then_release();
   const int half = head_dim / 2;
   const int group = half / 8;  // threads per head: 8 (hd 128) or 4 (hd 64)
@@ -289,8 +522,9 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int s
   load8<F>(vk + 8 * c, 0, ka);
   load8<F>(vk + half + 8 * c, 0, kb);
   float cs[8], sn[8];
-  load8<FMT_F32>(cos_tab + static_cast<int64_t>(s) * half + 8 * c, 0, cs);
-  load8<FMT_F32>(sin_tab + static_cast<int64_t>(s) * half + 8 * c, 0, sn);
+  const int64_t trow = tab_per_batch ? bs : static_cast<int64_t>(s);
+  load8<FMT_F32>(cos_tab + trow * half + 8 * c, 0, cs);
+  load8<FMT_F32>(sin_tab + trow * half + 8 * c, 0, sn);
   float sq = 0.f, sk = 0.f;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -335,17 +569,18 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int s
 
 cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
                                 const float* cos_tab, const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k,
-                                float eps, cudaStream_t s) {
+                                float eps, bool tab_per_batch, cudaStream_t s) {
+  const int tpb = tab_per_batch ? 1 : 0;
   const int64_t threads = static_cast<int64_t>(batch) * seq * n_heads * (head_dim / 16);
   if (threads <= 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
   uint16_t* q = static_cast<uint16_t*>(qkv);
   if (fmt == FMT_F16)
     launch_pdl(qknorm_mrope_kernel<FMT_F16>, dim3(blocks), dim3(256), 0, s, q, batch, seq, n_heads, head_dim, cos_tab,
-               sin_tab, g_q, g_k, eps);
+               sin_tab, g_q, g_k, eps, tpb);
   else if (fmt == FMT_BF16)
     launch_pdl(qknorm_mrope_kernel<FMT_BF16>, dim3(blocks), dim3(256), 0, s, q, batch, seq, n_heads, head_dim, cos_tab,
-               sin_tab, g_q, g_k, eps);
+               sin_tab, g_q, g_k, eps, tpb);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

@@ -66,14 +66,26 @@ cudaError_t launch_rmsnorm(const void* x, int x_fmt, const uint16_t* g, void* y,
                            float eps, cudaStream_t s);
 cudaError_t launch_euler_cfg(float* x, const uint16_t* vc, const uint16_t* vu, int64_t n, float g, float dt,
                              cudaStream_t s);
+// Denoising step: block inputs [text; bf16(latent)] of both branches, and the CFG + Euler update
+// of the latent from the image rows of the two stacks' outputs.  d % 8 == 0.
+cudaError_t launch_denoise_pack(const float* z, const uint16_t* text_c, const uint16_t* text_u, uint16_t* x_c,
+                                uint16_t* x_u, int batch, int n_img, int d, int lc, int lu, cudaStream_t s);
+cudaError_t launch_denoise_update(float* z, const uint16_t* out_c, const uint16_t* out_u, int batch, int n_img, int d,
+                                  int lc, int lu, float guidance, float dt, cudaStream_t s);
 cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos, cudaStream_t s);
 // cos/sin table [S, hd/2] fp32 each, from positions (derived when pos == nullptr).
 cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, int head_dim,
                               const int32_t sections[3], float theta, float* cos_tab, float* sin_tab,
                               cudaStream_t s);
+// Per-element tables [batch, S, hd/2] and key counts kv_len [batch] of a padded batch of prompts
+// (text_lens: device int32 [batch], each clamped to [0, n_text]).
+cudaError_t launch_rope_table_padded(int batch, int n_text, int grid_h, int grid_w, int t_img,
+                                     const int32_t* text_lens, int head_dim, const int32_t sections[3], float theta,
+                                     float* cos_tab, float* sin_tab, int32_t* kv_len, cudaStream_t s);
+// tab_per_batch: cos/sin tables are [batch, seq, hd/2] rather than [seq, hd/2].
 cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
                                 const float* cos_tab, const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k,
-                                float eps, cudaStream_t s);
+                                float eps, bool tab_per_batch, cudaStream_t s);
 
 // Activation storage formats (the ABI's format codes).
 enum Fmt : int { FMT_BF16 = 0, FMT_F16 = 1, FMT_F32 = 2 };
@@ -93,6 +105,25 @@ struct GemmArgs {
   int k_splits = 1;  // > 1: y is fp32 [k_splits, M, N] partial sums (scale applied; no act / residual)
 };
 cudaError_t launch_gemm_w8a16(const GemmArgs& args, const KernelGuard& g, cudaStream_t s);
+
+// Y[M, N] = act( A8[M, K] (W8[N, K])^T * sa[m] * sw[n] ), e4m3 activations with a per-row scale and
+// e4m3 weights with a per-row scale (tcgen05 kind::f8f6f4).  N % 32 == 0, K % 16 == 0.
+struct GemmArgs8 {
+  const uint8_t* a;  // e4m3 [M, K]
+  const float* sa;   // [M]
+  const uint8_t* w;  // e4m3 [N, K]
+  const float* sw;   // [N]
+  void* y;           // [M, N], y_fmt
+  int y_fmt;
+  int M, N, K;
+  int act;  // 0 none, 1 GELU
+  int gelu_tanh;
+};
+cudaError_t launch_gemm_w8a8(const GemmArgs8& args, const KernelGuard& g, cudaStream_t s);
+// y8 = e4m3(RMSNorm(x) * g / s_row) with s_row = amax_row / 448 (1 for a zero row) written to ys;
+// x in x_fmt (bf16 / f32); cols % 8 == 0 and cols <= 8192.
+cudaError_t launch_rmsnorm_e4m3(const void* x, int x_fmt, const uint16_t* g, uint8_t* y8, float* ys, int64_t rows,
+                                int64_t cols, float eps, cudaStream_t s);
 // Split count that fills the SMs for an M x N x K problem (1 when the tile grid already does).
 int gemm_pick_splits(int M, int N, int K);
 // out (bf16, n elements) = sum of `splits` fp32 partials laid out [splits, n]; n % 8 == 0.
@@ -102,7 +133,9 @@ cudaError_t launch_splitk_reduce(const float* part, uint16_t* out, int64_t n, in
 // A kernel whose only wait never completes (exercises the bounded-wait path).
 cudaError_t launch_wait_selftest(const KernelGuard& g, cudaStream_t s);
 
+// kv_len: optional device int32 [batch], the number of leading keys of each batch element that
+// take part (clamped to [1, seq]); nullptr = all seq keys.
 cudaError_t launch_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
-                             const KernelGuard& g, cudaStream_t s);
+                             const int32_t* kv_len, const KernelGuard& g, cudaStream_t s);
 
 }  // namespace jab

@@ -169,3 +169,35 @@ def euler_inputs(n: int, config_index: int = 3) -> Dict[str, np.ndarray]:
         "v_cond": to_bf16_bits(normal(config_index, 11, (n,))),
         "v_uncond": to_bf16_bits(normal(config_index, 12, (n,))),
     }
+
+
+def block_weights_device(shape: BlockShape, seed: int, device) -> Dict[str, "torch.Tensor"]:
+    """FP8 weights, scales and gains of one block drawn directly on a CUDA device (torch's own
+    generator, so not the numpy streams above): for throughput runs that cycle through many
+    distinct weight sets, where drawing hundreds of MB on the host would dominate.  Same
+    distributions and the same per-output-row quantisation as ``block_inputs``; bf16 gains are
+    returned as int16 bit patterns, like the host path's uint16 arrays on the device."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    d, f, hd = shape.d_model, shape.d_mlp, shape.head_dim
+    out = {}
+    for name, rows, cols in (("w_qkv", 3 * d, d), ("w_o", d, d), ("w_up", f, d), ("w_down", d, f)):
+        w = torch.randn((rows, cols), generator=gen, device=device, dtype=torch.float32) * 0.02
+        amax = w.abs().amax(dim=1)
+        scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+        q = (w / scale[:, None]).clamp_(-E4M3_MAX, E4M3_MAX)
+        out[name] = q.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+        out["s_" + name[2:]] = scale.contiguous()
+        del w, q
+    for name, n in (("g_norm1", d), ("g_norm2", d), ("g_q", hd), ("g_k", hd)):
+        g = 1.0 + 0.05 * torch.randn((n,), generator=gen, device=device, dtype=torch.float32)
+        out[name] = g.to(torch.bfloat16).view(torch.int16).contiguous()
+    return out
+
+
+def bf16_normal_device(shape, seed: int, device, std: float = 1.0) -> "torch.Tensor":
+    """bf16 ~ N(0, std^2) activations drawn on the device (int16 bit patterns)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return (torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * std).to(
+        torch.bfloat16).view(torch.int16)

@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_host_only_calls_without_gpu(lib):
-    assert lib.dit_abi_version() == 1
+    assert lib.dit_abi_version() == 2
     assert lib.dit_status_str(0) == b"ok"
     assert lib.dit_status_str(5).startswith(b"device-side bounded wait")
     cfg = _abi.BlockConfig()
