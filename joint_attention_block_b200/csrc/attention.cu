@@ -7,38 +7,36 @@
 // A batch of prompts padded to one length passes a per-element key count; keys at or
 // beyond it are left out of every row's softmax (padding sits at the end of each element).
 //
-// Two CTAs on two SMs (a cluster of 2) share 256 queries of one (batch, head): each CTA
-// holds 128 query rows, and the pair form of the MMA (tcgen05.mma.cta_group::2, M = 256)
-// lets each CTA load only half of every key/value block:
+// Two CTAs on two SMs (a cluster of 2) share 512 queries of one (batch, head) as two
+// query tiles A and B of 256 rows; each CTA holds 128 rows of each tile.  The pair form of
+// the MMA (tcgen05.mma.cta_group::2, M = 256) lets each CTA load only half of every
+// key/value block:
 //   S = Q K^T    N = 128 keys; CTA r loads keys [64 r, 64 r + 64) of the block
-//   O += P V     N = hd;      CTA r loads value columns [r hd/2, (r + 1) hd/2) of all 128 keys,
-//                             P (the A operand) is read from each CTA's own tensor memory.
-// The key blocks are processed by two independent groups: group 0 takes the even blocks,
-// group 1 the odd ones, each with its own S buffer, O accumulator and running max/sum in
-// TMEM (S0 | S1 | O0 | O1 = 512 columns for hd 128).  While one group's softmax runs, the
-// tensor core computes the other group's P V and next S, so the exponentials of one group
-// overlap the MMAs of the other.  At the end the two partial results of each row are merged
-// (a two-way split of the keys, combined with their maxima and sums).
-//
-//   warp 0       TMA producer: this CTA's Q rows once, then per key block its K and V halves
-//                (4-stage ring), straight from the fused qkv buffer [B, S, 3d]; every copy
+//   O += P V     N = hd;      CTA r loads value columns [r hd/2, (r + 1) hd/2) of the block,
+//                             P (the A operand) is read from each CTA's own tensor memory,
+// so a 4-stage key/value ring fits beside both query tiles.  Each tile owns 256 TMEM columns
+// (S: 128 fp32 columns, O: hd columns); the tiles ping-pong so that the tensor core works on
+// one tile while the other tile's softmax runs:
+//     MMA issue order per key block j:  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
+//   warp 0       TMA producer: this CTA's rows of Q_A and Q_B once, then per key block its K
+//                and V halves, straight from the fused qkv buffer [B, S, 3d]; every copy
 //                completes on the leader CTA's barriers.
-//   warp 1       TMEM allocation (pair); in the leader, one lane issues
-//                S(0), S(1), then per block j: P V(j) into O_{j%2}, S(j+2) into S_{j%2}.
-//   warps 2..5   softmax of group 0, warps 6..9 of group 1; thread = query row (TMEM lane),
-//                so the running max and sum are thread-local.  The whole row of S comes out of
-//                TMEM in one round trip; exp2 with log2(e)/sqrt(hd) folded in (packed fp32 pair
-//                arithmetic for the scaling and the sums); P is written back over S as 16-bit
-//                pairs.  The max in use is only raised (and O rescaled in TMEM) when a block
-//                exceeds it by 2^8, which leaves O / l unchanged and keeps P <= 256.
-//                At the end both groups merge the two partial results, each writing half of
-//                the head's columns.
+//   warp 1       TMEM allocation (pair); in the leader, one lane issues the pair MMAs.
+//   warps 2..5   softmax of tile A; warps 6..9 softmax of tile B.  Thread i owns query
+//                row i of its tile (TMEM lane i), so the running max and sum are thread-local.
+//                The whole row of S is read from TMEM at once; exp2 with the
+//                log2(e)/sqrt(hd) scale folded in (packed fp32 pair arithmetic for the
+//                scaling and the row sums).  P is written back over S in TMEM as 16-bit pairs.
+//                The running max is only raised (and O rescaled in TMEM) when it grows
+//                by more than 2^8; until then the stale max is used for both P and the
+//                row sum, which leaves O / l unchanged and keeps P <= 256.  At the end
+//                the same warps store O / l in the q/k/v format.
 #include "common.cuh"
 
 namespace jab {
 namespace attn {
 
-constexpr int BQ = 128;   // query rows per CTA (256 per pair)
+constexpr int BQ = 128;   // rows of each query tile per CTA (a tile spans 256 rows of the pair)
 constexpr int BKV = 128;  // keys per block
 constexpr int STAGES = 4;
 constexpr int THREADS = 320;
@@ -49,22 +47,24 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #endif
 // 0: every exp2 on the MUFU unit; n > 0: one key pair in n on the FMA pipe (exp2_poly).
 constexpr int POLY_EVERY = JAB_ATTN_POLY_EVERY;
+#ifndef JAB_ATTN_TWO_PASS
+#define JAB_ATTN_TWO_PASS 0
+#endif
 
 template <int HD>
 struct Layout {
   static constexpr int Q_SLAB = 128 * 128;  // 128 rows x 64 16-bit values, 128-byte swizzle
-  static constexpr int Q_BYTES = (HD / 64) * Q_SLAB;
+  static constexpr int Q_TILE = (HD / 64) * Q_SLAB;
   static constexpr int K_SLAB = 64 * 128;  // 64 keys x 64 16-bit values
   static constexpr int K_BYTES = (HD / 64) * K_SLAB;
   static constexpr int V_ROW = HD;  // bytes per key of this CTA's hd/2 value columns
   static constexpr int V_BYTES = BKV * V_ROW;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_Q = 0;  // [2] tiles
+  static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * V_BYTES;
   static constexpr int NUM_BARS = 1 + 3 * STAGES + 6;
-  static constexpr int OFF_XCH = OFF_BAR + NUM_BARS * 8;  // [group][m, l][row] fp32
-  static constexpr int OFF_MISC = OFF_XCH + 2 * 2 * BQ * 4;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static_assert(OFF_V % 1024 == 0 && V_BYTES % 1024 == 0, "swizzled tiles keep 1024-byte alignment");
 };
@@ -98,9 +98,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Barrier among the 256 softmax threads (warps 2..9) only.
-__device__ __forceinline__ void softmax_bar_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
 template <int HD, int F>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -114,15 +111,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* q_full = bars;                  // leader: both CTAs' Q rows landed
-  uint64_t* k_full = q_full + 1;            // [STAGES] leader: both K halves of a block landed
-  uint64_t* v_full = k_full + STAGES;       // [STAGES] leader: both V halves landed
-  uint64_t* kv_empty = v_full + STAGES;     // [STAGES] the block's last MMA (P V) is done
-  uint64_t* s_full = kv_empty + STAGES;     // [2 groups] S ready (all earlier MMAs done)
-  uint64_t* p_full = s_full + 2;            // [2 groups] leader: both CTAs' P written
-  uint64_t* o_full = p_full + 2;            // every MMA done
+  uint64_t* q_full = bars;               // leader: both CTAs' Q rows landed
+  uint64_t* k_full = q_full + 1;         // [STAGES] leader: both K halves of a block landed
+  uint64_t* v_full = k_full + STAGES;    // [STAGES] leader: both V halves landed
+  uint64_t* kv_empty = v_full + STAGES;  // [STAGES] both tiles' P V of the block are done
+  uint64_t* s_full = kv_empty + STAGES;  // [2 tiles] S_t(j) ready (and P V_t(j-1) done)
+  uint64_t* p_full = s_full + 2;         // [2 tiles] leader: both CTAs' P_t(j) written, O_t rescaled
+  uint64_t* o_full = p_full + 2;         // both tiles' O final
   uint64_t* drain_bar = o_full + 1;
-  float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 4);
 
@@ -130,7 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int lane = static_cast<int>(lane_id());
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int q0 = (blockIdx.x >> 1) * 2 * BQ + static_cast<int>(rank) * BQ;  // this CTA's first query row
+  const int q0 = (blockIdx.x >> 1) * 4 * BQ + static_cast<int>(rank) * BQ;  // tile t: rows q0 + 2 BQ t ..
   const int head = blockIdx.y;
   const int b = blockIdx.z;
   const int d = n_heads * HD;
@@ -142,9 +138,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&s_full[g], 1);
-      mbar_init(&p_full[g], 8);  // 4 softmax warps of the group in each CTA
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 8);  // 4 softmax warps of the tile in each CTA
     }
     mbar_init(o_full, 1);
     mbar_init(drain_bar, 1);
@@ -171,9 +167,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
-      if (leader) mbar_arrive_expect_tx(q_full, 2 * L::Q_BYTES);
+      if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * L::Q_TILE);
       const uint32_t qbar = mapa_shared(smem_u32(q_full), 0);
-      for (int c = 0; c < HD / 64; ++c) tma_load_3d_pair(sQ + c * L::Q_SLAB, &tm_q, qbar, head * HD + 64 * c, q0, b);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < HD / 64; ++c)
+          tma_load_3d_pair(sQ + t * L::Q_TILE + c * L::Q_SLAB, &tm_q, qbar, head * HD + 64 * c, q0 + 2 * BQ * t, b);
     }
     __syncwarp();
     int issued = 0;
@@ -215,58 +213,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (leader) {
       constexpr uint32_t idesc_s = idesc_f16kind(2 * BQ, BKV, kF16, false, false);
       constexpr uint32_t idesc_o = idesc_f16kind(2 * BQ, HD, kF16, false, true);
-      auto issue_s = [&](int j) {  // S(j) = Q K_j^T into S_{j%2}
-        const int g = j & 1;
-        const uint32_t qbase = smem_u32(sQ);
+      auto issue_s = [&](int t, int j) {  // S_t(j) = Q_t K_j^T into columns [256 t, 256 t + 128)
+        const uint32_t qbase = smem_u32(sQ + t * L::Q_TILE);
         const uint32_t kbase = smem_u32(sK + (j % STAGES) * L::K_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t oq = (kk >> 2) * L::Q_SLAB + (kk & 3) * 32;
           const uint32_t ok_ = (kk >> 2) * L::K_SLAB + (kk & 3) * 32;
-          mma_f16kind_ss_pair(tmem + 128 * g, smem_desc_sw128(qbase + oq, 16, 1024),
+          mma_f16kind_ss_pair(tmem + 256 * t, smem_desc_sw128(qbase + oq, 16, 1024),
                               smem_desc_sw128(kbase + ok_, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit_pair(&s_full[g], 0x3);
+        mma_commit_pair(&s_full[t], 0x3);
       };
-      auto issue_pv = [&](int j) {  // O_{j%2} += P(j) V_j, P from TMEM (the first 64 columns of S_{j%2})
-        const int g = j & 1;
+      auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P from TMEM (columns [256 t, 256 t + 64))
         const uint32_t vbase = smem_u32(sV + (j % STAGES) * L::V_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint32_t a = vbase + kk * 16 * L::V_ROW;
           const uint64_t bd = HD == 128 ? smem_desc_sw128(a, 16, 8 * L::V_ROW) : smem_desc_sw64(a, 16, 8 * L::V_ROW);
-          mma_f16kind_ts_pair(tmem + 256 + HD * g, tmem + 128 * g + 8 * kk, bd, idesc_o,
-                              (j >= 2 || kk > 0) ? 1u : 0u);
+          mma_f16kind_ts_pair(tmem + 256 * t + 128, tmem + 256 * t + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit_pair(&kv_empty[j % STAGES], 0x3);  // K_j and V_j fully consumed
       };
-      bool ok = mbar_wait(q_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, rank, 0));
-      for (int j = 0; j < 2 && j < nb && ok; ++j) {
-        ok = mbar_wait(&k_full[j], 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, rank, j));
-        if (!ok) break;
+      bool ok = mbar_wait(q_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, rank, 0)) &&
+                mbar_wait(&k_full[0], 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, rank, 0));
+      if (ok) {
         tc_fence_after();
-        if (lane == 0) issue_s(j);
+        if (lane == 0) {
+          issue_s(0, 0);
+          issue_s(1, 0);
+        }
         __syncwarp();
       }
       for (int j = 0; j < nb && ok; ++j) {
-        const int g = j & 1;
-        ok = mbar_wait(&v_full[j % STAGES], static_cast<uint32_t>(j / STAGES) & 1u, guard, abort_flag,
-                       where_code(ERR_TIMEOUT_ATTN_MMA, rank, j)) &&
-             mbar_wait(&p_full[g], static_cast<uint32_t>(j >> 1) & 1u, guard, abort_flag,
-                       where_code(ERR_TIMEOUT_ATTN_MMA, 2 + g, j));
+        const int st = j % STAGES;
+        const uint32_t par = static_cast<uint32_t>(j) & 1u;
+        const bool next = j + 1 < nb;
+        ok = mbar_wait(&v_full[st], static_cast<uint32_t>(j / STAGES) & 1u, guard, abort_flag,
+                       where_code(ERR_TIMEOUT_ATTN_MMA, 1, j)) &&
+             mbar_wait(&p_full[0], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 2, j)) &&
+             (!next || mbar_wait(&k_full[(j + 1) % STAGES], static_cast<uint32_t>((j + 1) / STAGES) & 1u, guard,
+                                 abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 3, j)));
         if (!ok) break;
         tc_fence_after();
-        if (lane == 0) issue_pv(j);
-        __syncwarp();
-        if (j + 2 < nb) {
-          // S(j+2) overwrites P(j) only after P V(j) has read it (MMAs run in issue order)
-          ok = mbar_wait(&k_full[(j + 2) % STAGES], static_cast<uint32_t>((j + 2) / STAGES) & 1u, guard, abort_flag,
-                         where_code(ERR_TIMEOUT_ATTN_MMA, 4 + g, j));
-          if (!ok) break;
-          tc_fence_after();
-          if (lane == 0) issue_s(j + 2);
-          __syncwarp();
+        if (lane == 0) {
+          issue_pv(0, j);
+          if (next) issue_s(0, j + 1);  // overwrites P_A(j) only after PV_A(j) has read it (in-order issue)
         }
+        __syncwarp();
+        ok = mbar_wait(&p_full[1], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 4, j));
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          issue_pv(1, j);
+          mma_commit_pair(&kv_empty[st], 0x3);  // K_j and V_j fully consumed by both tiles
+          if (next) issue_s(1, j + 1);
+        }
+        __syncwarp();
       }
       if (lane == 0) {
         if (ok) mma_commit_pair(o_full, 0x3);
@@ -276,28 +278,129 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     mbar_wait(drain_bar, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_DRAIN, rank, 1), true);
   } else {
-    // ---------------- softmax: warps 2..5 -> group 0 (even key blocks), 6..9 -> group 1 (odd)
-    const int g = (warp - 2) >> 2;
+    // ---------------- softmax: warps 2..5 -> tile A, 6..9 -> tile B; thread owns query row
+    const int t = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_col = tmem + lane_off + 128 * g;
-    const uint32_t o_col = tmem + lane_off + 256 + HD * g;
-    const uint32_t pbar = mapa_shared(smem_u32(&p_full[g]), 0);
+    const uint32_t s_col = tmem + lane_off + 256 * t;
+    const uint32_t o_col = s_col + 128;
+    const uint32_t pbar = mapa_shared(smem_u32(&p_full[t]), 0);
     const float c_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
     float m_used = -INFINITY;
     float l = 0.f;
     bool ok = true;
-    int i = 0;
-    for (int j = g; j < nb; j += 2, ++i) {
-      if (!mbar_wait(&s_full[g], static_cast<uint32_t>(i) & 1u, guard, abort_flag,
-                     where_code(ERR_TIMEOUT_ATTN_SOFTMAX, rank * 2 + g, j))) {
+    for (int j = 0; j < nb; ++j) {
+      if (!mbar_wait(&s_full[t], static_cast<uint32_t>(j) & 1u, guard, abort_flag,
+                     where_code(ERR_TIMEOUT_ATTN_SOFTMAX, rank * 2 + t, j))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int valid = nkv - j * BKV;  // keys beyond this element's key count are masked
       const bool full = valid >= BKV;    // every block but possibly the last
+#if JAB_ATTN_TWO_PASS
+      // Two passes over S in TMEM: the row max from four 32-column loads, then the
+      // exponentials chunk by chunk (the next chunk's load in flight), so that only 64 logits
+      // are in registers at a time.
+      float m8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+      {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(s_col, ra);
+        tmem_ld32(s_col + 32, rb);
+        tmem_ld_wait_regs(ra);
+        tmem_ld_wait_regs(rb);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          m8[k] = fmax3(fmax3(__uint_as_float(ra[k]), __uint_as_float(ra[8 + k]), __uint_as_float(ra[16 + k])),
+                        fmax3(__uint_as_float(ra[24 + k]), __uint_as_float(rb[k]), __uint_as_float(rb[8 + k])),
+                        fmaxf(__uint_as_float(rb[16 + k]), __uint_as_float(rb[24 + k])));
+        tmem_ld32(s_col + 64, ra);
+        tmem_ld32(s_col + 96, rb);
+        tmem_ld_wait_regs(ra);
+        tmem_ld_wait_regs(rb);
+        if (!full) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            ra[k] = 64 + k < valid ? ra[k] : __float_as_uint(-INFINITY);
+            rb[k] = 96 + k < valid ? rb[k] : __float_as_uint(-INFINITY);
+          }
+          if (valid <= 64) {  // the first half holds masked keys too
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+            uint32_t rc[32], rd[32];
+            tmem_ld32(s_col, rc);
+            tmem_ld32(s_col + 32, rd);
+            tmem_ld_wait_regs(rc);
+            tmem_ld_wait_regs(rd);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              m8[k & 7] = fmaxf(m8[k & 7], k < valid ? __uint_as_float(rc[k]) : -INFINITY);
+              m8[k & 7] = fmaxf(m8[k & 7], 32 + k < valid ? __uint_as_float(rd[k]) : -INFINITY);
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          m8[k] = fmax3(fmax3(m8[k], __uint_as_float(ra[k]), __uint_as_float(ra[8 + k])),
+                        fmax3(__uint_as_float(ra[16 + k]), __uint_as_float(ra[24 + k]), __uint_as_float(rb[k])),
+                        fmax3(__uint_as_float(rb[8 + k]), __uint_as_float(rb[16 + k]), __uint_as_float(rb[24 + k])));
+      }
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * c_log2;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mx > m_used + RESCALE_THRESHOLD) {
+        alpha = ex2_approx(m_used - mx);  // 0 on the first block
+        m_used = mx;
+        rescale = true;
+      }
+      // exponentiate 32 keys at a time, sum, and write P_t(j) as 16-bit pairs over the first
+      // 64 columns of S_t (the A operand of the PV MMA); a chunk's P lands in columns that
+      // the chunks already read
+      float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 c2 = make_float2(c_log2, c_log2);
+      const float2 nm2 = make_float2(-m_used, -m_used);
+      uint32_t cur[32], nxt[32];
+      tmem_ld32(s_col, cur);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        tmem_ld_wait_regs(cur);
+        if (h + 1 < 4) tmem_ld32(s_col + 32 * (h + 1), nxt);
+        uint32_t pk[16];
+#pragma unroll
+        for (int k2 = 0; k2 < 32; k2 += 2) {
+          const int k = 32 * h + k2;
+          float a = __uint_as_float(cur[k2]), bb = __uint_as_float(cur[k2 + 1]);
+          if (!full) {
+            a = k < valid ? a : -INFINITY;
+            bb = k + 1 < valid ? bb : -INFINITY;
+          }
+          const float2 x = fma2(make_float2(a, bb), c2, nm2);  // packed pair: s c - m
+          float2 e;
+          bool poly = false;
+          if constexpr (POLY_EVERY > 0) poly = (k >> 1) % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1;
+          if (poly) {
+            e.x = exp2_poly(x.x);
+            e.y = exp2_poly(x.y);
+          } else {
+            e.x = ex2_approx(x.x);
+            e.y = ex2_approx(x.y);
+          }
+          ps[(k2 >> 1) & 3] = add2(ps[(k2 >> 1) & 3], e);
+          pk[k2 >> 1] = pack2<F>(e.x, e.y);
+        }
+        tmem_st16(s_col + 16 * h, pk);
+        if (h + 1 < 4) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
+        }
+      }
+      const float2 ps01 = add2(ps[0], ps[1]), ps23 = add2(ps[2], ps[3]);
+      const float2 ps03 = add2(ps01, ps23);
+      const float sum = ps03.x + ps03.y;
+#else
       // The whole row of S (128 keys) comes out of TMEM in one round trip; the max and the
       // exponentials then run from registers with independent partial results.
       uint32_t s0[32], s1[32], s2[32], s3[32];
@@ -336,20 +439,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       float alpha = 1.f;
       bool rescale = false;
       if (mx > m_used + RESCALE_THRESHOLD) {
-        alpha = ex2_approx(m_used - mx);  // 0 on the group's first block
+        alpha = ex2_approx(m_used - mx);  // 0 on the first block
         m_used = mx;
         rescale = true;
       }
-      // exponentiate, sum, and write P as 16-bit pairs over the first 64 columns of S
+      // exponentiate, sum, and write P_t(j) as 16-bit pairs over the first 64 columns of S_t
+      // (the A operand of the PV MMA)
       float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 c2 = make_float2(c_log2, c_log2);
       const float2 nm2 = make_float2(-m_used, -m_used);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+      for (int h = 0; h < 4; ++h) {  // four 32-key chunks: 16 packed columns each
+        uint32_t pk[16];
 #pragma unroll
-        for (int k2 = 0; k2 < 64; k2 += 2) {
-          const int k = 64 * h + k2;
+        for (int k2 = 0; k2 < 32; k2 += 2) {
+          const int k = 32 * h + k2;
           const float2 x = fma2(make_float2(v[k], v[k + 1]), c2, nm2);  // packed pair: s c - m
           float2 e;
           bool poly = false;
@@ -364,14 +468,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           ps[(k2 >> 1) & 3] = add2(ps[(k2 >> 1) & 3], e);
           pk[k2 >> 1] = pack2<F>(e.x, e.y);
         }
-        tmem_st32(s_col + 32 * h, pk);
+        tmem_st16(s_col + 16 * h, pk);
       }
       const float2 ps01 = add2(ps[0], ps[1]), ps23 = add2(ps[2], ps[3]);
       const float2 ps03 = add2(ps01, ps23);
       const float sum = ps03.x + ps03.y;
-      // O of this group is up to date here: its last P V was issued before S(j), and the
-      // commit behind s_full covers every earlier MMA.
-      if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+#endif
+      // O_t is up to date here: PV_t(j-1) was issued before S_t(j) and s_full covers it.
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t raw[32];
@@ -388,43 +492,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(pbar);
     }
-    // ---- merge the two groups' partial results: each group writes half of the head's columns
-    if (ok) ok = mbar_wait(o_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_SOFTMAX, 4 + rank, 0));
-    xch[(2 * g) * BQ + r] = m_used;
-    xch[(2 * g + 1) * BQ + r] = l;
-    softmax_bar_sync();  // every softmax thread gets here exactly once, failed waits included
-    const float mA = xch[r], lA = xch[BQ + r], mB = xch[2 * BQ + r], lB = xch[3 * BQ + r];
-    const bool hasB = nb >= 2;  // group 1 saw at least one block
-    if (ok) {
+    if (ok && mbar_wait(o_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_SOFTMAX, 4 + rank, t))) {
       tc_fence_after();
-      const float m = hasB ? fmaxf(mA, mB) : mA;
-      const float aA = ex2_approx(mA - m);
-      const float aB = hasB ? ex2_approx(mB - m) : 0.f;
-      const float inv = 1.f / (lA * aA + lB * aB);
-      const float fA = aA * inv, fB = aB * inv;
-      const int row = q0 + r;
+      const float inv_l = 1.f / l;
+      const int row = q0 + 2 * BQ * t + r;
       uint16_t* dst = out + (static_cast<size_t>(b) * seq + row) * d + head * HD;
 #pragma unroll
-      for (int c = 0; c < HD / 64; ++c) {
-        const int col = g * (HD / 2) + 32 * c;
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tmem + lane_off + 256 + col, ra);
-        if (hasB) tmem_ld32(tmem + lane_off + 256 + HD + col, rb);
-        tmem_ld_wait_regs(ra);
-        if (hasB) {
-          tmem_ld_wait_regs(rb);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) rb[k] = 0u;
-        }
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(o_col + 32 * c, raw);
+        tmem_ld_wait();
         if (row < seq) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float o[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              o[k] = fmaf(__uint_as_float(ra[8 * q + k]), fA, __uint_as_float(rb[8 * q + k]) * fB);
-            store8<F>(dst + col, q, o);
+            for (int k = 0; k < 8; ++k) o[k] = __uint_as_float(raw[8 * q + k]) * inv_l;
+            store8<F>(dst + 32 * c, q, o);
           }
         }
       }
@@ -447,11 +531,9 @@ cudaError_t launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   cudaError_t e =
       cudaFuncSetAttribute(attention_kernel<HD, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(2 * ((seq + 2 * BQ - 1) / (2 * BQ)), n_heads, batch);
-  e = launch_pdl(attention_kernel<HD, F>, grid, dim3(THREADS), L::SMEM, s, tq, tk, tv, static_cast<uint16_t*>(out),
-                 seq, n_heads, kv_len, g);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  dim3 grid(2 * ((seq + 4 * BQ - 1) / (4 * BQ)), n_heads, batch);
+  return launch_pdl(attention_kernel<HD, F>, grid, dim3(THREADS), L::SMEM, s, tq, tk, tv,
+                    static_cast<uint16_t*>(out), seq, n_heads, kv_len, g);
 }
 
 }  // namespace attn
