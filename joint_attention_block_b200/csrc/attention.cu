@@ -47,9 +47,6 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #endif
 // 0: every exp2 on the MUFU unit; n > 0: one key pair in n on the FMA pipe (exp2_poly).
 constexpr int POLY_EVERY = JAB_ATTN_POLY_EVERY;
-#ifndef JAB_ATTN_TWO_PASS
-#define JAB_ATTN_TWO_PASS 0
-#endif
 
 template <int HD>
 struct Layout {
@@ -299,108 +296,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int valid = nkv - j * BKV;  // keys beyond this element's key count are masked
       const bool full = valid >= BKV;    // every block but possibly the last
-#if JAB_ATTN_TWO_PASS
-      // Two passes over S in TMEM: the row max from four 32-column loads, then the
-      // exponentials chunk by chunk (the next chunk's load in flight), so that only 64 logits
-      // are in registers at a time.
-      float m8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
-      {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(s_col, ra);
-        tmem_ld32(s_col + 32, rb);
-        tmem_ld_wait_regs(ra);
-        tmem_ld_wait_regs(rb);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          m8[k] = fmax3(fmax3(__uint_as_float(ra[k]), __uint_as_float(ra[8 + k]), __uint_as_float(ra[16 + k])),
-                        fmax3(__uint_as_float(ra[24 + k]), __uint_as_float(rb[k]), __uint_as_float(rb[8 + k])),
-                        fmaxf(__uint_as_float(rb[16 + k]), __uint_as_float(rb[24 + k])));
-        tmem_ld32(s_col + 64, ra);
-        tmem_ld32(s_col + 96, rb);
-        tmem_ld_wait_regs(ra);
-        tmem_ld_wait_regs(rb);
-        if (!full) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            ra[k] = 64 + k < valid ? ra[k] : __float_as_uint(-INFINITY);
-            rb[k] = 96 + k < valid ? rb[k] : __float_as_uint(-INFINITY);
-          }
-          if (valid <= 64) {  // the first half holds masked keys too
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
-            uint32_t rc[32], rd[32];
-            tmem_ld32(s_col, rc);
-            tmem_ld32(s_col + 32, rd);
-            tmem_ld_wait_regs(rc);
-            tmem_ld_wait_regs(rd);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              m8[k & 7] = fmaxf(m8[k & 7], k < valid ? __uint_as_float(rc[k]) : -INFINITY);
-              m8[k & 7] = fmaxf(m8[k & 7], 32 + k < valid ? __uint_as_float(rd[k]) : -INFINITY);
-            }
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          m8[k] = fmax3(fmax3(m8[k], __uint_as_float(ra[k]), __uint_as_float(ra[8 + k])),
-                        fmax3(__uint_as_float(ra[16 + k]), __uint_as_float(ra[24 + k]), __uint_as_float(rb[k])),
-                        fmax3(__uint_as_float(rb[8 + k]), __uint_as_float(rb[16 + k]), __uint_as_float(rb[24 + k])));
-      }
-      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * c_log2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mx > m_used + RESCALE_THRESHOLD) {
-        alpha = ex2_approx(m_used - mx);  // 0 on the first block
-        m_used = mx;
-        rescale = true;
-      }
-      // exponentiate 32 keys at a time, sum, and write P_t(j) as 16-bit pairs over the first
-      // 64 columns of S_t (the A operand of the PV MMA); a chunk's P lands in columns that
-      // the chunks already read
-      float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      const float2 c2 = make_float2(c_log2, c_log2);
-      const float2 nm2 = make_float2(-m_used, -m_used);
-      uint32_t cur[32], nxt[32];
-      tmem_ld32(s_col, cur);
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        tmem_ld_wait_regs(cur);
-        if (h + 1 < 4) tmem_ld32(s_col + 32 * (h + 1), nxt);
-        uint32_t pk[16];
-#pragma unroll
-        for (int k2 = 0; k2 < 32; k2 += 2) {
-          const int k = 32 * h + k2;
-          float a = __uint_as_float(cur[k2]), bb = __uint_as_float(cur[k2 + 1]);
-          if (!full) {
-            a = k < valid ? a : -INFINITY;
-            bb = k + 1 < valid ? bb : -INFINITY;
-          }
-          const float2 x = fma2(make_float2(a, bb), c2, nm2);  // packed pair: s c - m
-          float2 e;
-          bool poly = false;
-          if constexpr (POLY_EVERY > 0) poly = (k >> 1) % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1;
-          if (poly) {
-            e.x = exp2_poly(x.x);
-            e.y = exp2_poly(x.y);
-          } else {
-            e.x = ex2_approx(x.x);
-            e.y = ex2_approx(x.y);
-          }
-          ps[(k2 >> 1) & 3] = add2(ps[(k2 >> 1) & 3], e);
-          pk[k2 >> 1] = pack2<F>(e.x, e.y);
-        }
-        tmem_st16(s_col + 16 * h, pk);
-        if (h + 1 < 4) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
-        }
-      }
-      const float2 ps01 = add2(ps[0], ps[1]), ps23 = add2(ps[2], ps[3]);
-      const float2 ps03 = add2(ps01, ps23);
-      const float sum = ps03.x + ps03.y;
-#else
       // The whole row of S (128 keys) comes out of TMEM in one round trip; the max and the
       // exponentials then run from registers with independent partial results.
       uint32_t s0[32], s1[32], s2[32], s3[32];
@@ -473,7 +368,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const float2 ps01 = add2(ps[0], ps[1]), ps23 = add2(ps[2], ps[3]);
       const float2 ps03 = add2(ps01, ps23);
       const float sum = ps03.x + ps03.y;
-#endif
       // O_t is up to date here: PV_t(j-1) was issued before S_t(j) and s_full covers it.
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
