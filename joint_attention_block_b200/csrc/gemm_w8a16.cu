@@ -97,24 +97,6 @@ struct Params {
   int y_evict_first;            // output stream larger than L2: store it with an evict-first hint
 };
 
-// GELU, exact form: x * Phi(x), Phi the standard normal CDF.  Phi(-|x|) = erfc(|x| / sqrt 2) / 2
-// is evaluated with Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
-// erfc(z) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2) + e(z), t = 1 / (1 + p z),
-// |e(z)| <= 1.5e-7 for z >= 0, here with the hardware reciprocal and base-2 exponential.  Branch-free;
-// huge |x| gives x (x >= 0) or 0 (x < 0).
-__device__ __forceinline__ float gelu_erf(float x) {
-  constexpr float p = 0.3275911f;
-  // A&S coefficients, halved so that the sum is Phi(-|x|) rather than erfc
-  constexpr float a1 = 0.5f * 0.254829592f, a2 = 0.5f * -0.284496736f, a3 = 0.5f * 1.421413741f,
-                  a4 = 0.5f * -1.453152027f, a5 = 0.5f * 1.061405429f;
-  const float ax = fabsf(x);
-  const float t = rcp_approx(fmaf(p * 0.7071067811865476f, ax, 1.f));  // z = |x| / sqrt 2
-  const float q = fmaf(fmaf(fmaf(fmaf(a5, t, a4), t, a3), t, a2), t, a1) * t;
-  const float e = ex2_approx(x * (x * -0.7213475204444817f));  // exp(-x^2 / 2) = 2^(-x^2 log2(e) / 2)
-  // x Phi(x) = max(x, 0) - |x| Phi(-|x|)
-  return fmaf(-ax * e, q, fmaxf(x, 0.f));
-}
-
 // GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) = x / (1 + exp(-2y)).
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float y = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
@@ -386,7 +368,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+            for (int j = 0; j < 32; j += 2) {
+              const float2 g = gelu_erf_pair(make_float2(v[j], v[j + 1]));
+              v[j] = g.x;
+              v[j + 1] = g.y;
+            }
           }
         }
         if (has_res) {
@@ -499,21 +485,21 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, uint16_t* _
 }  // namespace gemm
 
 int gemm_pick_splits(int M, int N, int K) {
-  // The split count whose tile grid fills the pairs of SMs best (ties: fewer splits).
+  // The fewest K splits whose tile grid fills the pairs of SMs within 2 % of the best split count
+  // up to 16 (each split adds an fp32 partial of the output to write and reduce).
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
   const int kb = (K + gemm::BK - 1) / gemm::BK;
-  int best = 1;
+  double eff[17] = {0.0};
   double best_eff = 0.0;
-  for (int s = 1; s <= 8 && s <= kb / 16; ++s) {
+  for (int s = 1; s <= 16 && s <= kb / 16; ++s) {
     const int t = tiles * s;
     const int waves = (t + gemm::MAX_PAIRS - 1) / gemm::MAX_PAIRS;
-    const double eff = static_cast<double>(t) / (static_cast<double>(waves) * gemm::MAX_PAIRS);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = s;
-    }
+    eff[s] = static_cast<double>(t) / (static_cast<double>(waves) * gemm::MAX_PAIRS);
+    if (eff[s] > best_eff) best_eff = eff[s];
   }
-  return best;
+  for (int s = 1; s <= 16 && s <= kb / 16; ++s)
+    if (eff[s] >= best_eff - 0.02) return s;
+  return 1;
 }
 
 cudaError_t launch_splitk_reduce(const float* part, uint16_t* out, int64_t n, int splits, cudaStream_t s) {

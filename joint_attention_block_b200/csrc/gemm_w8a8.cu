@@ -61,19 +61,8 @@ struct Params {
   int y_evict_first;
 };
 
-// GELU, exact form, as in the W8A16 kernel: x Phi(x) with Phi(-|x|) from Abramowitz & Stegun,
-// Handbook of Mathematical Functions, 7.1.26 (|error| <= 1.5e-7).
-__device__ __forceinline__ float gelu_erf(float x) {
-  constexpr float p = 0.3275911f;
-  constexpr float a1 = 0.5f * 0.254829592f, a2 = 0.5f * -0.284496736f, a3 = 0.5f * 1.421413741f,
-                  a4 = 0.5f * -1.453152027f, a5 = 0.5f * 1.061405429f;
-  const float ax = fabsf(x);
-  const float t = rcp_approx(fmaf(p * 0.7071067811865476f, ax, 1.f));
-  const float q = fmaf(fmaf(fmaf(fmaf(a5, t, a4), t, a3), t, a2), t, a1) * t;
-  const float e = ex2_approx(x * (x * -0.7213475204444817f));
-  return fmaf(-ax * e, q, fmaxf(x, 0.f));
-}
-
+// GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) = x / (1 + exp(-2y)).  The exact
+// form is gelu_erf_pair (common.cuh).
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float y = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
   return x * rcp_approx(1.f + ex2_approx(-2.8853900817779268f * y));
@@ -269,7 +258,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+            for (int j = 0; j < 32; j += 2) {
+              const float2 g = gelu_erf_pair(make_float2(v[j], v[j + 1]));
+              v[j] = g.x;
+              v[j + 1] = g.y;
+            }
           }
         }
         if (lane == 0) bulk_wait_group_read<1>();  // the box written two chunks ago has been read
