@@ -7,5 +7,6 @@ the library has not been built.
 """
 from . import _abi as ops  # noqa: F401
 from . import synth  # noqa: F401
+from . import fp8_checkpoint  # noqa: F401
 
-__all__ = ["ops", "synth"]
+__all__ = ["ops", "synth", "fp8_checkpoint"]
