@@ -108,52 +108,116 @@ def traffic_per_launch(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi samples (every 50 ms) of SM clock and throttle reasons, kept with wall-clock stamps."""
+    """SM clock, power and clock-event (throttle) reasons sampled during the timed region.
+
+    NVML is polled from a thread every 5 ms (a 40 ms region still gets several samples); the GPU
+    is found by the PCI bus id of the CUDA device in use, so the samples are of this process's GPU
+    whatever CUDA_VISIBLE_DEVICES maps.  Without NVML, ``nvidia-smi -lms 50`` on the same bus id."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    PERIOD_S = 0.005
 
     def __init__(self, index: int):
-        self.samples = []
+        self.samples = []  # (wall time, sm MHz, max sm MHz, power W, set of active reason names)
         self.proc = None
         self.index = index
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _bus_id(self):
+        try:
+            p = torch.cuda.get_device_properties(self.index)
+            return "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        except Exception:
+            return None
 
     def start(self):
+        bus = self._bus_id()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode()) if bus
+                 else pynvml.nvmlDeviceGetHandleByIndex(self.index))
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self._start_smi(bus)
+            return
+        self.source = "nvml"
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.time(), sm, mx, pw, {n for n, b in bits.items() if r & b}))
+                except Exception:
+                    pass
+                self._stop.wait(self.PERIOD_S)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
+
+    def _start_smi(self, bus):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", "-i", bus or str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
-        threading.Thread(target=self._read, daemon=True).start()
+        self.source = "nvidia-smi"
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        def read():
+            for line in self.proc.stdout:
+                r = [x.strip() for x in line.split(",")]
+                if len(r) < 8:
+                    continue
+                act = {n for i, n in enumerate(self.REASONS) if r[4 + i] == "Active"}
+                self.samples.append((time.time(), num(r[0]), num(r[1]), num(r[2]), act))
+
+        self._thread = threading.Thread(target=read, daemon=True)
+        self._thread.start()
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
     def summary(self, t0: float, t1: float):
-        rows = [v for (t, v) in self.samples if t0 <= t <= t1 + 0.05]
+        rows = [v for (t, *v) in self.samples if t0 <= t <= t1 + self.PERIOD_S]
         if not rows:
-            rows = [v for (_, v) in self.samples[-5:]]
+            rows = [v for (_, *v) in self.samples[-5:]]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 4 + i and r[4 + i] == "Active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"], "samples": 0}
+        sm = [r[0] for r in rows if r[0] is not None]
+        mx = [r[1] for r in rows if r[1] is not None]
+        pw = [r[2] for r in rows if r[2] is not None]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)}
+                "reasons": sorted(set().union(*[r[3] for r in rows])), "samples": len(rows),
+                "power_w_max": round(max(pw), 1) if pw else None, "source": self.source}
 
 
 # ------------------------------------------------------------------ oracle sample (CPU baseline / reference arm)
