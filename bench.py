@@ -206,8 +206,10 @@ class ClockSampler:
         if self._thread is not None:
             self._thread.join(timeout=5)
 
-    def summary(self, t0: float, t1: float):
-        rows = [v for (t, *v) in self.samples if t0 <= t <= t1 + self.PERIOD_S]
+    def summary(self, t0: float, t1: float, windows=None):
+        """Samples taken in [t0, t1] (or in any of the (start, end) ``windows``)."""
+        spans = windows if windows is not None else [(t0, t1)]
+        rows = [v for (t, *v) in self.samples if any(a <= t <= b + self.PERIOD_S for a, b in spans)]
         if not rows:
             rows = [v for (_, *v) in self.samples[-5:]]
         if not rows:
@@ -364,13 +366,17 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     check_errors("during warm-up")
 
-    # ---- timed region: device-resident inputs, nothing but the step's own launches on the stream
+    # ---- timed region: device-resident inputs, nothing but the step's own launches on the stream,
+    # plus two events per step around the dominant kernel (the MLP up-projection GEMM), whose
+    # launch durations the roofline line reports
+    dom = "gemm_up"
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(1.0)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
+    ops.profile_enable(2 * args.steps + 8, kernels=[dom])
     w0 = time.time()
     ev0.record(stream)
     for _ in range(args.steps):
@@ -380,20 +386,35 @@ def run_ours(args, rank, world, local_rank):
     w1 = time.time()
     barrier()
     clocks.stop()
+    ops.profile_disable()
+    dom_records = [t for n, t in ops.profile_read(2 * args.steps + 8) if n == dom]
     ms = max_over_ranks(ev0.elapsed_time(ev1))
     check_errors("in the timed region")
 
-    # ---- per-kernel device times: the same steps again with the library's launch events, which
-    # sit between the kernels and so also stop each kernel from starting during its predecessor's
-    # tail (the un-instrumented run above lets them)
+    # ---- per-kernel device times: for each kernel, the same steps again with launch events around
+    # that kernel's launches only (an event between two kernels stops the second from starting
+    # during the first one's tail, so bracketing one kernel at a time keeps the rest of the step as
+    # it runs in the timed region).  Each pass starts after the same one-second idle as the timed
+    # region: back to back, the passes run the GPU into its power cap within ~0.1 s (SM clock
+    # ~1.6 GHz, sw_power_cap), and their times would not describe the timed steps.
     prof_steps = max(3, min(args.steps, 20))
-    ops.profile_enable(prof_steps * 24 + 64)
-    for _ in range(prof_steps):
-        step()
-    torch.cuda.synchronize(dev)
-    ops.profile_disable()
-    records = ops.profile_read(prof_steps * 24 + 64)
+    records = []
+    kclocks = ClockSampler(local_rank)
+    kclocks.start()
+    kw = []
+    for tag in ops.KERNEL_TAGS.values():
+        time.sleep(1.0)
+        kw.append(time.time())
+        ops.profile_enable(prof_steps * 8 + 16, kernels=[tag])
+        for _ in range(prof_steps):
+            step()
+        torch.cuda.synchronize(dev)
+        ops.profile_disable()
+        records += ops.profile_read(prof_steps * 8 + 16)
+        kw.append(time.time())
+    kclocks.stop()
     check_errors("in the profiled steps")
+    kclk = kclocks.summary(0.0, 0.0, windows=list(zip(kw[0::2], kw[1::2])))
 
     # ---- end to end through the public calls: pinned host inputs in, results out, every step.
     # Two buffer sets: while the compute stream runs step i on one set, a copy stream fills the
@@ -437,6 +458,7 @@ def run_ours(args, rank, world, local_rank):
     for i in range(2):
         e2e_step(i)
     torch.cuda.synchronize(dev)
+    time.sleep(1.0)  # the same idle before the timed steps as the device-resident timed region
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s_in)
@@ -494,9 +516,9 @@ def run_ours(args, rank, world, local_rank):
         if "tflops" in k:
             k["frac"] = round(k["tflops"] / peak_tc, 4)
         kernels[n] = k
-    # dominant kernel: the MLP up-projection GEMM (largest share of the step)
-    dom = "gemm_up"
-    cnt, t = per.get(dom, (0, 0.0))
+    # dominant kernel: the MLP up-projection GEMM (largest share of the step), its launches inside
+    # the timed region
+    cnt, t = len(dom_records), float(sum(dom_records))
     achieved = gf[dom] * cnt / (t / 1e3) / 1e12 if t > 0 else None
     gemm_names = [n for n in gf if n in per]
     gemm_ms = sum(per[n][1] for n in gemm_names)
@@ -529,10 +551,12 @@ def run_ours(args, rank, world, local_rank):
                          "sustained (kernels timed over >= 1 s)" if sustained else
                          f"burst (kernels timed over {prof_region_ms:.0f} ms, under the power cap's time scale)"),
                      "flops_per_launch": gf[dom], "launches": cnt, "ms_avg": round(t / cnt, 5) if cnt else None,
+                     "timed_in": "the timed region (events around this kernel only)",
                      "all_gemms_tflops": round(gemm_all, 1) if gemm_all else None,
                      "all_gemms_frac": round(gemm_all / peak_tc, 4) if gemm_all else None},
         "kernels": kernels,
-        "kernels_from": f"{prof_steps} instrumented steps after the timed ones",
+        "kernels_from": f"{prof_steps} steps per kernel after the timed ones, events around that kernel's launches only",
+        "kernels_clocks": kclk,
         "gpu_launches": len(records) // prof_steps * args.steps,
         "clocks": clk,
         "e2e": {"value": round(s.seq * e2e_steps * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
@@ -574,6 +598,7 @@ def measure_c2048(ops, weights, dev, stream):
     for _ in range(2):
         run()
     torch.cuda.synchronize(dev)
+    time.sleep(1.0)  # the same idle before the timed reps as the step's timed region
     reps = 5
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -582,7 +607,8 @@ def measure_c2048(ops, weights, dev, stream):
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     ms = ev0.elapsed_time(ev1) / reps
-    ops.profile_enable(64)
+    time.sleep(1.0)
+    ops.profile_enable(64, kernels=["attention"])  # events around the attention launches only
     for _ in range(3):
         run()
     torch.cuda.synchronize(dev)
@@ -596,7 +622,7 @@ def measure_c2048(ops, weights, dev, stream):
     if att:
         out["attention_ms"] = round(att[1] / att[0], 4)
         out["attention_tflops"] = round(att_fl / (att[1] / att[0] / 1e3) / 1e12, 1)
-        out["attention_share"] = round(att[1] / sum(v[1] for v in per.values()), 4)
+        out["attention_share"] = round(att[1] / att[0] / ms, 4)
     del x2, y2, ws2
     return out
 
@@ -615,6 +641,7 @@ def measure_w8a8(ops, cfg, weights, x_in, ws, dev, stream):
     for _ in range(3):
         run()
     torch.cuda.synchronize(dev)
+    time.sleep(1.0)  # the same idle before the timed reps as the step's timed region
     reps = 10
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -623,7 +650,8 @@ def measure_w8a8(ops, cfg, weights, x_in, ws, dev, stream):
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     ms = ev0.elapsed_time(ev1) / reps
-    ops.profile_enable(64)
+    time.sleep(1.0)
+    ops.profile_enable(64, kernels=["gemm_qkv", "gemm_up"])  # events around these two only
     for _ in range(3):
         run()
     torch.cuda.synchronize(dev)

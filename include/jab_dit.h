@@ -307,6 +307,11 @@ typedef enum {
   DIT_KERNEL_COND_REDUCE = 12
 } dit_kernel_tag;
 DIT_API int dit_profile_enable(int max_marks);
+/* As dit_profile_enable, but only the launches whose tag t has bit (1u << t) set in tag_mask
+ * are bracketed (e.g. 1u << DIT_KERNEL_GEMM_UP: two events per block, around the MLP
+ * up-projection only, so the other kernels keep their back-to-back launches).  The records
+ * read back are those launches alone.  INVALID_ARG for max_marks <= 0 or an empty mask. */
+DIT_API int dit_profile_enable_tags(int max_marks, uint32_t tag_mask);
 DIT_API int dit_profile_disable(void);
 DIT_API int dit_profile_read(int* tags, float* ms, int max_records);
 

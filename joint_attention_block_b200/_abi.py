@@ -95,6 +95,7 @@ SIGNATURES = {
     "dit_joint_attention": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
     "dit_poll_error": (_I, [_P]),
     "dit_profile_enable": (_I, [_I]),
+    "dit_profile_enable_tags": (_I, [_I, ctypes.c_uint32]),
     "dit_profile_disable": (_I, []),
     "dit_profile_read": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float), _I]),
     "dit_set_wait_timeout_ms": (_I, [ctypes.c_uint32]),
@@ -343,8 +344,17 @@ KERNEL_TAGS = {1: "rope_table", 2: "rmsnorm", 3: "gemm_qkv", 4: "qknorm_mrope", 
                12: "cond_reduce"}
 
 
-def profile_enable(max_marks: int) -> None:
-    _check("dit_profile_enable", lib().dit_profile_enable(max_marks))
+def profile_enable(max_marks: int, kernels=None) -> None:
+    """Bracket every launch (``kernels`` None) or only the launches of the named kernels
+    (names as in KERNEL_TAGS) with CUDA events."""
+    if kernels is None:
+        _check("dit_profile_enable", lib().dit_profile_enable(max_marks))
+        return
+    ids = {v: k for k, v in KERNEL_TAGS.items()}
+    mask = 0
+    for name in kernels:
+        mask |= 1 << ids[name]
+    _check("dit_profile_enable_tags", lib().dit_profile_enable_tags(max_marks, mask))
 
 
 def profile_disable() -> None:

@@ -73,14 +73,17 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base
 
 // ------------------------------------------------------------------ launch instrumentation
 
-// When enabled, every launch of the three calls is bracketed by CUDA events on
-// its stream (tag = which kernel), so a caller can read per-kernel device time
-// of the very launches it timed.  Off by default; events are created once, at
-// enable time.
+// When enabled, every launch of the three calls whose tag is in the mask is bracketed by
+// CUDA events on its stream (tag = which kernel), so a caller can read per-kernel device
+// time of the very launches it timed.  A mark starts the kernel launched after it and ends
+// the one before it: an END event is recorded only where a bracketed kernel is followed by
+// one that is not.  Off by default; events are created once, at enable time.
 struct ProfState {
   bool on = false;
   int cap = 0;
   int n = 0;
+  uint32_t mask = 0xFFFFFFFFu;
+  bool open = false;  // the last recorded event starts a bracketed kernel
   cudaEvent_t* ev = nullptr;
   int* tag = nullptr;
 };
@@ -90,10 +93,13 @@ static std::mutex g_prof_mu;
 void prof_mark(cudaStream_t s, int tag) {
   if (!g_prof.on) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
+  const bool want = tag != DIT_KERNEL_END && tag < 32 && ((g_prof.mask >> tag) & 1u) != 0u;
+  if (!want && !g_prof.open) return;  // nothing to end, nothing to start
   if (g_prof.n >= g_prof.cap) return;
   cudaEventRecord(g_prof.ev[g_prof.n], s);
-  g_prof.tag[g_prof.n] = tag;
+  g_prof.tag[g_prof.n] = want ? tag : DIT_KERNEL_END;
   ++g_prof.n;
+  g_prof.open = want;
 }
 
 }  // namespace jab
@@ -189,9 +195,11 @@ int dit_abi_version(void) { return 2; }
 
 int dit_last_cuda_error(void) { return g_last_cuda_error.load(); }
 
-int dit_profile_enable(int max_marks) {
+int dit_profile_enable(int max_marks) { return dit_profile_enable_tags(max_marks, 0xFFFFFFFFu); }
+
+int dit_profile_enable_tags(int max_marks, uint32_t tag_mask) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  if (max_marks <= 0) return DIT_ERR_INVALID_ARG;
+  if (max_marks <= 0 || tag_mask == 0u) return DIT_ERR_INVALID_ARG;
   if (g_prof.cap < max_marks) {
     for (int i = 0; i < g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
     delete[] g_prof.ev;
@@ -206,6 +214,8 @@ int dit_profile_enable(int max_marks) {
     g_prof.cap = max_marks;
   }
   g_prof.n = 0;
+  g_prof.mask = tag_mask;
+  g_prof.open = false;
   g_prof.on = true;
   return DIT_OK;
 }

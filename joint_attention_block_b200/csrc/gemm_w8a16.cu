@@ -39,9 +39,11 @@
 //               last stage, the epilogue: thread = one token row of TMEM (warp w reads
 //               lanes 32*(w%4).., accumulator (w-2)/4), scale, optional GELU, optional
 //               residual (TMA-loaded boxes), 32 x 32 output boxes stored by TMA.  The
-//               boxes live in the widened ring (idle until these same warps convert
-//               the next unit) and a small extra region.  The next unit's MMAs wait
-//               for both CTAs' converters, hence for both epilogues to have read TMEM.
+//               output boxes live in the widened ring (idle until these same warps
+//               convert the next unit); the channel scales and the first residual
+//               boxes live past it and are fetched while the unit's last MMAs run.
+//               The next unit's MMAs wait for both CTAs' converters, hence for both
+//               epilogues to have read TMEM.
 #include <string.h>
 
 #include "common.cuh"
@@ -69,14 +71,17 @@ constexpr int MAX_PAIRS = 74;  // 148 SMs / 2
 constexpr int OFF_X = 0;
 constexpr int OFF_W8 = OFF_X + RAW_STAGES * X_BYTES;
 constexpr int OFF_W16 = OFF_W8 + RAW_STAGES * W8_BYTES;
-// Epilogue boxes of 32 tokens x 32 channels, per epilogue warp two output boxes and two
-// residual boxes (2 KB each in 16-bit, 4 KB in fp32): at most 12 KB per warp (fp32 out
-// with an fp32 residual keeps one output box).  They start at the widened ring and run
-// 32 KB past it.
-constexpr int EPI_WARP_BYTES = 12 * 1024;
+// Epilogue boxes of 32 tokens x 32 channels (2 KB in 16-bit, 4 KB in fp32).  Per epilogue
+// warp: 8 KB over the widened ring for its two output boxes (one when both the output and
+// the residual are fp32) and, with an fp32 residual, its second residual box; 4 KB past the
+// ring for the first residual box(es) (both 16-bit boxes, or the first fp32 box), which can
+// therefore be loaded while the unit's last MMAs still read the ring.
+constexpr int EPI_RING_WARP = 8 * 1024;
+constexpr int EPI_EXTRA_WARP = 4 * 1024;
 constexpr int OFF_EPI = OFF_W16;
-constexpr int OFF_SCALE = OFF_EPI + CVT_WARPS * EPI_WARP_BYTES;  // per epilogue warp, 256 scales
-static_assert(OFF_SCALE >= OFF_W16 + CVT_STAGES * W16_BYTES, "epilogue region covers the widened ring");
+constexpr int OFF_EPI_EXTRA = OFF_W16 + CVT_STAGES * W16_BYTES;
+constexpr int OFF_SCALE = OFF_EPI_EXTRA + CVT_WARPS * EPI_EXTRA_WARP;  // per epilogue warp, 256 scales
+static_assert(CVT_WARPS * EPI_RING_WARP <= CVT_STAGES * W16_BYTES, "output boxes fit over the widened ring");
 constexpr int OFF_BAR = OFF_SCALE + CVT_WARPS * BN_MMA * 4;
 constexpr int NUM_BARS = 3 * RAW_STAGES + 2 * CVT_STAGES + 3 + 2 * CVT_WARPS;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -267,12 +272,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int acc = ew >> 2;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN_MMA;
     float* sScale = reinterpret_cast<float*>(smem + OFF_SCALE) + ew * BN_MMA;
+    const bool has_res = p.res_fmt >= 0;
+    const bool res32 = p.res_fmt == FMT_F32;
     const int out_box = 32 * 32 * (p.y_fmt == FMT_F32 ? 4 : 2);
-    const int res_box = p.res_fmt < 0 ? 0 : 32 * 32 * (p.res_fmt == FMT_F32 ? 4 : 2);
-    // two output boxes, except fp32 out with an fp32 residual, which gets one so that the
-    // warp's boxes stay within EPI_WARP_BYTES
-    const int n_out = 2 * (out_box + res_box) <= EPI_WARP_BYTES ? 2 : 1;
-    uint8_t* ebox = smem + OFF_EPI + ew * EPI_WARP_BYTES;  // out boxes, then residual 0, residual 1
+    const int res_box = has_res ? 32 * 32 * (res32 ? 4 : 2) : 0;
+    // two output boxes, except fp32 out with an fp32 residual (whose second box shares the
+    // warp's ring part), which gets one
+    const int n_out = 2 * out_box + (res32 ? res_box : 0) <= EPI_RING_WARP ? 2 : 1;
+    uint8_t* const ebox = smem + OFF_EPI + ew * EPI_RING_WARP;  // output boxes [, fp32 residual box 1]
+    uint8_t* const rbox0 = smem + OFF_EPI_EXTRA + ew * EPI_EXTRA_WARP;
+    uint8_t* const rbox1 = res32 ? ebox + n_out * out_box : rbox0 + res_box;
+    const int n_early = res32 ? 1 : 2;  // residual boxes past the ring
     uint64_t* rbar = res_full + 2 * ew;
     uint32_t rph = 0u;  // bit b: phase parity of residual box b
     bool ok = true;
@@ -327,29 +337,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       // writes the result row by row into a swizzled output box and hands the box to a
       // TMA store.  The residual boxes of the next two chunks and the stores of the last
       // two are in flight while a chunk is computed.
-      if (!mbar_wait(acc_full, static_cast<uint32_t>(ui) & 1u, guard, abort_flag,
-                     where_code(ERR_TIMEOUT_GEMM_EPILOGUE, rank, ui))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
       const int tok_warp = w.tok_cta + quarter * 32;
       const int ch_warp = w.tile_n * BN + acc * BN_MMA;
       // valid chunks (N % 32 == 0); none when all 32 of the warp's tokens lie beyond M
       const int nch = tok_warp < p.M ? min(BN_MMA, p.N - ch_warp) / 32 : 0;
-      {  // this warp's 256 channel scales
+      {  // this warp's 256 channel scales, loaded while the unit's last MMAs run
         const int n0 = ch_warp + 8 * lane;
 #pragma unroll
         for (int k = 0; k < 8; ++k) sScale[8 * lane + k] = n0 + k < p.N ? p.scale[n0 + k] : 0.f;
       }
-      __syncwarp();
-      const bool has_res = p.res_fmt >= 0;
       auto issue_res = [&](int c) {
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&rbar[c & 1], static_cast<uint32_t>(res_box));
-        tma_load_2d(ebox + n_out * out_box + (c & 1) * res_box, &tm_r, &rbar[c & 1], ch_warp + 32 * c, tok_warp);
+        tma_load_2d((c & 1) ? rbox1 : rbox0, &tm_r, &rbar[c & 1], ch_warp + 32 * c, tok_warp);
       };
+      // the residual boxes past the ring are loaded while the unit's last MMAs run
       int res_issued = 0;
+      if (has_res && lane == 0) {
+        for (; res_issued < min(n_early, nch); ++res_issued) issue_res(res_issued);
+      }
+      if (!mbar_wait(acc_full, static_cast<uint32_t>(ui) & 1u, guard, abort_flag,
+                     where_code(ERR_TIMEOUT_GEMM_EPILOGUE, rank, ui))) {
+        ok = false;
+        if (lane == 0) {  // no residual load left in flight
+          for (int k = 0; k < res_issued; ++k) {
+            mbar_wait(&rbar[k & 1], (rph >> (k & 1)) & 1u, guard, abort_flag,
+                      where_code(ERR_TIMEOUT_GEMM_DRAIN, rank, 0x200 + k), true);
+            rph ^= 1u << (k & 1);
+          }
+        }
+        __syncwarp();
+        break;
+      }
+      tc_fence_after();
+      __syncwarp();
       if (has_res && lane == 0) {
         for (; res_issued < min(2, nch); ++res_issued) issue_res(res_issued);
       }
@@ -383,8 +404,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             break;
           }
           rph ^= 1u << bx;
-          const uint8_t* rrow = ebox + n_out * out_box + bx * res_box;
-          if (p.res_fmt == FMT_F32) {  // 128-byte rows, 128-byte swizzle
+          const uint8_t* rrow = bx ? rbox1 : rbox0;
+          if (res32) {  // 128-byte rows, 128-byte swizzle
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 t = *reinterpret_cast<const float4*>(rrow + lane * 128 + ((q ^ (lane & 7)) << 4));

@@ -202,3 +202,22 @@ def test_stack_of_34_tiny_blocks_against_oracle():
     ref = oracle.dit_stack_forward(s, wsets, x_bits, s.n_text, s.grid_h, s.grid_w)
     k = float(np.sqrt(n))
     assert_close(as_f64(got), ref, max_rel=2e-2 * k, mean_rel=3e-3 * k, what="34-block stack")
+
+
+def test_profile_brackets_only_the_selected_kernels():
+    """Launch events around selected kernels only: one record per selected launch, none for the
+    others; with no selection every launch of the block is recorded."""
+    s = synth.TINY
+    inp = synth.block_inputs(s)
+    ops.profile_enable(64, kernels=["gemm_up", "attention"])
+    run_block(s, inp)
+    ops.profile_disable()
+    rec = ops.profile_read(64)
+    assert sorted(n for n, _ in rec) == ["attention", "gemm_up"]
+    assert all(ms > 0 for _, ms in rec)
+    ops.profile_enable(64)
+    run_block(s, inp)
+    ops.profile_disable()
+    names = [n for n, _ in ops.profile_read(64)]
+    for n in ("rope_table", "rmsnorm", "gemm_qkv", "qknorm_mrope", "attention", "gemm_o", "gemm_up", "gemm_down"):
+        assert n in names, (n, names)
