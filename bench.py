@@ -402,7 +402,7 @@ def run_ours(args, rank, world, local_rank):
     kclocks = ClockSampler(local_rank)
     kclocks.start()
     kw = []
-    for tag in ops.KERNEL_TAGS.values():
+    for tag in [n for n in ops.KERNEL_TAGS.values() if n != "rope_table"]:  # rope: inside the QK-norm kernel
         time.sleep(1.0)
         kw.append(time.time())
         ops.profile_enable(prof_steps * 8 + 16, kernels=[tag])

@@ -267,8 +267,9 @@ DIT_API int dit_rmsnorm_rows_e4m3(const void* x, int x_fmt, const void* g, uint8
 
 /* Per-head QK-RMSNorm + 3D M-RoPE, in place on a fused qkv buffer [batch, S, 3d] in fmt
  * (BF16 or F16; Q columns [0, d), K columns [d, 2d); V untouched).  pos: int32 [S, 3] or
- * NULL (derived from n_text/grid/t_img as in dit_block_forward).  workspace holds the
- * fp32 cos/sin tables: >= 2 * align256(S * head_dim/2 * 4) bytes. */
+ * NULL (derived from n_text/grid/t_img as in dit_block_forward).  The rotary angles are
+ * computed inside the kernel (exact fp64 product, fp64 reduction modulo 2 pi, fp32 cosine and
+ * sine); workspace and ws_bytes are not used and may be NULL / 0. */
 DIT_API int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                      const dit_block_config* cfg, const void* g_q, const void* g_k, void* workspace,
                      size_t ws_bytes, void* stream);
@@ -293,7 +294,7 @@ DIT_API int dit_poll_error(void* stream);
  * on error), then clears the record. */
 typedef enum {
   DIT_KERNEL_END = 0,
-  DIT_KERNEL_ROPE_TABLE = 1,
+  DIT_KERNEL_ROPE_TABLE = 1, /* no longer launched: the angles are computed by the QK-norm kernel */
   DIT_KERNEL_RMSNORM = 2,
   DIT_KERNEL_GEMM_QKV = 3,
   DIT_KERNEL_QKNORM_MROPE = 4,

@@ -140,8 +140,6 @@ int check_config(const dit_block_config* c) {
 // The rotary tables hold one [S, hd/2] pair per batch element (padded batches position each
 // element on its own; otherwise only the first is used) and kv_len the per-element key counts.
 struct BlockWorkspace {
-  float* cos_tab;
-  float* sin_tab;
   int32_t* kv_len;
   uint16_t* h;
   uint16_t* qkv;
@@ -155,21 +153,19 @@ struct BlockWorkspace {
 BlockWorkspace carve_block(const dit_block_config* c, int batch, int seq, void* base) {
   BlockWorkspace w{};
   const size_t M = static_cast<size_t>(batch) * seq;
-  const size_t d = c->d_model, F = c->d_mlp, half = c->head_dim / 2;
+  const size_t d = c->d_model, F = c->d_mlp;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off += align256(bytes);
     return o;
   };
-  const size_t o_cos = take(M * half * 4), o_sin = take(M * half * 4), o_kv = take(static_cast<size_t>(batch) * 4);
+  const size_t o_kv = take(static_cast<size_t>(batch) * 4);
   const size_t o_h = take(M * d * 2), o_qkv = take(M * 3 * d * 2), o_o = take(M * d * 2), o_x1 = take(M * d * 4);
   const size_t o_u = take(M * F * 2), o_sa = take(M * 4);
   w.bytes = off;
   if (base != nullptr) {
     uint8_t* b = static_cast<uint8_t*>(base);
-    w.cos_tab = reinterpret_cast<float*>(b + o_cos);
-    w.sin_tab = reinterpret_cast<float*>(b + o_sin);
     w.kv_len = reinterpret_cast<int32_t*>(b + o_kv);
     w.h = reinterpret_cast<uint16_t*>(b + o_h);
     w.qkv = reinterpret_cast<uint16_t*>(b + o_qkv);
@@ -354,18 +350,14 @@ int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int 
     return DIT_ERR_INVALID_ARG;
   if (fmt != FMT_BF16 && fmt != FMT_F16) return DIT_ERR_INVALID_ARG;
   const int S = n_text + grid_h * grid_w;
-  const size_t need = 2 * align256(static_cast<size_t>(S) * (cfg->head_dim / 2) * 4);
-  if (workspace == nullptr || ws_bytes < need) return DIT_ERR_WORKSPACE;
-  float* cos_tab = static_cast<float*>(workspace);
-  float* sin_tab = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + need / 2);
+  (void)workspace;  // the rotary angles are computed in the kernel; no scratch is needed
+  (void)ws_bytes;
   cudaStream_t s = as_stream(stream);
-  prof_mark(s, DIT_KERNEL_ROPE_TABLE);
-  cudaError_t e = launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections,
-                                    cfg->rope_theta, cos_tab, sin_tab, s);
-  if (e != cudaSuccess) return DIT_ERR_CUDA;
   prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
-  e = launch_qknorm_mrope(qkv, fmt, batch, S, cfg->n_heads, cfg->head_dim, cos_tab, sin_tab,
-                          static_cast<const uint16_t*>(g_q), static_cast<const uint16_t*>(g_k), cfg->eps, false, s);
+  cudaError_t e = launch_qknorm_mrope(qkv, fmt, batch, S, cfg->n_heads, cfg->head_dim, n_text, grid_w,
+                                      grid_h * grid_w, t_img, pos, nullptr, nullptr, cfg->rope_sections,
+                                      cfg->rope_theta, static_cast<const uint16_t*>(g_q),
+                                      static_cast<const uint16_t*>(g_k), cfg->eps, s);
   prof_mark(s, DIT_KERNEL_END);
   return from_cuda(e);
 }
@@ -426,13 +418,6 @@ int block_forward(const dit_block_config* cfg, const dit_block_weights* w, const
     if (jab_e != cudaSuccess) return from_cuda(jab_e); \
   } while (0)
   const bool padded = text_lens != nullptr;
-  prof_mark(s, DIT_KERNEL_ROPE_TABLE);
-  if (padded)
-    JAB_TRY(launch_rope_table_padded(batch, n_text, grid_h, grid_w, t_img, text_lens, cfg->head_dim,
-                                     cfg->rope_sections, cfg->rope_theta, ws.cos_tab, ws.sin_tab, ws.kv_len, s));
-  else
-    JAB_TRY(launch_rope_table(n_text, grid_h, grid_w, t_img, pos, cfg->head_dim, cfg->rope_sections,
-                              cfg->rope_theta, ws.cos_tab, ws.sin_tab, s));
   const uint16_t* g1 = static_cast<const uint16_t*>(w->g_norm1);
   const uint16_t* g2 = static_cast<const uint16_t*>(w->g_norm2);
   uint8_t* h8 = reinterpret_cast<uint8_t*>(ws.h);  // e4m3 codes of the W8A8 variant
@@ -448,9 +433,10 @@ int block_forward(const dit_block_config* cfg, const dit_block_weights* w, const
     JAB_TRY(launch_gemm_w8a16(
         GemmArgs{ws.h, FMT_F16, w->w_qkv, w->s_qkv, ws.qkv, FMT_F16, nullptr, -1, M, 3 * d, d, 0, 0}, g, s));
   prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
-  JAB_TRY(launch_qknorm_mrope(ws.qkv, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, ws.cos_tab, ws.sin_tab,
-                              static_cast<const uint16_t*>(w->g_q), static_cast<const uint16_t*>(w->g_k), cfg->eps,
-                              padded, s));
+  JAB_TRY(launch_qknorm_mrope(ws.qkv, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, n_text, grid_w,
+                              grid_h * grid_w, t_img, pos, text_lens, padded ? ws.kv_len : nullptr,
+                              cfg->rope_sections, cfg->rope_theta, static_cast<const uint16_t*>(w->g_q),
+                              static_cast<const uint16_t*>(w->g_k), cfg->eps, s));
   prof_mark(s, DIT_KERNEL_ATTENTION);
   JAB_TRY(launch_attention(ws.qkv, ws.o, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, padded ? ws.kv_len : nullptr,
                            g, s));

@@ -2,6 +2,8 @@
 // CFG + Euler update, the 3D M-RoPE position / angle tables and the standalone
 // per-head QK-RMSNorm + M-RoPE.  All loads and stores are 16-byte vectors where
 // the layout allows; math is fp32.
+#include <cmath>
+
 #include "common.cuh"
 
 namespace jab {
@@ -60,7 +62,8 @@ __device__ float block_sum(float v, float* red) {
 
 // One CTA per row.  kVec 8-element vectors per thread are kept in registers
 // between the two passes when the row fits (cols <= kThreads*8*kVec); longer
-// rows (the 53,248-wide conditioning features) are re-read from L2.
+// rows (the 53,248-wide conditioning features) are re-read from L2, four vectors
+// per thread in flight in each pass.
 // XF: input format (bf16 or fp32), YF: output format (bf16 or f16).
 template <int kThreads, int kVec, int XF, int YF>
 __global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const void* x, const uint16_t* __restrict__ g, void* y,
@@ -96,7 +99,7 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const void* x, const 
       for (int k = 0; k < 8; ++k) o[k] = v[j][k] * rstd * gv[k];
       store8<YF>(y, row8 + i, o);
     }
-  } else {
+  } else if constexpr (XF == FMT_F32) {
     for (int64_t i = threadIdx.x; i < nv; i += kThreads) {
       float v[8];
       load8<XF>(x, row8 + i, v);
@@ -111,6 +114,55 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const void* x, const 
 #pragma unroll
       for (int k = 0; k < 8; ++k) o[k] = v[k] * rstd * gv[k];
       store8<YF>(y, row8 + i, o);
+    }
+  } else {
+    // 16-bit rows: U raw 16-byte vectors per thread in flight in each pass, unpacked as used
+    constexpr int U = 4;
+    const uint4* xr = reinterpret_cast<const uint4*>(x) + row8;
+    const uint4* gr = reinterpret_cast<const uint4*>(g);
+    for (int64_t i0 = threadIdx.x; i0 < nv; i0 += U * kThreads) {
+      uint4 raw[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t i = i0 + static_cast<int64_t>(u) * kThreads;
+        raw[u] = i < nv ? xr[i] : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float a = unpack_lo<XF>(w[k]), b2 = unpack_hi<XF>(w[k]);
+          ss = fmaf(a, a, fmaf(b2, b2, ss));
+        }
+      }
+    }
+    const float rstd = rsqrtf(block_sum<kThreads>(ss, red) / static_cast<float>(cols) + eps);
+    for (int64_t i0 = threadIdx.x; i0 < nv; i0 += U * kThreads) {
+      uint4 raw[U], graw[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t i = i0 + static_cast<int64_t>(u) * kThreads;
+        if (i < nv) {
+          raw[u] = xr[i];
+          graw[u] = gr[i];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t i = i0 + static_cast<int64_t>(u) * kThreads;
+        if (i < nv) {
+          const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+          const uint32_t gw[4] = {graw[u].x, graw[u].y, graw[u].z, graw[u].w};
+          float o[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            o[2 * k] = unpack_lo<XF>(w[k]) * rstd * unpack_lo<FMT_BF16>(gw[k]);
+            o[2 * k + 1] = unpack_hi<XF>(w[k]) * rstd * unpack_hi<FMT_BF16>(gw[k]);
+          }
+          store8<YF>(y, row8 + i, o);
+        }
+      }
     }
   }
 }
@@ -375,6 +427,16 @@ cudaError_t launch_denoise_update(float* z, const uint16_t* out_c, const uint16_
 // ------------------------------------------------------------------ positions and angle tables
 
 // Text token j -> (j, j, j); image cell (r, c) in raster order -> (t_img, r, c).
+// Positions and inverse frequencies of the rotary embedding, passed by value to the QK-norm kernel.
+struct RopeArgs {
+  int n_text, grid_w, n_img, t_img;  // t_img < 0: n_text (or L_b in a padded batch)
+  const int32_t* pos;                // [S, 3] or NULL (ignored when text_lens is given)
+  const int32_t* text_lens;          // [batch] or NULL
+  int32_t* kv_len;                   // [batch], written when text_lens is given
+  int sec_t, sec_h;                  // rotary pairs on the t and h axes (w takes the rest)
+  float inv_freq[64];                // fp32(theta^(-2i/hd)), i < hd/2
+};
+
 __device__ __forceinline__ void token_position(int s, int n_text, int grid_w, int t_img, const int32_t* pos, int& pt,
                                                int& ph, int& pw) {
   if (pos != nullptr) {
@@ -409,110 +471,37 @@ cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int3
   return cudaGetLastError();
 }
 
-// cos/sin of angle(s, i) = pos[s][axis(i)] * inv_freq_i for the hd/2 rotary pairs.
-// inv_freq_i = fp32(theta^(-2i/hd)); the product and the trig are evaluated in
-// fp64 and rounded once to fp32.
-__global__ void rope_table_kernel(int S, int n_text, int grid_w, int t_img, const int32_t* pos, int half,
-                                  int sec_t, int sec_h, double theta, float* cos_tab, float* sin_tab) {
-  pdl_wait_then_release();
-  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (idx >= static_cast<int64_t>(S) * half) return;
-  const int s = static_cast<int>(idx / half);
-  const int i = static_cast<int>(idx - static_cast<int64_t>(s) * half);
-  int pt, ph, pw;
-  token_position(s, n_text, grid_w, t_img, pos, pt, ph, pw);
-  const int p = i < sec_t ? pt : (i < sec_t + sec_h ? ph : pw);
-  const float inv = static_cast<float>(pow(theta, -2.0 * i / (2.0 * half)));
-  double sn, cs;
-  sincos(static_cast<double>(p) * static_cast<double>(inv), &sn, &cs);
-  cos_tab[idx] = static_cast<float>(cs);
-  sin_tab[idx] = static_cast<float>(sn);
-}
+// ------------------------------------------------------------------ QK-RMSNorm + M-RoPE
 
-// Padded batches of prompts: element b holds L_b = clamp(text_lens[b], 0, n_text) text rows,
-// then its grid_h*grid_w image rows, then padding up to S.  Each element is positioned as if
-// alone: text j at (j, j, j), image cell (r, c) at (t_b, r, c) with t_b = L_b (or t_img when
-// t_img >= 0), padding rows at (0, 0, 0).  The tables are [batch, S, hd/2]; the (b, 0, 0) thread
-// also writes the element's key count L_b + grid_h*grid_w to kv_len[b].
-__global__ void rope_table_padded_kernel(int batch, int S, int n_text, int grid_w, int n_img, int t_img,
-                                         const int32_t* __restrict__ text_lens, int half, int sec_t, int sec_h,
-                                         double theta, float* cos_tab, float* sin_tab, int32_t* kv_len) {
-  pdl_wait_then_release();
-  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (idx >= static_cast<int64_t>(batch) * S * half) return;
-  const int64_t bs = idx / half;
-  const int i = static_cast<int>(idx - bs * half);
-  const int b = static_cast<int>(bs / S);
-  const int s = static_cast<int>(bs - static_cast<int64_t>(b) * S);
-  const int L = min(max(text_lens[b], 0), n_text);
-  if (s == 0 && i == 0) kv_len[b] = L + n_img;
-  int pt = 0, ph = 0, pw = 0;
-  if (s < L) {
-    pt = ph = pw = s;
-  } else if (s < L + n_img) {
-    const int k = s - L;
-    pt = t_img < 0 ? L : t_img;
-    ph = k / grid_w;
-    pw = k - ph * grid_w;
-  }
-  const int p = i < sec_t ? pt : (i < sec_t + sec_h ? ph : pw);
-  const float inv = static_cast<float>(pow(theta, -2.0 * i / (2.0 * half)));
-  double sn, cs;
-  sincos(static_cast<double>(p) * static_cast<double>(inv), &sn, &cs);
-  cos_tab[idx] = static_cast<float>(cs);
-  sin_tab[idx] = static_cast<float>(sn);
-}
-
-cudaError_t launch_rope_table_padded(int batch, int n_text, int grid_h, int grid_w, int t_img,
-                                     const int32_t* text_lens, int head_dim, const int32_t sections[3], float theta,
-                                     float* cos_tab, float* sin_tab, int32_t* kv_len, cudaStream_t s) {
-  const int S = n_text + grid_h * grid_w;
-  const int half = head_dim / 2;
-  const int64_t n = static_cast<int64_t>(batch) * S * half;
-  if (n <= 0) return cudaSuccess;
-  launch_pdl(rope_table_padded_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, batch, S, n_text,
-             grid_w, grid_h * grid_w, t_img, text_lens, half, sections[0], sections[1], static_cast<double>(theta),
-             cos_tab, sin_tab, kv_len);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, int head_dim,
-                              const int32_t sections[3], float theta, float* cos_tab, float* sin_tab,
-                              cudaStream_t s) {
-  const int S = n_text + grid_h * grid_w;
-  const int half = head_dim / 2;
-  const int64_t n = static_cast<int64_t>(S) * half;
-  if (n <= 0) return cudaSuccess;
-  if (t_img < 0) t_img = n_text;
-  launch_pdl(rope_table_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, S, n_text, grid_w, t_img,
-             pos, half, sections[0], sections[1], static_cast<double>(theta), cos_tab, sin_tab);
-  return cudaGetLastError();
-}
-
-// ------------------------------------------------------------------ QK-RMSNorm + M-RoPE (standalone)
-
-// One thread per (batch, token, head, 8 rotary pairs): it holds elements [8c, 8c+8) and
-// [half+8c, half+8c+8) of the head in both q and k as 16-byte vectors (four loads in
-// flight, one cos/sin fetch for both), so the hd/16 threads of one head are consecutive
-// lanes and reduce the two sums of squares with xor-shuffles.  F: storage format of the
-// qkv buffer (bf16 or f16).
-// tab_per_batch: the tables are [batch, seq, hd/2] (padded batches) rather than [seq, hd/2].
+// One CTA per (batch element b, token s).  The token's rotary angles come first: for pair i
+// (i < hd/2) the position on axis(i) (t for the first sec_t pairs, then h for sec_h, then w)
+// times inv_freq_i = fp32(theta^(-2i/hd)) (exact in fp64), reduced modulo 2 pi in fp64, and its
+// cosine and sine in fp32 (within a few fp32 ulps of the fp64 values), into shared memory.  Positions: text j at (j, j, j), image cell
+// (r, c) at (t_img, r, c), or the caller's pos[s]; in a padded batch (text_lens given) element
+// b has L_b = clamp(text_lens[b], 0, n_text) text rows, then its image rows at (t_b, r, c),
+// t_b = L_b (or t_img when t_img >= 0), then padding at (0, 0, 0), and the CTA of (b, 0) also
+// writes the element's key count L_b + n_img to kv_len[b].
+// Then one thread per (head, 8 rotary pairs): it holds elements [8c, 8c+8) and
+// [half+8c, half+8c+8) of the head in both q and k as 16-byte vectors (loaded before the
+// angles are computed), so the hd/16 threads of one head are consecutive lanes and reduce the
+// two sums of squares with xor-shuffles.  The CTA is a whole number of warps; lanes past the
+// last head shadow it so that the shuffles stay full.  F: storage format of the qkv buffer.
 template <int F>
-__global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int seq, int n_heads, int head_dim,
-                                    const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
-                                    const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps,
-                                    int tab_per_batch) {
+__global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int seq, int n_heads, int head_dim, RopeArgs ra,
+                                    const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
+  __shared__ float s_cos[64], s_sin[64];
   pdl_wait_then_release();
   const int half = head_dim / 2;
-  const int group = half / 8;  // threads per head: 8 (hd 128) or 4 (hd 64)
-  const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(batch) * seq * n_heads * group;
-  const bool live = tid < total;
-  const int64_t t = live ? tid : total - 1;  // dead lanes shadow the last head so the shuffles stay full
-  const int c = static_cast<int>(t % group);
-  const int h = static_cast<int>((t / group) % n_heads);
-  const int64_t bs = t / (group * n_heads);
-  const int s = static_cast<int>(bs % seq);
+  const int lg = head_dim == 128 ? 3 : 2;  // log2 of the threads per head: 8 (hd 128) or 4 (hd 64)
+  const int group = 1 << lg;
+  const int per_token = n_heads << lg;
+  const bool live = static_cast<int>(threadIdx.x) < per_token;
+  const int t = live ? static_cast<int>(threadIdx.x) : per_token - 1;
+  const int c = t & (group - 1);
+  const int h = t >> lg;
+  const int64_t bs = blockIdx.x;  // b * seq + s
+  const int b = static_cast<int>(bs / seq);
+  const int s = static_cast<int>(bs - static_cast<int64_t>(b) * seq);
   const int d = n_heads * head_dim;
   uint16_t* vq = qkv + bs * (3 * static_cast<int64_t>(d)) + h * head_dim;
   uint16_t* vk = vq + d;
@@ -521,10 +510,43 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int s
   load8<F>(vq + half + 8 * c, 0, qb);
   load8<F>(vk + 8 * c, 0, ka);
   load8<F>(vk + half + 8 * c, 0, kb);
+  {
+    int pt = 0, ph = 0, pw = 0;
+    if (ra.text_lens != nullptr) {
+      const int L = min(max(ra.text_lens[b], 0), ra.n_text);
+      if (s == 0 && threadIdx.x == 0) ra.kv_len[b] = L + ra.n_img;
+      if (s < L) {
+        pt = ph = pw = s;
+      } else if (s < L + ra.n_img) {
+        const int k = s - L;
+        pt = ra.t_img < 0 ? L : ra.t_img;
+        ph = k / ra.grid_w;
+        pw = k - ph * ra.grid_w;
+      }
+    } else {
+      token_position(s, ra.n_text, ra.grid_w, ra.t_img < 0 ? ra.n_text : ra.t_img, ra.pos, pt, ph, pw);
+    }
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+      const int p = i < ra.sec_t ? pt : (i < ra.sec_t + ra.sec_h ? ph : pw);
+      // the angle p * inv_freq_i is exact in fp64; it is reduced by the nearest multiple of 2 pi
+      // in fp64 (error ~1e-13 for the angles of any image), rounded once to fp32 in [-pi, pi],
+      // and its sine and cosine taken in fp32
+      const double x = static_cast<double>(p) * static_cast<double>(ra.inv_freq[i]);
+      const double k = rint(x * 0.15915494309189535);
+      const float r = static_cast<float>(fma(-k, 6.283185307179586, x));
+      float sn, cs;
+      sincosf(r, &sn, &cs);
+      s_cos[i] = cs;
+      s_sin[i] = sn;
+    }
+  }
+  __syncthreads();
   float cs[8], sn[8];
-  const int64_t trow = tab_per_batch ? bs : static_cast<int64_t>(s);
-  load8<FMT_F32>(cos_tab + trow * half + 8 * c, 0, cs);
-  load8<FMT_F32>(sin_tab + trow * half + 8 * c, 0, sn);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    cs[k] = s_cos[8 * c + k];
+    sn[k] = s_sin[8 * c + k];
+  }
   float sq = 0.f, sk = 0.f;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -567,20 +589,37 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int batch, int s
   }
 }
 
-cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
-                                const float* cos_tab, const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k,
-                                float eps, bool tab_per_batch, cudaStream_t s) {
-  const int tpb = tab_per_batch ? 1 : 0;
-  const int64_t threads = static_cast<int64_t>(batch) * seq * n_heads * (head_dim / 16);
-  if (threads <= 0) return cudaSuccess;
-  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim, int n_text,
+                                int grid_w, int n_img, int t_img, const int32_t* pos, const int32_t* text_lens,
+                                int32_t* kv_len, const int32_t sections[3], float theta, const uint16_t* g_q,
+                                const uint16_t* g_k, float eps, cudaStream_t s) {
+  const int64_t tokens = static_cast<int64_t>(batch) * seq;
+  if (tokens <= 0 || n_heads <= 0) return cudaSuccess;
+  if (head_dim != 64 && head_dim != 128) return cudaErrorInvalidValue;
+  if ((text_lens != nullptr) != (kv_len != nullptr)) return cudaErrorInvalidValue;
+  const int per_token = n_heads * (head_dim / 16);
+  if (per_token > 1024) return cudaErrorInvalidValue;
+  RopeArgs ra;
+  ra.n_text = n_text;
+  ra.grid_w = grid_w > 0 ? grid_w : 1;
+  ra.n_img = n_img;
+  ra.t_img = t_img;
+  ra.pos = pos;
+  ra.text_lens = text_lens;
+  ra.kv_len = kv_len;
+  ra.sec_t = sections[0];
+  ra.sec_h = sections[1];
+  for (int i = 0; i < head_dim / 2; ++i)
+    ra.inv_freq[i] = static_cast<float>(std::pow(static_cast<double>(theta), -2.0 * i / head_dim));
+  const unsigned threads = static_cast<unsigned>((per_token + 31) / 32 * 32);
+  const unsigned blocks = static_cast<unsigned>(tokens);
   uint16_t* q = static_cast<uint16_t*>(qkv);
   if (fmt == FMT_F16)
-    launch_pdl(qknorm_mrope_kernel<FMT_F16>, dim3(blocks), dim3(256), 0, s, q, batch, seq, n_heads, head_dim, cos_tab,
-               sin_tab, g_q, g_k, eps, tpb);
+    launch_pdl(qknorm_mrope_kernel<FMT_F16>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra, g_q,
+               g_k, eps);
   else if (fmt == FMT_BF16)
-    launch_pdl(qknorm_mrope_kernel<FMT_BF16>, dim3(blocks), dim3(256), 0, s, q, batch, seq, n_heads, head_dim, cos_tab,
-               sin_tab, g_q, g_k, eps, tpb);
+    launch_pdl(qknorm_mrope_kernel<FMT_BF16>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra, g_q,
+               g_k, eps);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

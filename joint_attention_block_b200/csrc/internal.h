@@ -73,19 +73,12 @@ cudaError_t launch_denoise_pack(const float* z, const uint16_t* text_c, const ui
 cudaError_t launch_denoise_update(float* z, const uint16_t* out_c, const uint16_t* out_u, int batch, int n_img, int d,
                                   int lc, int lu, float guidance, float dt, cudaStream_t s);
 cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int32_t* pos, cudaStream_t s);
-// cos/sin table [S, hd/2] fp32 each, from positions (derived when pos == nullptr).
-cudaError_t launch_rope_table(int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos, int head_dim,
-                              const int32_t sections[3], float theta, float* cos_tab, float* sin_tab,
-                              cudaStream_t s);
-// Per-element tables [batch, S, hd/2] and key counts kv_len [batch] of a padded batch of prompts
-// (text_lens: device int32 [batch], each clamped to [0, n_text]).
-cudaError_t launch_rope_table_padded(int batch, int n_text, int grid_h, int grid_w, int t_img,
-                                     const int32_t* text_lens, int head_dim, const int32_t sections[3], float theta,
-                                     float* cos_tab, float* sin_tab, int32_t* kv_len, cudaStream_t s);
-// tab_per_batch: cos/sin tables are [batch, seq, hd/2] rather than [seq, hd/2].
-cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
-                                const float* cos_tab, const float* sin_tab, const uint16_t* g_q, const uint16_t* g_k,
-                                float eps, bool tab_per_batch, cudaStream_t s);
+// Per-head QK-RMSNorm + 3D M-RoPE in place on the fused qkv buffer; the rotary angles of each
+// token are computed by the kernel from its position (text_lens / kv_len: padded batches).
+cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim, int n_text,
+                                int grid_w, int n_img, int t_img, const int32_t* pos, const int32_t* text_lens,
+                                int32_t* kv_len, const int32_t sections[3], float theta, const uint16_t* g_q,
+                                const uint16_t* g_k, float eps, cudaStream_t s);
 
 // Activation storage formats (the ABI's format codes).
 enum Fmt : int { FMT_BF16 = 0, FMT_F16 = 1, FMT_F32 = 2 };

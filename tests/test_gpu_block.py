@@ -219,5 +219,5 @@ def test_profile_brackets_only_the_selected_kernels():
     run_block(s, inp)
     ops.profile_disable()
     names = [n for n, _ in ops.profile_read(64)]
-    for n in ("rope_table", "rmsnorm", "gemm_qkv", "qknorm_mrope", "attention", "gemm_o", "gemm_up", "gemm_down"):
+    for n in ("rmsnorm", "gemm_qkv", "qknorm_mrope", "attention", "gemm_o", "gemm_up", "gemm_down"):
         assert n in names, (n, names)

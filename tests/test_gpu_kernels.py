@@ -32,7 +32,7 @@ def test_e4m3_to_bf16_every_code_bit_exact():
     assert set(oracle.bf16_to_f64(got[~fin]).tolist()) == {480.0, -480.0}
 
 
-@pytest.mark.parametrize("rows,cols", [(3, 256), (5, 4096), (2, 8200), (3, 53248)])
+@pytest.mark.parametrize("rows,cols", [(3, 256), (5, 4096), (2, 8200), (3, 53248), (2, 57344), (1, 57352)])
 @pytest.mark.parametrize("x_fmt,y_fmt", [(0, 0), (0, 1), (2, 1), (2, 0)], ids=["bf16-bf16", "bf16-f16", "f32-f16", "f32-bf16"])
 def test_rmsnorm_rows(rows, cols, x_fmt, y_fmt):
     xf = synth.normal(7, rows, (rows, cols), std=2.0)
