@@ -18,9 +18,13 @@
 // (S: 128 fp32 columns, O: hd columns); the tiles ping-pong so that the tensor core works on
 // one tile while the other tile's softmax runs:
 //     MMA issue order per key block j:  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
-//   warp 0       TMA producer: this CTA's rows of Q_A and Q_B once, then per key block its K
-//                and V halves, straight from the fused qkv buffer [B, S, 3d]; every copy
-//                completes on the leader CTA's barriers.
+// The kernel is persistent: one CTA pair per SM pair walks the work items (batch element, head,
+// 512 queries); the key/value ring and every barrier phase run on across items, the next item's
+// S MMAs are issued as soon as its Q has landed, and its first P V waits only for this pair's
+// epilogue of the previous item to have read O.
+//   warp 0       TMA producer: per item, this CTA's rows of Q_A and Q_B (once the previous item's
+//                S MMAs have read Q), then per key block its K and V halves, straight from the
+//                fused qkv buffer [B, S, 3d]; every copy completes on the leader CTA's barriers.
 //   warp 1       TMEM allocation (pair); in the leader, one lane issues the pair MMAs.
 //   warps 2..5   softmax of tile A; warps 6..9 softmax of tile B.  Thread i owns query
 //                row i of its tile (TMEM lane i), so the running max and sum are thread-local.
@@ -60,7 +64,7 @@ struct Layout {
   static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * V_BYTES;
-  static constexpr int NUM_BARS = 1 + 3 * STAGES + 6;
+  static constexpr int NUM_BARS = 2 + 3 * STAGES + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static_assert(OFF_V % 1024 == 0 && V_BYTES % 1024 == 0, "swizzled tiles keep 1024-byte alignment");
@@ -98,8 +102,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 template <int HD, int F>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int seq, int n_heads,
-                     const int32_t* __restrict__ kv_len, const KernelGuard guard) {
+                     const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int batch, int seq,
+                     int n_heads, const int32_t* __restrict__ kv_len, const KernelGuard guard) {
   using L = Layout<HD>;
   constexpr bool kF16 = F == FMT_F16;
   extern __shared__ uint8_t smem_raw[];
@@ -108,14 +112,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* q_full = bars;               // leader: both CTAs' Q rows landed
-  uint64_t* k_full = q_full + 1;         // [STAGES] leader: both K halves of a block landed
+  uint64_t* q_full = bars;               // leader: both CTAs' Q rows of a work item landed
+  uint64_t* q_empty = q_full + 1;        // every S MMA of a work item has read Q
+  uint64_t* k_full = q_empty + 1;        // [STAGES] leader: both K halves of a block landed
   uint64_t* v_full = k_full + STAGES;    // [STAGES] leader: both V halves landed
   uint64_t* kv_empty = v_full + STAGES;  // [STAGES] both tiles' P V of the block are done
   uint64_t* s_full = kv_empty + STAGES;  // [2 tiles] S_t(j) ready (and P V_t(j-1) done)
   uint64_t* p_full = s_full + 2;         // [2 tiles] leader: both CTAs' P_t(j) written, O_t rescaled
-  uint64_t* o_full = p_full + 2;         // both tiles' O final
-  uint64_t* drain_bar = o_full + 1;
+  uint64_t* o_full = p_full + 2;         // both tiles' O of a work item final
+  uint64_t* o_empty = o_full + 1;        // [2 tiles] leader: both CTAs' epilogue warps have read O_t
+  uint64_t* drain_bar = o_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 4);
 
@@ -123,13 +129,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int lane = static_cast<int>(lane_id());
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int q0 = (blockIdx.x >> 1) * 4 * BQ + static_cast<int>(rank) * BQ;  // tile t: rows q0 + 2 BQ t ..
-  const int head = blockIdx.y;
-  const int b = blockIdx.z;
+  // Persistent: CTA pair p takes work items p, p + pairs, ...; item i = ((b * n_heads) + head) *
+  // ntile + qt covers queries [512 qt, 512 qt + 512) of (b, head).
+  const int pair = blockIdx.x >> 1;
+  const int pairs = gridDim.x >> 1;
+  const int ntile = (seq + 4 * BQ - 1) / (4 * BQ);
+  const int items = batch * n_heads * ntile;
   const int d = n_heads * HD;
+  struct Item {
+    int b, head, q0, nkv, nb;  // q0: this CTA's first row of tile A (tile t starts at q0 + 2 BQ t)
+  };
+  auto item = [&](int i) {
+    Item it;
+    const int qt = i % ntile;
+    it.head = (i / ntile) % n_heads;
+    it.b = i / (ntile * n_heads);
+    it.q0 = qt * 4 * BQ + static_cast<int>(rank) * BQ;
+    // keys of this batch element: all of them, or its key count (clamped to [1, seq])
+    it.nkv = kv_len == nullptr ? seq : min(max(kv_len[it.b], 1), seq);
+    it.nb = (it.nkv + BKV - 1) / BKV;
+    return it;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
@@ -140,6 +164,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&p_full[t], 8);  // 4 softmax warps of the tile in each CTA
     }
     mbar_init(o_full, 1);
+    mbar_init(&o_empty[0], 8);  // 4 epilogue warps of the tile in each CTA
+    mbar_init(&o_empty[1], 8);
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -157,47 +183,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   pdl_wait_then_release();  // the setup above overlaps the previous kernel's tail
 
-  // keys of this batch element: all of them, or its key count (clamped to [1, seq])
-  const int nkv = kv_len == nullptr ? seq : min(max(kv_len[b], 1), seq);
-  const int nb = (nkv + BKV - 1) / BKV;
-
   if (warp == 0) {
-    // ---------------- TMA producer
-    if (lane == 0) {
-      if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * L::Q_TILE);
-      const uint32_t qbar = mapa_shared(smem_u32(q_full), 0);
-      for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < HD / 64; ++c)
-          tma_load_3d_pair(sQ + t * L::Q_TILE + c * L::Q_SLAB, &tm_q, qbar, head * HD + 64 * c, q0 + 2 * BQ * t, b);
-    }
-    __syncwarp();
-    int issued = 0;
-    for (int j = 0; j < nb; ++j) {
-      const int st = j % STAGES;
-      const uint32_t it = static_cast<uint32_t>(j / STAGES);
-      if (!mbar_wait(&kv_empty[st], (it & 1u) ^ 1u, guard, abort_flag,
-                     where_code(ERR_TIMEOUT_ATTN_PRODUCER, rank, j)))
+    // ---------------- TMA producer: per work item this CTA's rows of Q_A and Q_B (once the
+    // previous item's S MMAs have read Q), then its K and V halves of every key block, through
+    // the key/value ring that runs on across items
+    int issued = 0;    // key blocks issued, all items
+    int q_issued = 0;  // work items whose Q load was issued
+    int ui = 0;        // work items started
+    bool ok = true;
+    for (int i = pair; i < items && ok; i += pairs, ++ui) {
+      const Item it = item(i);
+      if (ui > 0 && !mbar_wait(q_empty, static_cast<uint32_t>(ui - 1) & 1u, guard, abort_flag,
+                               where_code(ERR_TIMEOUT_ATTN_PRODUCER, rank, 0xFFFF))) {
+        ok = false;
         break;
+      }
       if (lane == 0) {
-        if (leader) {
-          mbar_arrive_expect_tx(&k_full[st], 2 * L::K_BYTES);
-          mbar_arrive_expect_tx(&v_full[st], 2 * L::V_BYTES);
-        }
-        const uint32_t kbar = mapa_shared(smem_u32(&k_full[st]), 0);
-        const uint32_t vbar = mapa_shared(smem_u32(&v_full[st]), 0);
-        for (int c = 0; c < HD / 64; ++c)
-          tma_load_3d_pair(sK + st * L::K_BYTES + c * L::K_SLAB, &tm_k, kbar, d + head * HD + 64 * c,
-                           j * BKV + 64 * static_cast<int>(rank), b);
-        tma_load_3d_pair(sV + st * L::V_BYTES, &tm_v, vbar, 2 * d + head * HD + static_cast<int>(rank) * (HD / 2),
-                         j * BKV, b);
+        if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * L::Q_TILE);
+        const uint32_t qbar = mapa_shared(smem_u32(q_full), 0);
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < HD / 64; ++c)
+            tma_load_3d_pair(sQ + t * L::Q_TILE + c * L::Q_SLAB, &tm_q, qbar, it.head * HD + 64 * c,
+                             it.q0 + 2 * BQ * t, it.b);
       }
       __syncwarp();
-      issued = j + 1;
+      ++q_issued;
+      for (int j = 0; j < it.nb; ++j) {
+        const int st = issued % STAGES;
+        const uint32_t rnd = static_cast<uint32_t>(issued / STAGES);
+        if (!mbar_wait(&kv_empty[st], (rnd & 1u) ^ 1u, guard, abort_flag,
+                       where_code(ERR_TIMEOUT_ATTN_PRODUCER, rank, issued))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          if (leader) {
+            mbar_arrive_expect_tx(&k_full[st], 2 * L::K_BYTES);
+            mbar_arrive_expect_tx(&v_full[st], 2 * L::V_BYTES);
+          }
+          const uint32_t kbar = mapa_shared(smem_u32(&k_full[st]), 0);
+          const uint32_t vbar = mapa_shared(smem_u32(&v_full[st]), 0);
+          for (int c = 0; c < HD / 64; ++c)
+            tma_load_3d_pair(sK + st * L::K_BYTES + c * L::K_SLAB, &tm_k, kbar, d + it.head * HD + 64 * c,
+                             j * BKV + 64 * static_cast<int>(rank), it.b);
+          tma_load_3d_pair(sV + st * L::V_BYTES, &tm_v, vbar,
+                           2 * d + it.head * HD + static_cast<int>(rank) * (HD / 2), j * BKV, it.b);
+        }
+        __syncwarp();
+        ++issued;
+      }
     }
     // Never leave with copies in flight: the leader's barriers count both CTAs' copies, and
-    // the peer is held by the final cluster barrier until the leader has drained.
+    // the peer is held by the final cluster barrier until the leader has drained.  At most one
+    // Q load is outstanding (each waits for the previous item's S MMAs).
     if (leader) {
-      mbar_wait(q_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_DRAIN, rank, 0), true);
+      if (q_issued > 0)
+        mbar_wait(q_full, static_cast<uint32_t>(q_issued - 1) & 1u, guard, abort_flag,
+                  where_code(ERR_TIMEOUT_ATTN_DRAIN, rank, 0), true);
       for (int st = 0; st < STAGES && st < issued; ++st) {
         const int last = st + ((issued - 1 - st) / STAGES) * STAGES;
         const uint32_t par = static_cast<uint32_t>(last / STAGES) & 1u;
@@ -210,9 +252,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (leader) {
       constexpr uint32_t idesc_s = idesc_f16kind(2 * BQ, BKV, kF16, false, false);
       constexpr uint32_t idesc_o = idesc_f16kind(2 * BQ, HD, kF16, false, true);
-      auto issue_s = [&](int t, int j) {  // S_t(j) = Q_t K_j^T into columns [256 t, 256 t + 128)
+      // g: key block index over all work items (the ring slot and the barrier phases); j: the
+      // block within the item
+      auto issue_s = [&](int t, int g) {  // S_t = Q_t K_g^T into columns [256 t, 256 t + 128)
         const uint32_t qbase = smem_u32(sQ + t * L::Q_TILE);
-        const uint32_t kbase = smem_u32(sK + (j % STAGES) * L::K_BYTES);
+        const uint32_t kbase = smem_u32(sK + (g % STAGES) * L::K_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t oq = (kk >> 2) * L::Q_SLAB + (kk & 3) * 32;
@@ -222,8 +266,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         mma_commit_pair(&s_full[t], 0x3);
       };
-      auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P from TMEM (columns [256 t, 256 t + 64))
-        const uint32_t vbase = smem_u32(sV + (j % STAGES) * L::V_BYTES);
+      auto issue_pv = [&](int t, int g, int j) {  // O_t += P_t V_g, P from TMEM (columns [256 t, 256 t + 64))
+        const uint32_t vbase = smem_u32(sV + (g % STAGES) * L::V_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint32_t a = vbase + kk * 16 * L::V_ROW;
@@ -231,46 +275,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           mma_f16kind_ts_pair(tmem + 256 * t + 128, tmem + 256 * t + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, rank, 0)) &&
-                mbar_wait(&k_full[0], 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, rank, 0));
-      if (ok) {
-        tc_fence_after();
-        if (lane == 0) {
-          issue_s(0, 0);
-          issue_s(1, 0);
-        }
-        __syncwarp();
-      }
-      for (int j = 0; j < nb && ok; ++j) {
-        const int st = j % STAGES;
-        const uint32_t par = static_cast<uint32_t>(j) & 1u;
-        const bool next = j + 1 < nb;
-        ok = mbar_wait(&v_full[st], static_cast<uint32_t>(j / STAGES) & 1u, guard, abort_flag,
-                       where_code(ERR_TIMEOUT_ATTN_MMA, 1, j)) &&
-             mbar_wait(&p_full[0], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 2, j)) &&
-             (!next || mbar_wait(&k_full[(j + 1) % STAGES], static_cast<uint32_t>((j + 1) / STAGES) & 1u, guard,
-                                 abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 3, j)));
+      bool ok = true;
+      int gb = 0;  // key blocks of the items before this one
+      int ui = 0;
+      for (int i = pair; i < items && ok; i += pairs, ++ui) {
+        const Item it = item(i);
+        const int nb = it.nb;
+        // S_A(0), S_B(0) overwrite S (and P) of the previous item only after its P V MMAs,
+        // issued before them, have read P
+        ok = mbar_wait(q_full, static_cast<uint32_t>(ui) & 1u, guard, abort_flag,
+                       where_code(ERR_TIMEOUT_ATTN_MMA, rank, 0)) &&
+             mbar_wait(&k_full[gb % STAGES], static_cast<uint32_t>(gb / STAGES) & 1u, guard, abort_flag,
+                       where_code(ERR_TIMEOUT_ATTN_MMA, rank, gb));
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
-          issue_pv(0, j);
-          if (next) issue_s(0, j + 1);  // overwrites P_A(j) only after PV_A(j) has read it (in-order issue)
+          issue_s(0, gb);
+          issue_s(1, gb);
+          if (nb == 1) mma_commit_pair(q_empty, 0x3);  // the item's last S MMAs are issued: Q free after them
         }
         __syncwarp();
-        ok = mbar_wait(&p_full[1], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 4, j));
-        if (!ok) break;
-        tc_fence_after();
-        if (lane == 0) {
-          issue_pv(1, j);
-          mma_commit_pair(&kv_empty[st], 0x3);  // K_j and V_j fully consumed by both tiles
-          if (next) issue_s(1, j + 1);
+        for (int j = 0; j < nb && ok; ++j) {
+          const int g = gb + j;
+          const int st = g % STAGES;
+          const uint32_t par = static_cast<uint32_t>(g) & 1u;
+          const bool next = j + 1 < nb;
+          // the first P V of an item overwrites O_t: both CTAs' epilogues of the previous item
+          // must have read it
+          ok = mbar_wait(&v_full[st], static_cast<uint32_t>(g / STAGES) & 1u, guard, abort_flag,
+                         where_code(ERR_TIMEOUT_ATTN_MMA, 1, g)) &&
+               mbar_wait(&p_full[0], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 2, g)) &&
+               (!next || mbar_wait(&k_full[(g + 1) % STAGES], static_cast<uint32_t>((g + 1) / STAGES) & 1u, guard,
+                                   abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 3, g))) &&
+               (j > 0 || ui == 0 ||
+                mbar_wait(&o_empty[0], static_cast<uint32_t>(ui - 1) & 1u, guard, abort_flag,
+                          where_code(ERR_TIMEOUT_ATTN_MMA, 5, g)));
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            issue_pv(0, g, j);
+            if (next) issue_s(0, g + 1);  // overwrites P_A only after P V_A has read it (in-order issue)
+          }
+          __syncwarp();
+          ok = mbar_wait(&p_full[1], par, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_MMA, 4, g)) &&
+               (j > 0 || ui == 0 ||
+                mbar_wait(&o_empty[1], static_cast<uint32_t>(ui - 1) & 1u, guard, abort_flag,
+                          where_code(ERR_TIMEOUT_ATTN_MMA, 6, g)));
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            issue_pv(1, g, j);
+            mma_commit_pair(&kv_empty[st], 0x3);  // K_g and V_g fully consumed by both tiles
+            if (next) {
+              issue_s(1, g + 1);
+              if (j + 2 == nb) mma_commit_pair(q_empty, 0x3);  // the item's last S MMAs are issued
+            }
+          }
+          __syncwarp();
         }
+        if (ok && lane == 0) mma_commit_pair(o_full, 0x3);  // this item's O final
         __syncwarp();
+        gb += nb;
       }
-      if (lane == 0) {
-        if (ok) mma_commit_pair(o_full, 0x3);
-        mma_commit_pair(drain_bar, 0x3);  // all MMAs retired before either CTA frees TMEM
-      }
+      if (lane == 0) mma_commit_pair(drain_bar, 0x3);  // all MMAs retired before either CTA frees TMEM
       __syncwarp();
     }
     mbar_wait(drain_bar, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_DRAIN, rank, 1), true);
@@ -282,17 +349,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_col = tmem + lane_off + 256 * t;
     const uint32_t o_col = s_col + 128;
-    const uint32_t pbar = mapa_shared(smem_u32(&p_full[t]), 0);
-    const float c_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
+    // log2(e) / sqrt(hd), the same fp32 quotient as dividing by the fp32 square root of hd
+    constexpr float c_log2 = 1.4426950408889634f / (HD == 128 ? 11.313708498984761f : 8.0f);
+    bool ok = true;
+    uint32_t sph = 0u;  // phase parity of s_full[t]: one phase per key block, all items
+    for (int ui = 0; pair + ui * pairs < items && ok; ++ui) {
+    int nkv, nb;
+    {
+      const Item it = item(pair + ui * pairs);
+      nkv = it.nkv;
+      nb = it.nb;
+    }
     float m_used = -INFINITY;
     float l = 0.f;
-    bool ok = true;
     for (int j = 0; j < nb; ++j) {
-      if (!mbar_wait(&s_full[t], static_cast<uint32_t>(j) & 1u, guard, abort_flag,
-                     where_code(ERR_TIMEOUT_ATTN_SOFTMAX, rank * 2 + t, j))) {
+      if (!mbar_wait(&s_full[t], sph, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_SOFTMAX, rank * 2 + t, j))) {
         ok = false;
         break;
       }
+      sph ^= 1u;
       tc_fence_after();
       const int valid = nkv - j * BKV;  // keys beyond this element's key count are masked
       const bool full = valid >= BKV;    // every block but possibly the last
@@ -384,13 +459,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(pbar);
+      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&p_full[t]), 0));
     }
-    if (ok && mbar_wait(o_full, 0u, guard, abort_flag, where_code(ERR_TIMEOUT_ATTN_SOFTMAX, 4 + rank, t))) {
+    if (!ok) break;
+    if (!mbar_wait(o_full, static_cast<uint32_t>(ui) & 1u, guard, abort_flag,
+                   where_code(ERR_TIMEOUT_ATTN_SOFTMAX, 4 + rank, t))) {
+      ok = false;
+      break;
+    }
+    {
       tc_fence_after();
+      const Item it = item(pair + ui * pairs);
       const float inv_l = 1.f / l;
-      const int row = q0 + 2 * BQ * t + r;
-      uint16_t* dst = out + (static_cast<size_t>(b) * seq + row) * d + head * HD;
+      const int row = it.q0 + 2 * BQ * t + r;
+      uint16_t* dst = out + (static_cast<size_t>(it.b) * seq + row) * d + it.head * HD;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t raw[32];
@@ -406,6 +488,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
       }
+    }
+    // O_t read: the next item's first P V may overwrite it
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&o_empty[t]), 0));
     }
   }
 
@@ -425,9 +512,16 @@ cudaError_t launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   cudaError_t e =
       cudaFuncSetAttribute(attention_kernel<HD, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(2 * ((seq + 4 * BQ - 1) / (4 * BQ)), n_heads, batch);
+  // persistent: one CTA pair per SM pair at most, each walking work items (b, head, 512 queries)
+  const long long items = static_cast<long long>(batch) * n_heads * ((seq + 4 * BQ - 1) / (4 * BQ));
+  int sms = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;
+  const long long pairs = items < sms / 2 ? items : sms / 2;
+  if (items >= (1ll << 31) || pairs < 1) return cudaErrorInvalidValue;
+  dim3 grid(static_cast<unsigned>(2 * pairs), 1, 1);
   return launch_pdl(attention_kernel<HD, F>, grid, dim3(THREADS), L::SMEM, s, tq, tk, tv,
-                    static_cast<uint16_t*>(out), seq, n_heads, kv_len, g);
+                    static_cast<uint16_t*>(out), batch, seq, n_heads, kv_len, g);
 }
 
 }  // namespace attn
