@@ -429,8 +429,11 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (h_feats, h_img, h_lat, h_vc, h_vu))
     d2h = h_out.numel() * h_out.element_size() + h_lat_out.numel() * h_lat_out.element_size()
     sets = [B0, Buffers()]
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    # host-to-device copies split over two streams (the 54.5 MB conditioning features on one, the
+    # rest on the other) so that two copy engines share them
+    s_in, s_in2, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     in_ready = [torch.cuda.Event() for _ in sets]
+    in_ready2 = [torch.cuda.Event() for _ in sets]
     out_ready = [torch.cuda.Event() for _ in sets]
     out_done = [torch.cuda.Event() for _ in sets]
 
@@ -438,14 +441,18 @@ def run_ours(args, rank, world, local_rank):
         k = i % 2
         b = sets[k]
         s_in.wait_event(out_done[k])  # step i-2 on this set is computed and copied out
+        s_in2.wait_event(out_done[k])
         with torch.cuda.stream(s_in):
             b.feats.copy_(h_feats, non_blocking=True)
+            in_ready[k].record(s_in)
+        with torch.cuda.stream(s_in2):
             b.img_rows.copy_(h_img, non_blocking=True)
             b.lat.copy_(h_lat, non_blocking=True)
             b.vc.copy_(h_vc, non_blocking=True)
             b.vu.copy_(h_vu, non_blocking=True)
-            in_ready[k].record(s_in)
+            in_ready2[k].record(s_in2)
         stream.wait_event(in_ready[k])
+        stream.wait_event(in_ready2[k])
         step(b)
         out_ready[k].record(stream)
         s_out.wait_event(out_ready[k])
@@ -561,7 +568,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "e2e": {"value": round(s.seq * e2e_steps * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "pipeline": "two buffer sets; host-to-device and device-to-host copies on their own streams"},
+                "pipeline": "two buffer sets; host-to-device copies on two streams, device-to-host on a third"},
         "check": check,
     }
     if c2048 is not None:
