@@ -198,8 +198,8 @@ DIT_API int dit_tokens_from_latent(const float* z, const void* text, void* x, in
  * Limits and behaviour:
  *  - shapes whose dit_block_workspace_bytes() exceeds DIT_NOALLOC_SCRATCH_BYTES return
  *    DIT_ERR_UNSUPPORTED (e.g. the tiny 16 + 8x8 block fits; the 1024 px block does not);
- *  - the first call on a device looks up the array's device address with that device
- *    current; make that first call before any stream capture;
+ *  - the first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current and keeps it for later calls on that device;
  *  - all calls share the one array and it keeps the last call's contents; calls that
  *    overlap on the GPU (other streams, other threads) race on it, so serialise them. */
 DIT_API int dit_block_forward_noalloc(const dit_block_config* cfg, const dit_block_weights* w, const void* x_in,
