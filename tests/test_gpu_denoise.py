@@ -70,3 +70,41 @@ def test_denoise_zero_steps_leaves_z():
     ops.dit_denoise_steps(cfg, w, w, t, t, z, s.grid_h, s.grid_w, [], [], ws)
     torch.cuda.synchronize()
     assert np.array_equal(z.cpu().numpy(), z0)
+
+
+def test_cfg1024_step_sampled_rows():
+    """The dual-branch CFG step at 1024 px through dit_denoise_steps: the conditional block (512 text
+    + 64x64 image tokens) and a separate-weights unconditional block (32 text + the same image
+    tokens), then z + dt (g v_c + (1 - g) v_u) with g = 4, dt = -1/50 (Ideogram 4 deep dive, section
+    4-6).  The oracle computes the image rows it is asked for one by one (K and V over all tokens of
+    each branch); the update of a latent row depends only on that row of the two block outputs."""
+    sc, su = synth.C1024, synth.UNCOND1024
+    d, gh, gw = sc.d_model, sc.grid_h, sc.grid_w
+    wc = {k: v for k, v in synth.block_inputs(sc).items() if k != "x"}
+    wu = {k: v for k, v in synth.block_inputs(su).items() if k != "x"}
+    r = np.random.default_rng(70)
+    z0 = r.standard_normal((1, gh * gw, d)).astype(np.float32)
+    tc = synth.to_bf16_bits(r.standard_normal((1, sc.n_text, d)))
+    tu = synth.to_bf16_bits(r.standard_normal((1, su.n_text, d)))
+    g, dt = synth.CFG_GUIDANCE, synth.CFG_DT
+
+    cfg = ops.make_config(sc)
+    z = dev(z0)
+    ws = workspace(ops.denoise_workspace_bytes(cfg, 1, sc.n_text, su.n_text, gh, gw))
+    ops.dit_denoise_steps(cfg, [ops.make_weights({k: dev(v) for k, v in wc.items()})],
+                          [ops.make_weights({k: dev(v) for k, v in wu.items()})], dev(tc), dev(tu), z, gh, gw,
+                          [g], [dt], ws)
+    torch.cuda.synchronize()
+    got = z.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+
+    rows = np.sort(np.random.default_rng(71).choice(gh * gw, size=3, replace=False))
+    zb = oracle.f64_to_bf16_bits(z0.astype(np.float64))
+    xc = np.concatenate([tc, zb], axis=1)
+    xu = np.concatenate([tu, zb], axis=1)
+    oc = oracle.dit_block_forward(sc, wc, xc, sc.n_text, gh, gw, rows=sc.n_text + rows)
+    ou = oracle.dit_block_forward(su, wu, xu, su.n_text, gh, gw, rows=su.n_text + rows)
+    vc = oracle.f64_to_bf16_bits(oc.reshape(-1, d))
+    vu = oracle.f64_to_bf16_bits(ou.reshape(-1, d))
+    ref = oracle.euler_cfg_step(z0[0, rows].astype(np.float64), vc, vu, g, dt)
+    assert_close(got[0, rows] - z0[0, rows], ref - z0[0, rows], what="cfg1024 update on sampled rows")
