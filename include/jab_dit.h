@@ -55,7 +55,7 @@ typedef enum { DIT_FMT_BF16 = 0, DIT_FMT_F16 = 1, DIT_FMT_F32 = 2 } dit_format;
  * rope_theta: RoPE base (10000 by default); inv_freq_i = fp32(theta^(-2i/head_dim)).
  * eps: RMSNorm epsilon of every norm in the block.
  * gelu_tanh: 0 = exact erf GELU, 1 = tanh approximation.
- * Supported: d_model = n_heads * head_dim, head_dim in {64, 128}, d_model and d_mlp
+ * Supported: d_model = n_heads * head_dim <= 8192, head_dim in {64, 128}, d_model and d_mlp
  * multiples of 256. */
 typedef struct {
   int32_t d_model, n_heads, head_dim, d_mlp;

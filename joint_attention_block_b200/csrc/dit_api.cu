@@ -129,6 +129,7 @@ int check_config(const dit_block_config* c) {
   if (c->n_heads <= 0 || c->head_dim <= 0 || c->d_model != c->n_heads * c->head_dim) return DIT_ERR_INVALID_ARG;
   if (c->head_dim != 64 && c->head_dim != 128) return DIT_ERR_UNSUPPORTED;
   if (c->d_model % 256 != 0 || c->d_mlp <= 0 || c->d_mlp % 256 != 0) return DIT_ERR_UNSUPPORTED;
+  if (c->d_model > 8192) return DIT_ERR_UNSUPPORTED;  // the QK-norm kernel: one CTA of d/16 <= 512 threads per token
   if (c->rope_sections[0] < 0 || c->rope_sections[1] < 0 || c->rope_sections[2] < 0) return DIT_ERR_INVALID_ARG;
   if (c->rope_sections[0] + c->rope_sections[1] + c->rope_sections[2] != c->head_dim / 2) return DIT_ERR_INVALID_ARG;
   if (!(c->rope_theta > 0.f) || !(c->eps >= 0.f)) return DIT_ERR_INVALID_ARG;

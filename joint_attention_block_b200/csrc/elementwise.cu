@@ -487,7 +487,8 @@ cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int3
 // two sums of squares with xor-shuffles.  The CTA is a whole number of warps; lanes past the
 // last head shadow it so that the shuffles stay full.  F: storage format of the qkv buffer.
 template <int F>
-__global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int seq, int n_heads, int head_dim, RopeArgs ra,
+__global__ void __launch_bounds__(512, 2)  // <= 64 registers: four 256-thread CTAs per SM
+    qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int seq, int n_heads, int head_dim, RopeArgs ra,
                                     const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
   __shared__ float s_cos[64], s_sin[64];
   pdl_wait_then_release();
@@ -505,11 +506,11 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int seq, int n_h
   const int d = n_heads * head_dim;
   uint16_t* vq = qkv + bs * (3 * static_cast<int64_t>(d)) + h * head_dim;
   uint16_t* vk = vq + d;
-  float qa[8], qb[8], ka[8], kb[8];
-  load8<F>(vq + 8 * c, 0, qa);
-  load8<F>(vq + half + 8 * c, 0, qb);
-  load8<F>(vk + 8 * c, 0, ka);
-  load8<F>(vk + half + 8 * c, 0, kb);
+  // q and k halves stay packed (8 16-bit values per 16-byte vector) until they are used
+  const uint4 rqa = *reinterpret_cast<const uint4*>(vq + 8 * c);
+  const uint4 rqb = *reinterpret_cast<const uint4*>(vq + half + 8 * c);
+  const uint4 rka = *reinterpret_cast<const uint4*>(vk + 8 * c);
+  const uint4 rkb = *reinterpret_cast<const uint4*>(vk + half + 8 * c);
   {
     int pt = 0, ph = 0, pw = 0;
     if (ra.text_lens != nullptr) {
@@ -540,52 +541,58 @@ __global__ void qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int seq, int n_h
       s_sin[i] = sn;
     }
   }
-  __syncthreads();
-  float cs[8], sn[8];
+  auto sumsq = [](const uint4& a, const uint4& b2) {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b2.x, b2.y, b2.z, b2.w};
+    float acc = 0.f;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    cs[k] = s_cos[8 * c + k];
-    sn[k] = s_sin[8 * c + k];
-  }
-  float sq = 0.f, sk = 0.f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    sq = fmaf(qa[k], qa[k], fmaf(qb[k], qb[k], sq));
-    sk = fmaf(ka[k], ka[k], fmaf(kb[k], kb[k], sk));
-  }
+    for (int k = 0; k < 8; ++k) {
+      const float lo = unpack_lo<F>(w[k]), hi = unpack_hi<F>(w[k]);
+      acc = fmaf(lo, lo, fmaf(hi, hi, acc));
+    }
+    return acc;
+  };
+  float sq = sumsq(rqa, rqb), sk = sumsq(rka, rkb);
   for (int o = group / 2; o > 0; o >>= 1) {
     sq += __shfl_xor_sync(0xffffffffu, sq, o);
     sk += __shfl_xor_sync(0xffffffffu, sk, o);
   }
   const float rq = rsqrtf(sq / static_cast<float>(head_dim) + eps);
   const float rk = rsqrtf(sk / static_cast<float>(head_dim) + eps);
-  float ga[8], gb[8];
-  float oa[8], ob[8];
-  load8<FMT_BF16>(g_q + 8 * c, 0, ga);
-  load8<FMT_BF16>(g_q + half + 8 * c, 0, gb);
+  __syncthreads();  // the token's angles are in shared memory
+  // rotate pairs (i, i + hd/2): x1 = a * r * g_a, x2 = b * r * g_b; (x1 cos - x2 sin, x2 cos + x1 sin)
+  auto rotate = [&](const uint4& a, const uint4& b2, float rr, const uint16_t* g, uint16_t* dst) {
+    const uint4 ga4 = *reinterpret_cast<const uint4*>(g + 8 * c);
+    const uint4 gb4 = *reinterpret_cast<const uint4*>(g + half + 8 * c);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b2.x, b2.y, b2.z, b2.w};
+    const uint32_t wga[4] = {ga4.x, ga4.y, ga4.z, ga4.w}, wgb[4] = {gb4.x, gb4.y, gb4.z, gb4.w};
+    uint4 oa, ob;
+    uint32_t* poa = reinterpret_cast<uint32_t*>(&oa);
+    uint32_t* pob = reinterpret_cast<uint32_t*>(&ob);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float x1 = qa[k] * rq * ga[k];
-    const float x2 = qb[k] * rq * gb[k];
-    oa[k] = x1 * cs[k] - x2 * sn[k];
-    ob[k] = x2 * cs[k] + x1 * sn[k];
-  }
-  if (live) {
-    store8<F>(vq + 8 * c, 0, oa);
-    store8<F>(vq + half + 8 * c, 0, ob);
-  }
-  load8<FMT_BF16>(g_k + 8 * c, 0, ga);
-  load8<FMT_BF16>(g_k + half + 8 * c, 0, gb);
+    for (int k = 0; k < 4; ++k) {
+      float ra2[2], rb2[2];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float x1 = ka[k] * rk * ga[k];
-    const float x2 = kb[k] * rk * gb[k];
-    oa[k] = x1 * cs[k] - x2 * sn[k];
-    ob[k] = x2 * cs[k] + x1 * sn[k];
-  }
+      for (int e = 0; e < 2; ++e) {
+        const int i = 8 * c + 2 * k + e;
+        const float av = e ? unpack_hi<F>(wa[k]) : unpack_lo<F>(wa[k]);
+        const float bv = e ? unpack_hi<F>(wb[k]) : unpack_lo<F>(wb[k]);
+        const float gav = e ? unpack_hi<FMT_BF16>(wga[k]) : unpack_lo<FMT_BF16>(wga[k]);
+        const float gbv = e ? unpack_hi<FMT_BF16>(wgb[k]) : unpack_lo<FMT_BF16>(wgb[k]);
+        const float x1 = av * rr * gav;
+        const float x2 = bv * rr * gbv;
+        const float cs = s_cos[i], sn = s_sin[i];
+        ra2[e] = x1 * cs - x2 * sn;
+        rb2[e] = x2 * cs + x1 * sn;
+      }
+      poa[k] = pack2<F>(ra2[0], ra2[1]);
+      pob[k] = pack2<F>(rb2[0], rb2[1]);
+    }
+    *reinterpret_cast<uint4*>(dst + 8 * c) = oa;
+    *reinterpret_cast<uint4*>(dst + half + 8 * c) = ob;
+  };
   if (live) {
-    store8<F>(vk + 8 * c, 0, oa);
-    store8<F>(vk + half + 8 * c, 0, ob);
+    rotate(rqa, rqb, rq, g_q, vq);
+    rotate(rka, rkb, rk, g_k, vk);
   }
 }
 
@@ -598,7 +605,7 @@ cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_he
   if (head_dim != 64 && head_dim != 128) return cudaErrorInvalidValue;
   if ((text_lens != nullptr) != (kv_len != nullptr)) return cudaErrorInvalidValue;
   const int per_token = n_heads * (head_dim / 16);
-  if (per_token > 1024) return cudaErrorInvalidValue;
+  if (per_token > 512) return cudaErrorInvalidValue;  // the kernel's launch bound
   RopeArgs ra;
   ra.n_text = n_text;
   ra.grid_w = grid_w > 0 ? grid_w : 1;

@@ -60,6 +60,11 @@ def test_argument_validation_without_gpu(lib):
     hd96 = _abi.make_config(synth.TINY)
     hd96.head_dim, hd96.n_heads, hd96.d_model = 96, 4, 384
     assert lib.dit_block_forward(ctypes.byref(hd96), ctypes.byref(w), 16, 32, 1, 16, 8, 8, -1, None, None, 0, None) == 2
+    wide = _abi.make_config(synth.TINY)  # d_model 8448 > 8192: beyond the one-CTA-per-token QK-norm
+    wide.head_dim, wide.n_heads, wide.d_model, wide.d_mlp = 128, 66, 8448, 8448
+    wide.rope_sections[0], wide.rope_sections[1], wide.rope_sections[2] = 24, 20, 20
+    assert lib.dit_block_workspace_bytes(ctypes.byref(wide), 1, 16, 8, 8) == 0
+    assert lib.dit_block_forward(ctypes.byref(wide), ctypes.byref(w), 16, 32, 1, 16, 8, 8, -1, None, None, 0, None) == 2
     assert lib.euler_cfg_step(None, None, None, 8, 4.0, -0.02, None) == 1
     assert lib.euler_cfg_step(None, None, None, 0, 4.0, -0.02, None) == 0  # empty update: nothing to do
     assert lib.dit_gemm_w8a16(16, 0, 16, 16, 16, 0, None, 0, 128, 100, 64, 0, 0, None) == 2  # N % 32 != 0
