@@ -206,7 +206,10 @@ def test_qknorm_mrope(shape, fmt):
     assert torch.equal(qkv.view(1, S, 3, -1)[:, :, 2], before.view(1, S, 3, -1)[:, :, 2])
 
 
-@pytest.mark.parametrize("S,H,hd,batch", [(80, 4, 64, 1), (300, 2, 128, 1), (1, 2, 128, 1), (129, 1, 64, 2), (640, 2, 128, 1)])
+# (129, 160, 64, 1) and (200, 48, 128, 2): more work items (batch, head, 512 queries) than SM pairs,
+# so each persistent CTA pair walks several items, each ending in a ragged key block.
+@pytest.mark.parametrize("S,H,hd,batch", [(80, 4, 64, 1), (300, 2, 128, 1), (1, 2, 128, 1), (129, 1, 64, 2), (640, 2, 128, 1),
+                                          (129, 160, 64, 1), (200, 48, 128, 2)])
 @pytest.mark.parametrize("fmt", [0, 1], ids=["bf16", "f16"])
 def test_joint_attention(S, H, hd, batch, fmt):
     d = H * hd
