@@ -21,6 +21,8 @@ from .ideogram4 import (  # noqa: F401
     mrope,
     mrope_angles,
     mrope_positions,
+    qk_e4m3_scale,
+    quantize_qk,
     quantize_rows_act,
     rmsnorm,
 )

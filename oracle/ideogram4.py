@@ -92,6 +92,22 @@ def quantize_rows_act(h: np.ndarray):
     return e4m3_round(h / scale) * scale, scale[..., 0]
 
 
+def qk_e4m3_scale(g: np.ndarray, head_dim: int) -> float:
+    """Static e4m3 scale of the normalised, rotated q (or k) of the W8A8 variant: after the per-head
+    RMSNorm a head vector has Euclidean norm at most sqrt(hd) * max|g| (its mean square before the
+    gain is at most 1), and each rotation of a pair (i, i + hd/2) keeps that norm, so no component
+    exceeds it.  Dividing by sqrt(hd) * max|g| / 448 therefore never leaves the e4m3 range.  Each
+    step is rounded to fp32: the scale is an fp32 number the kernels share."""
+    s = np.float32(np.sqrt(np.float32(head_dim)))
+    s = np.float32(s * np.float32(np.abs(np.asarray(g, dtype=np.float64)).max()))
+    return float(np.float32(s / np.float32(448.0)))
+
+
+def quantize_qk(x: np.ndarray, scale: float) -> np.ndarray:
+    """q or k of the W8A8 variant as the attention product sees them: e4m3_round(x / scale) * scale."""
+    return e4m3_round(np.asarray(x, dtype=np.float64) / scale) * scale
+
+
 def dequant(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     """Real weight = fp8 value * weight_scale[:, None] (scale indexed by output row)."""
     return e4m3_to_f64(codes) * np.asarray(scale, dtype=np.float32).astype(np.float64)[:, None]
@@ -194,7 +210,8 @@ def dit_block_forward(
 
     ``w8a8`` quantises the inputs of the QKV and MLP-up projections (the two pre-norm outputs)
     to e4m3 per token (quantize_rows_act) before the FP8-weight products, as an FP8-activation
-    pipeline would; the other products keep 16-bit activations.
+    pipeline would, and the normalised, rotated q and k to e4m3 with one static scale each
+    (qk_e4m3_scale, quantize_qk) before q k^T; P V and the other products keep 16-bit activations.
 
     ``cfg`` carries d_model, n_heads, head_dim, d_mlp, rope_sections, rope_theta,
     eps, gelu_tanh.  ``w`` holds e4m3 codes w_qkv [3d, d], w_o [d, d], w_up [F, d],
@@ -246,6 +263,9 @@ def dit_block_forward(
         k = rmsnorm(k, gk, eps)
         q = mrope(q, pos_b[sel], cfg.rope_sections, cfg.rope_theta)
         k = mrope(k, pos_b, cfg.rope_sections, cfg.rope_theta)
+        if w8a8:
+            q = quantize_qk(q, qk_e4m3_scale(gq, hd))
+            k = quantize_qk(k, qk_e4m3_scale(gk, hd))
         o = attention(q, k, v, key_valid).reshape(len(sel), d)
         x1 = x[sel] + o @ W_o.T
         h2 = rmsnorm(x1, g2, eps)

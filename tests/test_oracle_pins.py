@@ -598,6 +598,36 @@ def test_activation_quantiser_scale_and_range():
     assert np.allclose(q2, q, rtol=0, atol=1e-12 * np.abs(q).max())  # quantised rows stay put
 
 
+def test_qk_e4m3_scale_is_reached_by_a_one_hot_head_and_never_exceeded():
+    """The static q/k scale against the closed-form bound it rests on: a head vector with all its
+    energy in the component of the largest gain comes out of the per-head RMSNorm at sqrt(hd) times
+    that gain (up to eps), i.e. at code 448 exactly; random head vectors, rotated by M-RoPE at
+    random positions, never exceed it; and the rounding error is at most half an e4m3 step."""
+    r = np.random.default_rng(83)
+    for hd in (64, 128):
+        g_bits = synth.to_bf16_bits(1.0 + 0.05 * r.standard_normal(hd))
+        g = oracle.bf16_to_f64(g_bits)
+        s = oracle.qk_e4m3_scale(g, hd)
+        assert s == float(np.float32(np.float32(np.sqrt(np.float32(hd)) * np.float32(np.abs(g).max())) / np.float32(448)))
+        i = int(np.argmax(np.abs(g)))
+        x = np.zeros((1, 1, hd))
+        x[0, 0, i] = 1000.0  # eps negligible against mean(x^2) = 1e6 / hd
+        xn = oracle.rmsnorm(x, g, 1e-6)
+        assert abs(abs(xn[0, 0, i]) - np.sqrt(hd) * np.abs(g).max()) < 1e-8
+        assert abs(oracle.quantize_qk(xn, s)[0, 0, i]) / s == 448.0
+        secs = (8, 12, 12) if hd == 64 else (24, 20, 20)
+        xs = r.standard_normal((200, 3, hd)) * np.exp(r.uniform(-3, 3, (200, 3, 1)))
+        xs[:, 0, :] = 0.0
+        xs[:, 0, r.integers(0, hd, 200)] = 1.0  # some one-hot heads among them
+        pos = r.integers(0, 4096, (200, 3))
+        y = oracle.mrope(oracle.rmsnorm(xs, g, 1e-6), pos, secs, 1e4)
+        assert np.abs(y).max() / s <= 448.0 * (1 + 1e-9)
+        qy = oracle.quantize_qk(y, s)
+        mag = np.abs(y) / s
+        bound = np.maximum(np.exp2(np.floor(np.log2(np.maximum(mag, 2.0 ** -6))) - 4.0), 2.0 ** -10)
+        assert np.all(np.abs(qy - y) / s <= bound * (1 + 1e-9))
+
+
 def test_w8a8_block_is_the_block_with_quantised_norm_outputs():
     """The W8A8 block differs from the W8A16 block only through the two quantised inputs: with the
     attention and MLP output projections zeroed both reduce to the residual path exactly, and with
