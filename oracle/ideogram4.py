@@ -211,7 +211,8 @@ def dit_block_forward(
     ``w8a8`` quantises the inputs of the QKV and MLP-up projections (the two pre-norm outputs)
     to e4m3 per token (quantize_rows_act) before the FP8-weight products, as an FP8-activation
     pipeline would, and the normalised, rotated q and k to e4m3 with one static scale each
-    (qk_e4m3_scale, quantize_qk) before q k^T; P V and the other products keep 16-bit activations.
+    (qk_e4m3_scale, quantize_qk) before q k^T, taken from q and k as the QKV product stores them
+    (f16); P V and the other products keep 16-bit activations.
 
     ``cfg`` carries d_model, n_heads, head_dim, d_mlp, rope_sections, rope_theta,
     eps, gelu_tanh.  ``w`` holds e4m3 codes w_qkv [3d, d], w_o [d, d], w_up [F, d],
@@ -259,6 +260,11 @@ def dit_block_forward(
         k = (h @ W_qkv[d : 2 * d].T).reshape(S, nh, hd)
         v = (h @ W_qkv[2 * d :].T).reshape(S, nh, hd)
         q = (h[sel] @ W_qkv[:d].T).reshape(len(sel), nh, hd)
+        if w8a8:
+            # the variant rounds q and k to e4m3 after the QK-norm; it takes them from the
+            # 16-bit (f16, round to nearest even) values its QKV product stores
+            q = q.astype(np.float16).astype(np.float64)
+            k = k.astype(np.float16).astype(np.float64)
         q = rmsnorm(q, gq, eps)
         k = rmsnorm(k, gk, eps)
         q = mrope(q, pos_b[sel], cfg.rope_sections, cfg.rope_theta)
