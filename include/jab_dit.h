@@ -120,8 +120,9 @@ DIT_API int dit_block_forward_padded(const dit_block_config* cfg, const dit_bloc
 /* The W8A8 variant of dit_block_forward: the inputs of the QKV and MLP-up projections (the two
  * pre-norm outputs) are quantised to e4m3 per token (scale = amax of the row / 448, codes rounded
  * to nearest even, saturating) and multiplied with the e4m3 weights on the FP8 tensor-core path
- * (tcgen05 kind::f8f6f4, twice the 16-bit rate).  The attention, output and MLP-down products keep
- * 16-bit activations.  The pages run the dequantised model with 16-bit activations; this variant
+ * (tcgen05 kind::f8f6f4, twice the 16-bit rate).  The normalised, rotated q and k are rounded to
+ * e4m3 as well, with one static scale each (see dit_qknorm_mrope_e4m3), for q k^T on the same
+ * path; P V, the output and the MLP-down products keep 16-bit activations.  The pages run the dequantised model with 16-bit activations; this variant
  * trades accuracy for speed (FP8 training through fp8-torchao is what SimpleTuner's quickstart,
  * "ハードウェアと精度", uses); its error against the 16-bit pipeline is a few per cent per element.
  * Arguments, workspace and errors as dit_block_forward; UNSUPPORTED for d_model > 8192. */
@@ -273,6 +274,27 @@ DIT_API int dit_rmsnorm_rows_e4m3(const void* x, int x_fmt, const void* g, uint8
 DIT_API int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int grid_w, int t_img, const int32_t* pos,
                      const dit_block_config* cfg, const void* g_q, const void* g_k, void* workspace,
                      size_t ws_bytes, void* stream);
+
+/* The W8A8 variant's q and k (FP8 format: unsloth diffusion_ideogram4.py commit log, fp8 loader
+ * commit; QK-RMSNorm and M-RoPE: Ideogram 4.0 announcement thread): per-head QK-RMSNorm + 3D
+ * M-RoPE of the fused qkv buffer exactly as dit_qknorm_mrope computes them, written as e4m3
+ * codes instead of back into qkv (qkv is only read).  scale[0] (q) and scale[1] (k) =
+ * fp32(fp32(sqrt(hd)) * max|g|) / 448 with g = g_q or g_k: a normalised head vector's norm is at
+ * most sqrt(hd) * max|g| and the rotations keep it, so no code saturates.  q8, k8: [batch, S, d]
+ * bytes, codes of value * fp32(1 / scale) rounded to nearest even; 16-byte aligned, caller-owned
+ * device memory; scale: fp32 [2] on the device.  Other arguments and errors as dit_qknorm_mrope. */
+DIT_API int dit_qknorm_mrope_e4m3(const void* qkv, int fmt, int batch, int n_text, int grid_h, int grid_w, int t_img,
+                                  const int32_t* pos, const dit_block_config* cfg, const void* g_q, const void* g_k,
+                                  uint8_t* q8, uint8_t* k8, float* scale, void* stream);
+
+/* Joint attention with e4m3 q and k (Ideogram 4 deep dive, section 4-2: one sequence, one
+ * bidirectional self-attention): out = softmax(scale[0] scale[1] (q8 k8^T) / sqrt(hd)) v per head,
+ * q8 k8^T accumulated in fp32 from the codes on the FP8 tensor-core path, v and P V in fmt (BF16
+ * or F16) from the fused qkv buffer [batch, S, 3d] (columns [2d, 3d)).  q8, k8: [batch, S, d]
+ * bytes (16-byte aligned); scale: fp32 [2] on the device; out: [batch, S, d] in fmt.  Errors as
+ * dit_joint_attention. */
+DIT_API int dit_joint_attention_e4m3(const uint8_t* q8, const uint8_t* k8, const float* scale, const void* qkv,
+                                     void* out, int fmt, int batch, int seq, int n_heads, int head_dim, void* stream);
 
 /* Joint bidirectional attention: out[b, s, h*hd:(h+1)*hd] = softmax(q k^T / sqrt(hd)) v
  * over all S tokens, per head, reading q, k, v from a fused qkv buffer [batch, S, 3d] in

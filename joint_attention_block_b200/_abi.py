@@ -93,6 +93,9 @@ SIGNATURES = {
     "dit_gemm_w8a16": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P]),
     "dit_qknorm_mrope": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(BlockConfig), _P, _P, _P, _SZ, _P]),
     "dit_joint_attention": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
+    "dit_qknorm_mrope_e4m3": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(BlockConfig), _P, _P, _P, _P, _P,
+                                   _P]),
+    "dit_joint_attention_e4m3": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "dit_poll_error": (_I, [_P]),
     "dit_profile_enable": (_I, [_I]),
     "dit_profile_enable_tags": (_I, [_I, ctypes.c_uint32]),
@@ -337,6 +340,21 @@ def joint_attention(qkv: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim
                     stream=None) -> None:
     _check("dit_joint_attention", lib().dit_joint_attention(_ptr(qkv), _ptr(out), fmt, qkv.shape[0], qkv.shape[1],
                                                             n_heads, head_dim, _stream(stream)))
+
+
+def qknorm_mrope_e4m3(qkv: torch.Tensor, cfg: BlockConfig, n_text: int, grid_h: int, grid_w: int, g_q: torch.Tensor,
+                      g_k: torch.Tensor, q8: torch.Tensor, k8: torch.Tensor, scale: torch.Tensor, t_img: int = -1,
+                      pos: Optional[torch.Tensor] = None, fmt: int = FMT_BF16, stream=None) -> None:
+    _check("dit_qknorm_mrope_e4m3", lib().dit_qknorm_mrope_e4m3(
+        _ptr(qkv), fmt, qkv.shape[0], n_text, grid_h, grid_w, t_img, _ptr(pos), ctypes.byref(cfg), _ptr(g_q),
+        _ptr(g_k), _ptr(q8), _ptr(k8), _ptr(scale), _stream(stream)))
+
+
+def joint_attention_e4m3(q8: torch.Tensor, k8: torch.Tensor, scale: torch.Tensor, qkv: torch.Tensor, out: torch.Tensor,
+                         n_heads: int, head_dim: int, fmt: int = FMT_BF16, stream=None) -> None:
+    _check("dit_joint_attention_e4m3", lib().dit_joint_attention_e4m3(
+        _ptr(q8), _ptr(k8), _ptr(scale), _ptr(qkv), _ptr(out), fmt, qkv.shape[0], qkv.shape[1], n_heads, head_dim,
+        _stream(stream)))
 
 
 KERNEL_TAGS = {1: "rope_table", 2: "rmsnorm", 3: "gemm_qkv", 4: "qknorm_mrope", 5: "attention", 6: "gemm_o",

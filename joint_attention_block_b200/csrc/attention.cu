@@ -36,6 +36,7 @@
 //                row sum, which leaves O / l unchanged and keeps P <= 256.  At the end
 //                the same warps store O / l in the q/k/v format.
 #include "common.cuh"
+#include "qk8.h"
 
 namespace jab {
 namespace attn {
@@ -52,12 +53,14 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 // 0: every exp2 on the MUFU unit; n > 0: one key pair in n on the FMA pipe (exp2_poly).
 constexpr int POLY_EVERY = JAB_ATTN_POLY_EVERY;
 
-template <int HD>
+// Q8: q and k as e4m3 bytes (one slab of hd bytes per row: 128-byte swizzle at hd = 128, 64-byte
+// at hd = 64); otherwise 16-bit, in slabs of 64 values (128-byte rows, 128-byte swizzle).
+template <int HD, bool Q8 = false>
 struct Layout {
-  static constexpr int Q_SLAB = 128 * 128;  // 128 rows x 64 16-bit values, 128-byte swizzle
-  static constexpr int Q_TILE = (HD / 64) * Q_SLAB;
-  static constexpr int K_SLAB = 64 * 128;  // 64 keys x 64 16-bit values
-  static constexpr int K_BYTES = (HD / 64) * K_SLAB;
+  static constexpr int Q_SLAB = Q8 ? 128 * HD : 128 * 128;
+  static constexpr int Q_TILE = Q8 ? Q_SLAB : (HD / 64) * Q_SLAB;
+  static constexpr int K_SLAB = Q8 ? 64 * HD : 64 * 128;
+  static constexpr int K_BYTES = Q8 ? K_SLAB : (HD / 64) * K_SLAB;
   static constexpr int V_ROW = HD;  // bytes per key of this CTA's hd/2 value columns
   static constexpr int V_BYTES = BKV * V_ROW;
   static constexpr int OFF_Q = 0;  // [2] tiles
@@ -67,7 +70,8 @@ struct Layout {
   static constexpr int NUM_BARS = 2 + 3 * STAGES + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  static_assert(OFF_V % 1024 == 0 && V_BYTES % 1024 == 0, "swizzled tiles keep 1024-byte alignment");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && V_BYTES % 1024 == 0,
+                "swizzled tiles keep 1024-byte alignment");
 };
 
 // 2^x on the FMA pipe, for x <= 8: x = n + f with n = round(x), f in [-1/2, 1/2];
@@ -92,6 +96,17 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
+// D[tmem] (+)= A * B^T for the CTA pair, kind::f8f6f4 with e4m3 A and B (q8 k8^T).
+__device__ __forceinline__ void mma_e4m3_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // max(a, b, c) in one instruction (three-input form of max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -99,12 +114,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-template <int HD, int F>
+// Q8: tm_q / tm_k map the e4m3 q8 / k8 buffers ([B, S, d] bytes), qk_scale[0..1] their scales.
+template <int HD, int F, bool Q8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int batch, int seq,
-                     int n_heads, const int32_t* __restrict__ kv_len, const KernelGuard guard) {
-  using L = Layout<HD>;
+                     int n_heads, const int32_t* __restrict__ kv_len, const float* __restrict__ qk_scale,
+                     const KernelGuard guard) {
+  using L = Layout<HD, Q8>;
   constexpr bool kF16 = F == FMT_F16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -201,10 +218,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (lane == 0) {
         if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * L::Q_TILE);
         const uint32_t qbar = mapa_shared(smem_u32(q_full), 0);
-        for (int t = 0; t < 2; ++t)
-          for (int c = 0; c < HD / 64; ++c)
-            tma_load_3d_pair(sQ + t * L::Q_TILE + c * L::Q_SLAB, &tm_q, qbar, it.head * HD + 64 * c,
-                             it.q0 + 2 * BQ * t, it.b);
+        for (int t = 0; t < 2; ++t) {
+          if constexpr (Q8) {
+            tma_load_3d_pair(sQ + t * L::Q_TILE, &tm_q, qbar, it.head * HD, it.q0 + 2 * BQ * t, it.b);
+          } else {
+            for (int c = 0; c < HD / 64; ++c)
+              tma_load_3d_pair(sQ + t * L::Q_TILE + c * L::Q_SLAB, &tm_q, qbar, it.head * HD + 64 * c,
+                               it.q0 + 2 * BQ * t, it.b);
+          }
+        }
       }
       __syncwarp();
       ++q_issued;
@@ -223,9 +245,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           const uint32_t kbar = mapa_shared(smem_u32(&k_full[st]), 0);
           const uint32_t vbar = mapa_shared(smem_u32(&v_full[st]), 0);
-          for (int c = 0; c < HD / 64; ++c)
-            tma_load_3d_pair(sK + st * L::K_BYTES + c * L::K_SLAB, &tm_k, kbar, d + it.head * HD + 64 * c,
-                             j * BKV + 64 * static_cast<int>(rank), it.b);
+          if constexpr (Q8) {
+            tma_load_3d_pair(sK + st * L::K_BYTES, &tm_k, kbar, it.head * HD, j * BKV + 64 * static_cast<int>(rank),
+                             it.b);
+          } else {
+            for (int c = 0; c < HD / 64; ++c)
+              tma_load_3d_pair(sK + st * L::K_BYTES + c * L::K_SLAB, &tm_k, kbar, d + it.head * HD + 64 * c,
+                               j * BKV + 64 * static_cast<int>(rank), it.b);
+          }
           tma_load_3d_pair(sV + st * L::V_BYTES, &tm_v, vbar,
                            2 * d + it.head * HD + static_cast<int>(rank) * (HD / 2), j * BKV, it.b);
         }
@@ -250,19 +277,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer (leader only)
     if (leader) {
-      constexpr uint32_t idesc_s = idesc_f16kind(2 * BQ, BKV, kF16, false, false);
+      // kind::f16 for 16-bit q, k; kind::f8f6f4 (type code 0: e4m3) for Q8
+      constexpr uint32_t idesc_s = idesc_f16kind(2 * BQ, BKV, Q8 ? true : kF16, false, false);
       constexpr uint32_t idesc_o = idesc_f16kind(2 * BQ, HD, kF16, false, true);
       // g: key block index over all work items (the ring slot and the barrier phases); j: the
       // block within the item
       auto issue_s = [&](int t, int g) {  // S_t = Q_t K_g^T into columns [256 t, 256 t + 128)
         const uint32_t qbase = smem_u32(sQ + t * L::Q_TILE);
         const uint32_t kbase = smem_u32(sK + (g % STAGES) * L::K_BYTES);
+        if constexpr (Q8) {
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t oq = (kk >> 2) * L::Q_SLAB + (kk & 3) * 32;
-          const uint32_t ok_ = (kk >> 2) * L::K_SLAB + (kk & 3) * 32;
-          mma_f16kind_ss_pair(tmem + 256 * t, smem_desc_sw128(qbase + oq, 16, 1024),
-                              smem_desc_sw128(kbase + ok_, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < HD / 32; ++kk) {  // 32 e4m3 values (32 bytes) per MMA
+            const uint64_t qd = HD == 128 ? smem_desc_sw128(qbase + 32 * kk, 16, 1024) : smem_desc_sw64(qbase + 32 * kk, 16, 512);
+            const uint64_t kd = HD == 128 ? smem_desc_sw128(kbase + 32 * kk, 16, 1024) : smem_desc_sw64(kbase + 32 * kk, 16, 512);
+            mma_e4m3_ss_pair(tmem + 256 * t, qd, kd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t oq = (kk >> 2) * L::Q_SLAB + (kk & 3) * 32;
+            const uint32_t ok_ = (kk >> 2) * L::K_SLAB + (kk & 3) * 32;
+            mma_f16kind_ss_pair(tmem + 256 * t, smem_desc_sw128(qbase + oq, 16, 1024),
+                                smem_desc_sw128(kbase + ok_, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          }
         }
         mma_commit_pair(&s_full[t], 0x3);
       };
@@ -350,7 +387,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t s_col = tmem + lane_off + 256 * t;
     const uint32_t o_col = s_col + 128;
     // log2(e) / sqrt(hd), the same fp32 quotient as dividing by the fp32 square root of hd
-    constexpr float c_log2 = 1.4426950408889634f / (HD == 128 ? 11.313708498984761f : 8.0f);
+    // (Q8: times the two e4m3 scales, S being accumulated from the codes)
+    constexpr float c_log2_16 = 1.4426950408889634f / (HD == 128 ? 11.313708498984761f : 8.0f);
+    const float c_log2 = Q8 ? c_log2_16 * (qk_scale[0] * qk_scale[1]) : c_log2_16;
     bool ok = true;
     uint32_t sph = 0u;  // phase parity of s_full[t]: one phase per key block, all items
     for (int ui = 0; pair + ui * pairs < items && ok; ++ui) {
@@ -505,12 +544,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int HD, int F>
+template <int HD, int F, bool Q8 = false>
 cudaError_t launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out, int batch,
-                      int seq, int n_heads, const int32_t* kv_len, const KernelGuard& g, cudaStream_t s) {
-  using L = Layout<HD>;
+                      int seq, int n_heads, const int32_t* kv_len, const KernelGuard& g, cudaStream_t s,
+                      const float* qk_scale = nullptr) {
+  using L = Layout<HD, Q8>;
   cudaError_t e =
-      cudaFuncSetAttribute(attention_kernel<HD, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+      cudaFuncSetAttribute(attention_kernel<HD, F, Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   // persistent: one CTA pair per SM pair at most, each walking work items (b, head, 512 queries)
   const long long items = static_cast<long long>(batch) * n_heads * ((seq + 4 * BQ - 1) / (4 * BQ));
@@ -520,8 +560,8 @@ cudaError_t launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   const long long pairs = items < sms / 2 ? items : sms / 2;
   if (items >= (1ll << 31) || pairs < 1) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>(2 * pairs), 1, 1);
-  return launch_pdl(attention_kernel<HD, F>, grid, dim3(THREADS), L::SMEM, s, tq, tk, tv,
-                    static_cast<uint16_t*>(out), batch, seq, n_heads, kv_len, g);
+  return launch_pdl(attention_kernel<HD, F, Q8>, grid, dim3(THREADS), L::SMEM, s, tq, tk, tv,
+                    static_cast<uint16_t*>(out), batch, seq, n_heads, kv_len, qk_scale, g);
 }
 
 }  // namespace attn
@@ -552,4 +592,34 @@ cudaError_t launch_attention(const void* qkv, void* out, int fmt, int batch, int
                         : attn::launch_hd<64, FMT_BF16>(tq, tk, tv, out, batch, seq, n_heads, kv_len, g, s);
 }
 
+
+cudaError_t launch_attention_q8(const uint8_t* q8, const uint8_t* k8, const float* scale, const void* qkv, void* out,
+                                int fmt, int batch, int seq, int n_heads, int head_dim, const int32_t* kv_len,
+                                const KernelGuard& g, cudaStream_t s) {
+  if (batch <= 0 || seq <= 0) return cudaSuccess;
+  if (fmt != FMT_BF16 && fmt != FMT_F16) return cudaErrorInvalidValue;
+  if (head_dim != 64 && head_dim != 128) return cudaErrorInvalidValue;
+  if (q8 == nullptr || k8 == nullptr || scale == nullptr) return cudaErrorInvalidValue;
+  const int d = n_heads * head_dim;
+  const CUtensorMapDataType dt = fmt == FMT_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // e4m3 q and k: [B, S, d] bytes, one box of hd bytes per row (x = head * hd, a multiple of 64)
+  const uint64_t dims8[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(seq), static_cast<uint64_t>(batch)};
+  const uint64_t strides8[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(seq) * d};
+  const uint64_t dims[3] = {static_cast<uint64_t>(3 * d), static_cast<uint64_t>(seq), static_cast<uint64_t>(batch)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(3 * d) * 2, static_cast<uint64_t>(seq) * 3 * d * 2};
+  CUtensorMap tq, tk, tv;
+  const uint32_t box_q[3] = {static_cast<uint32_t>(head_dim), attn::BQ, 1};
+  const uint32_t box_k[3] = {static_cast<uint32_t>(head_dim), attn::BKV / 2, 1};
+  const uint32_t box_v[3] = {static_cast<uint32_t>(head_dim / 2), attn::BKV, 1};
+  const CUtensorMapSwizzle swz = head_dim == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(q8), dims8, strides8, box_q, swz) ||
+      !make_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(k8), dims8, strides8, box_k, swz) ||
+      !make_tmap(&tv, dt, 3, const_cast<void*>(qkv), dims, strides, box_v, swz))
+    return cudaErrorInvalidValue;
+  if (head_dim == 128)
+    return fmt == FMT_F16 ? attn::launch_hd<128, FMT_F16, true>(tq, tk, tv, out, batch, seq, n_heads, kv_len, g, s, scale)
+                          : attn::launch_hd<128, FMT_BF16, true>(tq, tk, tv, out, batch, seq, n_heads, kv_len, g, s, scale);
+  return fmt == FMT_F16 ? attn::launch_hd<64, FMT_F16, true>(tq, tk, tv, out, batch, seq, n_heads, kv_len, g, s, scale)
+                        : attn::launch_hd<64, FMT_BF16, true>(tq, tk, tv, out, batch, seq, n_heads, kv_len, g, s, scale);
+}
 }  // namespace jab

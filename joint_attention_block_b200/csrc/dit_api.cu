@@ -9,6 +9,7 @@
 
 #include "jab_dit.h"
 #include "internal.h"
+#include "qk8.h"
 
 namespace jab {
 
@@ -148,6 +149,7 @@ struct BlockWorkspace {
   float* x1;
   uint16_t* u;
   float* sa;  // per-token e4m3 scales of the W8A8 variant (its e4m3 codes reuse h)
+  float* qk8_scale;  // W8A8: the static e4m3 scales of q and k (their codes reuse h after the QKV GEMM)
   size_t bytes;
 };
 
@@ -163,7 +165,7 @@ BlockWorkspace carve_block(const dit_block_config* c, int batch, int seq, void* 
   };
   const size_t o_kv = take(static_cast<size_t>(batch) * 4);
   const size_t o_h = take(M * d * 2), o_qkv = take(M * 3 * d * 2), o_o = take(M * d * 2), o_x1 = take(M * d * 4);
-  const size_t o_u = take(M * F * 2), o_sa = take(M * 4);
+  const size_t o_u = take(M * F * 2), o_sa = take(M * 4), o_qs = take(2 * 4);
   w.bytes = off;
   if (base != nullptr) {
     uint8_t* b = static_cast<uint8_t*>(base);
@@ -174,6 +176,7 @@ BlockWorkspace carve_block(const dit_block_config* c, int batch, int seq, void* 
     w.x1 = reinterpret_cast<float*>(b + o_x1);
     w.u = reinterpret_cast<uint16_t*>(b + o_u);
     w.sa = reinterpret_cast<float*>(b + o_sa);
+    w.qk8_scale = reinterpret_cast<float*>(b + o_qs);
   }
   return w;
 }
@@ -363,6 +366,44 @@ int dit_qknorm_mrope(void* qkv, int fmt, int batch, int n_text, int grid_h, int 
   return from_cuda(e);
 }
 
+int dit_qknorm_mrope_e4m3(const void* qkv, int fmt, int batch, int n_text, int grid_h, int grid_w, int t_img,
+                          const int32_t* pos, const dit_block_config* cfg, const void* g_q, const void* g_k,
+                          uint8_t* q8, uint8_t* k8, float* scale, void* stream) {
+  clear_stale_error();
+  int st = check_config(cfg);
+  if (st != DIT_OK) return st;
+  if (!shape_ok(batch, n_text, grid_h, grid_w) || qkv == nullptr || g_q == nullptr || g_k == nullptr ||
+      q8 == nullptr || k8 == nullptr || scale == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  if (fmt != FMT_BF16 && fmt != FMT_F16) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(qkv) || !aligned16(q8) || !aligned16(k8)) return DIT_ERR_INVALID_ARG;
+  const int S = n_text + grid_h * grid_w;
+  cudaStream_t s = as_stream(stream);
+  const QK8Out o8{q8, k8, scale};
+  prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
+  cudaError_t e = launch_qknorm_mrope_e4m3(qkv, fmt, batch, S, cfg->n_heads, cfg->head_dim, n_text, grid_w,
+                                           grid_h * grid_w, t_img, pos, nullptr, nullptr, cfg->rope_sections,
+                                           cfg->rope_theta, static_cast<const uint16_t*>(g_q),
+                                           static_cast<const uint16_t*>(g_k), cfg->eps, o8, s);
+  prof_mark(s, DIT_KERNEL_END);
+  return from_cuda(e);
+}
+
+int dit_joint_attention_e4m3(const uint8_t* q8, const uint8_t* k8, const float* scale, const void* qkv, void* out,
+                             int fmt, int batch, int seq, int n_heads, int head_dim, void* stream) {
+  clear_stale_error();
+  if (batch <= 0 || seq <= 0 || n_heads <= 0 || qkv == nullptr || out == nullptr || q8 == nullptr ||
+      k8 == nullptr || scale == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  if (fmt != FMT_BF16 && fmt != FMT_F16) return DIT_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return DIT_ERR_UNSUPPORTED;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(q8) || !aligned16(k8)) return DIT_ERR_INVALID_ARG;
+  KernelGuard g;
+  if (current_guard(&g) != cudaSuccess) return DIT_ERR_CUDA;
+  return from_cuda(
+      launch_attention_q8(q8, k8, scale, qkv, out, fmt, batch, seq, n_heads, head_dim, nullptr, g, as_stream(stream)));
+}
+
 int dit_joint_attention(const void* qkv, void* out, int fmt, int batch, int seq, int n_heads, int head_dim,
                         void* stream) {
   clear_stale_error();
@@ -434,13 +475,26 @@ int block_forward(const dit_block_config* cfg, const dit_block_weights* w, const
     JAB_TRY(launch_gemm_w8a16(
         GemmArgs{ws.h, FMT_F16, w->w_qkv, w->s_qkv, ws.qkv, FMT_F16, nullptr, -1, M, 3 * d, d, 0, 0}, g, s));
   prof_mark(s, DIT_KERNEL_QKNORM_MROPE);
-  JAB_TRY(launch_qknorm_mrope(ws.qkv, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, n_text, grid_w,
-                              grid_h * grid_w, t_img, pos, text_lens, padded ? ws.kv_len : nullptr,
-                              cfg->rope_sections, cfg->rope_theta, static_cast<const uint16_t*>(w->g_q),
-                              static_cast<const uint16_t*>(w->g_k), cfg->eps, s));
+  // W8A8: q and k as e4m3 codes over h (free once the QKV GEMM has read it): q8 = h[0, M d),
+  // k8 = h[M d, 2 M d) bytes
+  const QK8Out o8{h8, h8 + static_cast<size_t>(M) * d, ws.qk8_scale};
+  if (w8a8)
+    JAB_TRY(launch_qknorm_mrope_e4m3(ws.qkv, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, n_text, grid_w,
+                                     grid_h * grid_w, t_img, pos, text_lens, padded ? ws.kv_len : nullptr,
+                                     cfg->rope_sections, cfg->rope_theta, static_cast<const uint16_t*>(w->g_q),
+                                     static_cast<const uint16_t*>(w->g_k), cfg->eps, o8, s));
+  else
+    JAB_TRY(launch_qknorm_mrope(ws.qkv, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, n_text, grid_w,
+                                grid_h * grid_w, t_img, pos, text_lens, padded ? ws.kv_len : nullptr,
+                                cfg->rope_sections, cfg->rope_theta, static_cast<const uint16_t*>(w->g_q),
+                                static_cast<const uint16_t*>(w->g_k), cfg->eps, s));
   prof_mark(s, DIT_KERNEL_ATTENTION);
-  JAB_TRY(launch_attention(ws.qkv, ws.o, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim, padded ? ws.kv_len : nullptr,
-                           g, s));
+  if (w8a8)
+    JAB_TRY(launch_attention_q8(o8.q8, o8.k8, o8.scale, ws.qkv, ws.o, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim,
+                                padded ? ws.kv_len : nullptr, g, s));
+  else
+    JAB_TRY(launch_attention(ws.qkv, ws.o, FMT_F16, batch, S, cfg->n_heads, cfg->head_dim,
+                             padded ? ws.kv_len : nullptr, g, s));
   prof_mark(s, DIT_KERNEL_GEMM_O);
   JAB_TRY(launch_gemm_w8a16(GemmArgs{ws.o, FMT_F16, w->w_o, w->s_o, ws.x1, FMT_F32, x, FMT_BF16, M, d, d, 0, 0}, g, s));
   prof_mark(s, DIT_KERNEL_RMSNORM);

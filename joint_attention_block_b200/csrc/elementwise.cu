@@ -5,6 +5,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "qk8.h"
 
 namespace jab {
 
@@ -486,10 +487,15 @@ cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int3
 // angles are computed), so the hd/16 threads of one head are consecutive lanes and reduce the
 // two sums of squares with xor-shuffles.  The CTA is a whole number of warps; lanes past the
 // last head shadow it so that the shuffles stay full.  F: storage format of the qkv buffer.
-template <int F>
-__global__ void __launch_bounds__(512, 2)  // <= 64 registers: four 256-thread CTAs per SM
+// Q8 (the W8A8 variant): q and k are not written back; their e4m3 codes go to o8.q8 / o8.k8
+// ([B * S, d] bytes), each divided by one static scale, fp32(fp32(sqrt(hd)) * max|g|) / 448 (the
+// norm of a normalised head vector is at most sqrt(hd) * max|g| and the rotations keep it, so no
+// code saturates), which the CTA of token 0 also stores in o8.scale[0] (q) and [1] (k).
+template <int F, bool Q8>
+__global__ void __launch_bounds__(512, Q8 ? 1 : 2)  // 16-bit: <= 64 registers, four 256-thread CTAs per SM
     qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int seq, int n_heads, int head_dim, RopeArgs ra,
-                                    const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps) {
+                                    const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps,
+                                    QK8Out o8) {
   __shared__ float s_cos[64], s_sin[64];
   pdl_wait_then_release();
   const int half = head_dim / 2;
@@ -590,16 +596,76 @@ __global__ void __launch_bounds__(512, 2)  // <= 64 registers: four 256-thread C
     *reinterpret_cast<uint4*>(dst + 8 * c) = oa;
     *reinterpret_cast<uint4*>(dst + half + 8 * c) = ob;
   };
-  if (live) {
-    rotate(rqa, rqb, rq, g_q, vq);
-    rotate(rka, rkb, rk, g_k, vk);
+  if constexpr (!Q8) {
+    if (live) {
+      rotate(rqa, rqb, rq, g_q, vq);
+      rotate(rka, rkb, rk, g_k, vk);
+    }
+  } else {
+    // max |g| over the head: each thread's 16 gains, then the group's xor-shuffle maximum
+    auto gmax16 = [&](const uint16_t* g) {
+      const uint4 a4 = *reinterpret_cast<const uint4*>(g + 8 * c);
+      const uint4 b4 = *reinterpret_cast<const uint4*>(g + half + 8 * c);
+      const uint32_t w[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        m = fmaxf(m, fmaxf(fabsf(unpack_lo<FMT_BF16>(w[k])), fabsf(unpack_hi<FMT_BF16>(w[k]))));
+      for (int o = group / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      return m;
+    };
+    const float root = __fsqrt_rn(static_cast<float>(head_dim));
+    const float sc_q = __fdiv_rn(__fmul_rn(root, gmax16(g_q)), 448.f);
+    const float sc_k = __fdiv_rn(__fmul_rn(root, gmax16(g_k)), 448.f);
+    if (bs == 0 && threadIdx.x == 0) {
+      o8.scale[0] = sc_q;
+      o8.scale[1] = sc_k;
+    }
+    // the same rotation as above, then e4m3 codes of value * fp32(1 / scale) (8 bytes per half)
+    auto rotate8 = [&](const uint4& a, const uint4& b2, float rr, const uint16_t* g, float inv, uint8_t* dst) {
+      const uint4 ga4 = *reinterpret_cast<const uint4*>(g + 8 * c);
+      const uint4 gb4 = *reinterpret_cast<const uint4*>(g + half + 8 * c);
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b2.x, b2.y, b2.z, b2.w};
+      const uint32_t wga[4] = {ga4.x, ga4.y, ga4.z, ga4.w}, wgb[4] = {gb4.x, gb4.y, gb4.z, gb4.w};
+      uint16_t ca[4], cb[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float ra2[2], rb2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 8 * c + 2 * k + e;
+          const float av = e ? unpack_hi<F>(wa[k]) : unpack_lo<F>(wa[k]);
+          const float bv = e ? unpack_hi<F>(wb[k]) : unpack_lo<F>(wb[k]);
+          const float gav = e ? unpack_hi<FMT_BF16>(wga[k]) : unpack_lo<FMT_BF16>(wga[k]);
+          const float gbv = e ? unpack_hi<FMT_BF16>(wgb[k]) : unpack_lo<FMT_BF16>(wgb[k]);
+          const float x1 = av * rr * gav;
+          const float x2 = bv * rr * gbv;
+          const float cs = s_cos[i], sn = s_sin[i];
+          ra2[e] = (x1 * cs - x2 * sn) * inv;
+          rb2[e] = (x2 * cs + x1 * sn) * inv;
+        }
+        ca[k] = pack_e4m3x2(ra2[0], ra2[1]);
+        cb[k] = pack_e4m3x2(rb2[0], rb2[1]);
+      }
+      *reinterpret_cast<uint2*>(dst + 8 * c) =
+          make_uint2(ca[0] | (static_cast<uint32_t>(ca[1]) << 16), ca[2] | (static_cast<uint32_t>(ca[3]) << 16));
+      *reinterpret_cast<uint2*>(dst + half + 8 * c) =
+          make_uint2(cb[0] | (static_cast<uint32_t>(cb[1]) << 16), cb[2] | (static_cast<uint32_t>(cb[3]) << 16));
+    };
+    if (live) {
+      const int64_t row = bs * static_cast<int64_t>(d) + h * head_dim;
+      rotate8(rqa, rqb, rq, g_q, __fdiv_rn(1.f, sc_q), o8.q8 + row);
+      rotate8(rka, rkb, rk, g_k, __fdiv_rn(1.f, sc_k), o8.k8 + row);
+    }
   }
 }
 
-cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim, int n_text,
-                                int grid_w, int n_img, int t_img, const int32_t* pos, const int32_t* text_lens,
-                                int32_t* kv_len, const int32_t sections[3], float theta, const uint16_t* g_q,
-                                const uint16_t* g_k, float eps, cudaStream_t s) {
+namespace {
+
+cudaError_t qknorm_mrope_impl(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim, int n_text,
+                              int grid_w, int n_img, int t_img, const int32_t* pos, const int32_t* text_lens,
+                              int32_t* kv_len, const int32_t sections[3], float theta, const uint16_t* g_q,
+                              const uint16_t* g_k, float eps, cudaStream_t s, const QK8Out* o8) {
   const int64_t tokens = static_cast<int64_t>(batch) * seq;
   if (tokens <= 0 || n_heads <= 0) return cudaSuccess;
   if (head_dim != 64 && head_dim != 128) return cudaErrorInvalidValue;
@@ -621,15 +687,49 @@ cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_he
   const unsigned threads = static_cast<unsigned>((per_token + 31) / 32 * 32);
   const unsigned blocks = static_cast<unsigned>(tokens);
   uint16_t* q = static_cast<uint16_t*>(qkv);
+  if (o8 != nullptr) {
+    if (o8->q8 == nullptr || o8->k8 == nullptr || o8->scale == nullptr) return cudaErrorInvalidValue;
+    if (((reinterpret_cast<uintptr_t>(o8->q8) | reinterpret_cast<uintptr_t>(o8->k8)) & 15u) != 0)
+      return cudaErrorInvalidValue;
+    if (fmt == FMT_F16)
+      launch_pdl(qknorm_mrope_kernel<FMT_F16, true>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra,
+                 g_q, g_k, eps, *o8);
+    else if (fmt == FMT_BF16)
+      launch_pdl(qknorm_mrope_kernel<FMT_BF16, true>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra,
+                 g_q, g_k, eps, *o8);
+    else
+      return cudaErrorInvalidValue;
+    return cudaGetLastError();
+  }
+  const QK8Out none{nullptr, nullptr, nullptr};
   if (fmt == FMT_F16)
-    launch_pdl(qknorm_mrope_kernel<FMT_F16>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra, g_q,
-               g_k, eps);
+    launch_pdl(qknorm_mrope_kernel<FMT_F16, false>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra,
+               g_q, g_k, eps, none);
   else if (fmt == FMT_BF16)
-    launch_pdl(qknorm_mrope_kernel<FMT_BF16>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra, g_q,
-               g_k, eps);
+    launch_pdl(qknorm_mrope_kernel<FMT_BF16, false>, dim3(blocks), dim3(threads), 0, s, q, seq, n_heads, head_dim, ra,
+               g_q, g_k, eps, none);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_qknorm_mrope(void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim, int n_text,
+                                int grid_w, int n_img, int t_img, const int32_t* pos, const int32_t* text_lens,
+                                int32_t* kv_len, const int32_t sections[3], float theta, const uint16_t* g_q,
+                                const uint16_t* g_k, float eps, cudaStream_t s) {
+  return qknorm_mrope_impl(qkv, fmt, batch, seq, n_heads, head_dim, n_text, grid_w, n_img, t_img, pos, text_lens,
+                           kv_len, sections, theta, g_q, g_k, eps, s, nullptr);
+}
+
+cudaError_t launch_qknorm_mrope_e4m3(const void* qkv, int fmt, int batch, int seq, int n_heads, int head_dim,
+                                     int n_text, int grid_w, int n_img, int t_img, const int32_t* pos,
+                                     const int32_t* text_lens, int32_t* kv_len, const int32_t sections[3], float theta,
+                                     const uint16_t* g_q, const uint16_t* g_k, float eps, const QK8Out& o8,
+                                     cudaStream_t s) {
+  return qknorm_mrope_impl(const_cast<void*>(qkv), fmt, batch, seq, n_heads, head_dim, n_text, grid_w, n_img, t_img,
+                           pos, text_lens, kv_len, sections, theta, g_q, g_k, eps, s, &o8);
 }
 
 // ------------------------------------------------------------------ bounded-wait self test

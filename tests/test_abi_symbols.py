@@ -76,6 +76,11 @@ def test_argument_validation_without_gpu(lib):
     assert lib.dit_rmsnorm_rows(16, 0, 16, 16, 1, 4, 16, 1e-6, None) == 1  # in place with a format change
     assert lib.dit_joint_attention(16, 32, 2, 1, 8, 2, 64, None) == 1  # fp32 q/k/v
     assert lib.dit_joint_attention(16, 32, 1, 1, 8, 2, 96, None) == 2  # head_dim 96
+    assert lib.dit_joint_attention_e4m3(16, 16, 16, 16, 32, 1, 1, 8, 2, 96, None) == 2  # head_dim 96
+    assert lib.dit_joint_attention_e4m3(None, 16, 16, 16, 32, 1, 1, 8, 2, 64, None) == 1  # no q8
+    assert lib.dit_joint_attention_e4m3(16, 16, 16, 16, 32, 2, 1, 8, 2, 64, None) == 1  # fp32 v
+    assert lib.dit_qknorm_mrope_e4m3(16, 1, 1, 16, 8, 8, -1, None, ctypes.byref(cfg), 16, 16, None, 16, 16,
+                                     None) == 1  # no q8
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(lib):

@@ -1,11 +1,13 @@
-"""The W8A8 variant (e4m3 activations into the QKV and MLP-up projections) against the oracle
-(needs a B200).
+"""The W8A8 variant (e4m3 activations into the QKV and MLP-up projections, e4m3 q and k into
+q k^T) against the oracle (needs a B200).
 
 The FP8 GEMM is checked on its own (e4m3 x e4m3 products are exact in fp32, so only the fp32
 accumulation differs from fp64), the RMSNorm-to-e4m3 kernel code by code (a code may differ only
 where the fp32 and fp64 quotients fall on opposite sides of a rounding tie), and the whole block
-against oracle.dit_block_forward(..., w8a8=True) at the block tolerances.  The variant's own error
-against the 16-bit pipeline is reported, not bounded by the 16-bit tolerances.
+against oracle.dit_block_forward(..., w8a8=True): at the block tolerances on the small shapes, at
+its own (mean 6e-3, reasons at the test) on the 1024 px block.  The e4m3 QK-norm is checked code by
+code and the e4m3 attention against the oracle on seeded codes.  The variant's own error against
+the 16-bit pipeline is reported, not bounded by the 16-bit tolerances.
 """
 import dataclasses
 
@@ -96,6 +98,77 @@ def test_rmsnorm_e4m3_codes_and_scales(x_fmt):
     assert np.array_equal(y8.cpu().numpy()[5], np.zeros(cols, np.uint8))
 
 
+@pytest.mark.parametrize("shape,n_text,gh,gw,batch", [(synth.TINY, 16, 8, 8, 1), (synth.TINY, 5, 7, 9, 2),
+                                                     (synth.C1024, 37, 9, 11, 1)], ids=["hd64", "hd64-b2", "hd128"])
+@pytest.mark.parametrize("fmt", [ops.FMT_BF16, ops.FMT_F16], ids=["bf16", "f16"])
+def test_qknorm_mrope_e4m3_codes_and_scales(shape, n_text, gh, gw, batch, fmt):
+    """q and k codes of the e4m3 QK-norm against the oracle's normalised, rotated q and k divided by
+    the static scale: the scales bit for bit, the codes equal except where the kernel's fp32 value
+    and the fp64 one fall on opposite sides of a rounding tie (then one step apart); qkv untouched."""
+    cfg = ops.make_config(shape)
+    S, d, H, hd = n_text + gh * gw, shape.d_model, shape.n_heads, shape.head_dim
+    r = np.random.default_rng(97)
+    vals = (r.standard_normal((batch, S, 3 * d)) * np.exp(r.uniform(-2, 2, (batch, S, 1)))).astype(np.float32)
+    if fmt == ops.FMT_BF16:
+        qkv = dev(synth.to_bf16_bits(vals))
+    else:
+        qkv = torch.from_numpy(vals.astype(np.float16)).cuda()
+    xv = (as_f64(qkv) if fmt == ops.FMT_BF16 else qkv.cpu().numpy().astype(np.float64)).reshape(batch, S, 3, H, hd)
+    gq = synth.to_bf16_bits(1 + 0.05 * r.standard_normal(hd))
+    gk = synth.to_bf16_bits(1 + 0.05 * r.standard_normal(hd))
+    before = qkv.clone()
+    q8 = torch.empty((batch, S, d), dtype=torch.uint8, device="cuda")
+    k8 = torch.empty_like(q8)
+    sc = torch.full((2,), float("nan"), dtype=torch.float32, device="cuda")
+    ops.qknorm_mrope_e4m3(qkv, cfg, n_text, gh, gw, dev(gq), dev(gk), q8, k8, sc, fmt=fmt)
+    torch.cuda.synchronize()
+    assert torch.equal(qkv, before)
+    got_sc = sc.cpu().numpy()
+    want_sc = [oracle.qk_e4m3_scale(oracle.bf16_to_f64(g), hd) for g in (gq, gk)]
+    assert got_sc.tolist() == want_sc
+    pos = oracle.mrope_positions(n_text, gh, gw)
+    for which, g, codes, s in ((0, gq, q8, want_sc[0]), (1, gk, k8, want_sc[1])):
+        ref = oracle.mrope(oracle.rmsnorm(xv[:, :, which], oracle.bf16_to_f64(g), shape.eps), pos,
+                           shape.rope_sections, shape.rope_theta)
+        want = oracle.e4m3_round(ref / s)
+        got = oracle.e4m3_to_f64(codes.cpu().numpy()).reshape(want.shape)
+        diff = got != want
+        assert diff.mean() < 1e-3, diff.mean()
+        step = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), 2.0 ** -6))) - 3.0)
+        assert np.all(np.abs(got - want)[diff] <= step[diff] * 1.0000001)
+        assert np.abs(got).max() <= 448.0
+
+
+# (129, 160, 64, 1) and (200, 48, 128, 2): more work items than SM pairs (each pair walks several).
+@pytest.mark.parametrize("S,H,hd,batch", [(80, 4, 64, 1), (300, 2, 128, 1), (1, 2, 128, 1), (129, 1, 64, 2),
+                                          (640, 2, 128, 1), (129, 160, 64, 1), (200, 48, 128, 2)])
+@pytest.mark.parametrize("fmt", [ops.FMT_BF16, ops.FMT_F16], ids=["bf16", "f16"])
+def test_joint_attention_e4m3(S, H, hd, batch, fmt):
+    """Attention with e4m3 q and k (seeded codes, static scales) and 16-bit v against the oracle's
+    attention on the decoded q and k times their scales."""
+    d = H * hd
+    r = np.random.default_rng(S * 11 + H)
+    vals = (r.standard_normal((batch, S, 3 * d)) * 1.5).astype(np.float32)
+    if fmt == ops.FMT_BF16:
+        qkv = dev(synth.to_bf16_bits(vals))
+    else:
+        qkv = torch.from_numpy(vals.astype(np.float16)).cuda()
+    v = (as_f64(qkv) if fmt == ops.FMT_BF16 else qkv.cpu().numpy().astype(np.float64)).reshape(batch, S, 3, H, hd)[:, :, 2]
+    # seeded e4m3 codes of N(0, 1) * 40 values (the range the static scale gives normalised q and k)
+    q8 = torch.from_numpy(r.standard_normal((batch, S, d)).astype(np.float32) * 40).to(torch.float8_e4m3fn).view(torch.uint8)
+    k8 = torch.from_numpy(r.standard_normal((batch, S, d)).astype(np.float32) * 40).to(torch.float8_e4m3fn).view(torch.uint8)
+    scales = np.array([0.028, 0.031], dtype=np.float32)
+    out = torch.empty((batch, S, d), dtype=torch.int16 if fmt == ops.FMT_BF16 else torch.float16, device="cuda")
+    ops.joint_attention_e4m3(q8.cuda(), k8.cuda(), torch.from_numpy(scales).cuda(), qkv, out, H, hd, fmt=fmt)
+    torch.cuda.synchronize()
+    got = (as_f64(out) if fmt == ops.FMT_BF16 else out.cpu().numpy().astype(np.float64)).reshape(batch, S, H, hd)
+    qd = oracle.e4m3_to_f64(q8.numpy()).reshape(batch, S, H, hd) * float(scales[0])
+    kd = oracle.e4m3_to_f64(k8.numpy()).reshape(batch, S, H, hd) * float(scales[1])
+    for b in range(batch):
+        ref = oracle.attention(qd[b], kd[b], v[b])
+        assert_close(got[b], ref, max_rel=2e-2, mean_rel=3e-3, what=f"e4m3 attention S={S} H={H} hd={hd}")
+
+
 def _run_w8a8(shape, inp):
     cfg = ops.make_config(shape)
     w = ops.make_weights({k: dev(v) for k, v in inp.items() if k != "x"})
@@ -127,4 +200,14 @@ def test_block_w8a8_1024px_sampled_rows():
     got = _run_w8a8(s, inp)
     rows = np.array([0, 100, s.n_text - 1, s.n_text, 2000, s.seq - 1])
     ref8 = oracle.dit_block_forward(s, inp, inp["x"], s.n_text, s.grid_h, s.grid_w, rows=rows, w8a8=True)
-    assert_close(got[:, rows], ref8, what="c1024 w8a8 sampled")
+    # The variant's own tolerance at this size (mean 6e-3 instead of 3e-3): with bf16 inputs and
+    # gains about 1.4e-4 of the per-token activation codes fall exactly on an e4m3 rounding tie,
+    # where the last bit of the fp32 scale decides (the kernel and the fp64 oracle can round
+    # either way; test_rmsnorm_e4m3_codes_and_scales allows it code by code).  Each such code moves
+    # k by one e4m3 step of one product term, and rounding k to e4m3 again turns those moves into
+    # whole-step differences in ~1.75 % of the k codes over 4608 tokens: 3.7e-3 mean-rel measured.
+    assert_close(got[:, rows], ref8, max_rel=2e-2, mean_rel=6e-3, what="c1024 w8a8 sampled")
+    ref16 = oracle.dit_block_forward(s, inp, inp["x"], s.n_text, s.grid_h, s.grid_w, rows=rows)
+    d = np.abs(got[:, rows] - ref16)
+    print(f"c1024 w8a8 vs 16-bit oracle: max-rel {d.max() / np.abs(ref16).max():.3e}, "
+          f"mean-rel {d.mean() / np.abs(ref16).mean():.3e}")
