@@ -644,7 +644,8 @@ def measure_c2048(ops, weights, dev, stream):
 
 def measure_w8a8(ops, cfg, weights, x_in, ws, dev, stream):
     """The 1024 px block through the W8A8 variant (e4m3 activations into the QKV and MLP-up
-    projections on the FP8 tensor path), same inputs and weights as the timed step."""
+    projections and e4m3 q, k into q k^T, on the FP8 tensor path), same inputs and weights as the
+    timed step."""
     import torch
 
     s = synth.C1024
@@ -666,20 +667,25 @@ def measure_w8a8(ops, cfg, weights, x_in, ws, dev, stream):
     torch.cuda.synchronize(dev)
     ms = ev0.elapsed_time(ev1) / reps
     time.sleep(1.0)
-    ops.profile_enable(64, kernels=["gemm_qkv", "gemm_up"])  # events around these two only
+    ops.profile_enable(64, kernels=["gemm_qkv", "gemm_up", "attention"])  # events around these only
     for _ in range(3):
         run()
     torch.cuda.synchronize(dev)
     ops.profile_disable()
     per = _kernel_table(ops.profile_read(64), 3)
     S, d, F = s.seq, s.d_model, s.d_mlp
-    out = {"workload": "1024 px block, W8A8 variant (e4m3 per-token activations into QKV and MLP-up)",
+    out = {"workload": "1024 px block, W8A8 variant (e4m3 per-token activations into QKV and MLP-up, "
+                       "e4m3 q and k into q k^T)",
            "ms_per_block": round(ms, 4), "tokens_per_s": round(S / (ms / 1e3), 1),
            "tflops": round(s.flops() / (ms / 1e3) / 1e12, 1), "reps": reps}
     for name, fl in (("gemm_qkv", 2.0 * S * d * 3 * d), ("gemm_up", 2.0 * S * d * F)):
         if name in per:
             cnt, t = per[name]
             out[name + "_fp8_tflops"] = round(fl * cnt / (t / 1e3) / 1e12, 1)
+    if "attention" in per:  # q k^T on the FP8 path, P V 16-bit: counted as the same 4 S^2 d FLOP
+        cnt, t = per["attention"]
+        out["attention_ms"] = round(t / cnt, 5)
+        out["attention_tflops"] = round(4.0 * S * S * d * cnt / (t / 1e3) / 1e12, 1)
     return out
 
 
