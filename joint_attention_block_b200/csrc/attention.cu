@@ -35,6 +35,10 @@
 //                by more than 2^8; until then the stale max is used for both P and the
 //                row sum, which leaves O / l unchanged and keeps P <= 256.  At the end
 //                the same warps store O / l in the q/k/v format.
+// e4m3 form (Q8, the W8A8 variant): Q and K come from separate e4m3 buffers [B, S, d] (one slab
+// of hd bytes per row), S = Q K^T is issued as kind::f8f6f4 pair MMAs (K = 32 per instruction)
+// and the two static scales of q and k multiply the softmax's log2(e)/sqrt(hd) factor; V, P and
+// P V are as above.
 #include "common.cuh"
 #include "qk8.h"
 
