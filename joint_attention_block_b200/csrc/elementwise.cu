@@ -492,11 +492,12 @@ cudaError_t launch_positions(int n_text, int grid_h, int grid_w, int t_img, int3
 // norm of a normalised head vector is at most sqrt(hd) * max|g| and the rotations keep it, so no
 // code saturates), which the CTA of token 0 also stores in o8.scale[0] (q) and [1] (k).
 template <int F, bool Q8>
-__global__ void __launch_bounds__(512, Q8 ? 1 : 2)  // 16-bit: <= 64 registers, four 256-thread CTAs per SM
+__global__ void __launch_bounds__(512, 2)  // <= 64 registers: four 256-thread CTAs per SM
     qknorm_mrope_kernel(uint16_t* __restrict__ qkv, int seq, int n_heads, int head_dim, RopeArgs ra,
                                     const uint16_t* __restrict__ g_q, const uint16_t* __restrict__ g_k, float eps,
                                     QK8Out o8) {
   __shared__ float s_cos[64], s_sin[64];
+  __shared__ float s_gmax[2];  // Q8: max |g_q|, max |g_k|
   pdl_wait_then_release();
   const int half = head_dim / 2;
   const int lg = head_dim == 128 ? 3 : 2;  // log2 of the threads per head: 8 (hd 128) or 4 (hd 64)
@@ -545,6 +546,23 @@ __global__ void __launch_bounds__(512, Q8 ? 1 : 2)  // 16-bit: <= 64 registers, 
       sincosf(r, &sn, &cs);
       s_cos[i] = cs;
       s_sin[i] = sn;
+    }
+  }
+  if constexpr (Q8) {
+    if (threadIdx.x < 32) {  // max |g| of both gains, hd <= 128 values each: four per lane
+      float mq = 0.f, mk = 0.f;
+      for (int i = static_cast<int>(threadIdx.x); i < head_dim; i += 32) {
+        mq = fmaxf(mq, fabsf(__uint_as_float(static_cast<uint32_t>(g_q[i]) << 16)));
+        mk = fmaxf(mk, fabsf(__uint_as_float(static_cast<uint32_t>(g_k[i]) << 16)));
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+        mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+      }
+      if (threadIdx.x == 0) {
+        s_gmax[0] = mq;
+        s_gmax[1] = mk;
+      }
     }
   }
   auto sumsq = [](const uint4& a, const uint4& b2) {
@@ -602,21 +620,9 @@ __global__ void __launch_bounds__(512, Q8 ? 1 : 2)  // 16-bit: <= 64 registers, 
       rotate(rka, rkb, rk, g_k, vk);
     }
   } else {
-    // max |g| over the head: each thread's 16 gains, then the group's xor-shuffle maximum
-    auto gmax16 = [&](const uint16_t* g) {
-      const uint4 a4 = *reinterpret_cast<const uint4*>(g + 8 * c);
-      const uint4 b4 = *reinterpret_cast<const uint4*>(g + half + 8 * c);
-      const uint32_t w[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
-      float m = 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        m = fmaxf(m, fmaxf(fabsf(unpack_lo<FMT_BF16>(w[k])), fabsf(unpack_hi<FMT_BF16>(w[k]))));
-      for (int o = group / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      return m;
-    };
     const float root = __fsqrt_rn(static_cast<float>(head_dim));
-    const float sc_q = __fdiv_rn(__fmul_rn(root, gmax16(g_q)), 448.f);
-    const float sc_k = __fdiv_rn(__fmul_rn(root, gmax16(g_k)), 448.f);
+    const float sc_q = __fdiv_rn(__fmul_rn(root, s_gmax[0]), 448.f);  // after the __syncthreads above
+    const float sc_k = __fdiv_rn(__fmul_rn(root, s_gmax[1]), 448.f);
     if (bs == 0 && threadIdx.x == 0) {
       o8.scale[0] = sc_q;
       o8.scale[1] = sc_k;
