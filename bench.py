@@ -268,9 +268,10 @@ def run_reference(args, rank, world):
         return
     st = oracle_state()
     # One sample step costs seconds of fp64 work (the K/V projection over all 4608 tokens
-    # dominates), so at most 18 are timed to keep the arm within a few minutes.
-    steps = max(1, min(args.steps, 18))
-    warm = min(args.warmup, 1)
+    # dominates), so at most 18 run in all (up to 3 warm-up, the rest timed) to keep the arm
+    # within a few minutes.
+    warm = min(args.warmup, 3)
+    steps = max(1, min(args.steps, 18 - warm))
     for _ in range(warm):
         oracle_sample_step(st)
     t0 = time.perf_counter()
@@ -283,7 +284,8 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": steps, "warmup": warm, "ms_per_step": dt * 1e3 / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": SAMPLE_DESC, "steps_requested": args.steps},
+        "config": {"workload": WORKLOAD, "sample": SAMPLE_DESC, "steps_requested": args.steps,
+                   "warmup_requested": args.warmup},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": SAMPLE_DESC},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
