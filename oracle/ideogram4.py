@@ -33,7 +33,9 @@ count frequency pairs and are laid out contiguously (t, then h, then w);
 (i, i + hd/2); text token j sits at (j, j, j) and image cell (r, c) at
 (t_img, r, c) with t_img = n_text; softmax scale 1/sqrt(hd); the block is
 sequential pre-norm ``x1 = x + Attn(RMSNorm(x))``, ``y = x1 + MLP(RMSNorm(x1))``
-with no biases and an exact-erf GELU MLP.
+with no biases and an exact-erf GELU MLP.  The W8A8 variant (not on the pages) rounds the two
+pre-norm outputs to e4m3 per token (scale amax / 448) and q, k (taken from their f16 storage, after
+the QK-norm and the rotations) to e4m3 with one static scale each, sqrt(hd) * max|g| / 448.
 """
 from __future__ import annotations
 
